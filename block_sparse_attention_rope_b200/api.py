@@ -1,0 +1,261 @@
+"""Python binding of liblcbsa.so (argument marshalling only).
+
+Every step of the computation runs in the CUDA library declared in
+``include/lc_bsa.h``; this module checks tensor shapes, hands raw device
+pointers and the current CUDA stream to the C ABI and turns status codes into
+exceptions.  PyTorch provides device memory and streams.  There is no CPU
+fallback: if the shared library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblcbsa.so")
+
+LC_OK, LC_ERR_INVALID_ARGUMENT, LC_ERR_UNSUPPORTED, LC_ERR_CUDA = 0, 1, 2, 3
+LC_ERR_OUT_OF_MEMORY, LC_ERR_TIMEOUT, LC_ERR_DEVICE_CHECK = 4, 5, 6
+LC_DTYPE_BF16, LC_DTYPE_F32 = 0, 1
+
+
+class LcError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("num_q_blocks", ctypes.c_int), ("num_cond_blocks", ctypes.c_int),
+                ("num_noisy_blocks", ctypes.c_int), ("nnz", ctypes.c_longlong),
+                ("n_cond_tokens", ctypes.c_int), ("n_noisy_tokens", ctypes.c_int),
+                ("attended_token_pairs", ctypes.c_longlong),
+                ("attended_token_pairs_noisy", ctypes.c_longlong)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("liblcbsa.so is not built (python -m block_sparse_attention_rope_b200.build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, I, LL, F, D = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_double
+    S = ctypes.c_int
+    sig = {
+        "lc_bsa_plan_create": (S, [ctypes.POINTER(vp), I, I, I, I, I, I, I, vp]),
+        "lc_bsa_plan_destroy": (S, [vp, vp]),
+        "lc_bsa_plan_info": (S, [vp, ctypes.POINTER(PlanInfo)]),
+        "lc_bsa_plan_copy_csr": (S, [vp, vp, vp, vp]),
+        "lc_rope3d_tables": (S, [ctypes.POINTER(vp), I, I, I, D, I, I, I, vp]),
+        "lc_rope3d_destroy": (S, [vp, vp]),
+        "lc_rope3d_copy_tables": (S, [vp, vp, vp]),
+        "lc_rope3d_apply": (S, [vp, vp, I, LL, I, I, LL, I, vp, vp]),
+        "lc_bsa_forward": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_bsa_forward_cached": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_last_device_status": (S, [vp]),
+        "lc_debug_watchdog_selftest": (S, [I, vp]),
+        "lc_status_string": (ctypes.c_char_p, [S]),
+        "lc_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(s: int) -> str:
+    return lib.lc_status_string(int(s)).decode()
+
+
+def version() -> str:
+    return lib.lc_version().decode()
+
+
+def _check(s: int, where: str):
+    if s != LC_OK:
+        raise LcError(s, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LC_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return LC_DTYPE_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check_bmhk(name: str, t: torch.Tensor, shape, dtype):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous [B, N, heads, head_dim]" % name)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype != dtype:
+        raise ValueError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+
+
+class Plan:
+    """Device-resident block-sparse plan (lc_bsa_plan_create)."""
+
+    def __init__(self, T: int, H: int, W: int, *, local: int, stride: int, n_cond: int = 0,
+                 block: int = 64, stream=None):
+        self.T, self.H, self.W, self.n_cond = T, H, W, n_cond
+        self.local, self.stride, self.block = local, stride, block
+        h = ctypes.c_void_p()
+        _check(lib.lc_bsa_plan_create(ctypes.byref(h), T, H, W, block, local, stride, n_cond,
+                                      _stream(stream)), "lc_bsa_plan_create")
+        self.handle = h
+
+    def info(self) -> PlanInfo:
+        inf = PlanInfo()
+        _check(lib.lc_bsa_plan_info(self.handle, ctypes.byref(inf)), "lc_bsa_plan_info")
+        return inf
+
+    def csr(self, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        inf = self.info()
+        rp = torch.empty(inf.num_q_blocks + 1, dtype=torch.int32)
+        ci = torch.empty(max(inf.nnz, 1), dtype=torch.int32)
+        _check(lib.lc_bsa_plan_copy_csr(self.handle, rp.data_ptr(), ci.data_ptr(), _stream(stream)),
+               "lc_bsa_plan_copy_csr")
+        return rp, ci[:inf.nnz]
+
+    @property
+    def n_tokens(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def n_cond_tokens(self) -> int:
+        return self.n_cond * self.H * self.W
+
+    def close(self, stream=None):
+        if getattr(self, "handle", None):
+            lib.lc_bsa_plan_destroy(self.handle, _stream(stream))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "handle", None) and torch.cuda.is_available():
+                lib.lc_bsa_plan_destroy(self.handle, None)
+        except Exception:
+            pass
+
+
+class Rope3D:
+    """Device-resident partitioned 3D-RoPE tables (lc_rope3d_tables)."""
+
+    def __init__(self, T: int, H: int, W: int, theta: float = 10000.0,
+                 dims: Sequence[int] = (16, 24, 24), stream=None):
+        self.T, self.H, self.W, self.theta, self.dims = T, H, W, theta, tuple(dims)
+        h = ctypes.c_void_p()
+        _check(lib.lc_rope3d_tables(ctypes.byref(h), T, H, W, float(theta), *self.dims,
+                                    _stream(stream)), "lc_rope3d_tables")
+        self.handle = h
+
+    def tables(self, stream=None) -> torch.Tensor:
+        n = self.T * self.dims[0] + self.H * self.dims[1] + self.W * self.dims[2]
+        out = torch.empty(n, dtype=torch.float32)
+        _check(lib.lc_rope3d_copy_tables(self.handle, out.data_ptr(), _stream(stream)),
+               "lc_rope3d_copy_tables")
+        return out
+
+    def apply(self, x: torch.Tensor, tok_offset: int = 0, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+        B, n, heads, hd = x.shape
+        if out is None:
+            out = torch.empty_like(x)
+        _check_bmhk("x", x, x.shape, x.dtype)
+        _check_bmhk("out", out, x.shape, x.dtype)
+        _check(lib.lc_rope3d_apply(x.data_ptr(), out.data_ptr(), B, n, heads, hd, tok_offset,
+                                   _dtype_code(x), self.handle, _stream(stream)), "lc_rope3d_apply")
+        return out
+
+    def close(self, stream=None):
+        if getattr(self, "handle", None):
+            lib.lc_rope3d_destroy(self.handle, _stream(stream))
+            self.handle = None
+
+    def __del__(self):
+        try:
+            if getattr(self, "handle", None) and torch.cuda.is_available():
+                lib.lc_rope3d_destroy(self.handle, None)
+        except Exception:
+            pass
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D, *,
+            out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            return_lse: bool = False, softmax_scale: float = 0.0, stream=None):
+    """Block-sparse 3D-RoPE attention over the full sequence (lc_bsa_forward).
+
+    q, k, v: [B, T*H*W, heads, 64], bf16 or fp32, on the plan's device.
+    Returns out (and lse [B, heads, N] fp32 when asked)."""
+    B, N, heads, hd = q.shape
+    for name, t in (("k", k), ("v", v)):
+        _check_bmhk(name, t, q.shape, q.dtype)
+    _check_bmhk("q", q, (B, plan.n_tokens, heads, hd), q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_bmhk("out", out, q.shape, q.dtype)
+    if return_lse and lse is None:
+        lse = torch.empty(B, heads, N, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_bmhk("lse", lse, (B, heads, N), torch.float32)
+    _check(lib.lc_bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
+                              B, heads, hd, _dtype_code(q), float(softmax_scale), plan.handle,
+                              rope.handle, _stream(stream)), "lc_bsa_forward")
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Optional[torch.Tensor],
+                   cond_v: Optional[torch.Tensor], plan: Plan, rope: Rope3D, *,
+                   out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                   return_lse: bool = False, softmax_scale: float = 0.0, stream=None):
+    """Noisy-query attention with the condition tokens' K/V passed separately
+    (lc_bsa_forward_cached).  q, k, v: [B, Nn, heads, 64]; cond_k, cond_v:
+    [B, Nc, heads, 64], pre-RoPE."""
+    B, Nn, heads, hd = q.shape
+    Nc = plan.n_cond_tokens
+    _check_bmhk("q", q, (B, plan.n_tokens - Nc, heads, hd), q.dtype)
+    for name, t in (("k", k), ("v", v)):
+        _check_bmhk(name, t, q.shape, q.dtype)
+    if Nc > 0:
+        for name, t in (("cond_k", cond_k), ("cond_v", cond_v)):
+            if t is None:
+                raise ValueError("%s is required when the plan has condition frames" % name)
+            _check_bmhk(name, t, (B, Nc, heads, hd), q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    _check_bmhk("out", out, q.shape, q.dtype)
+    if return_lse and lse is None:
+        lse = torch.empty(B, heads, Nn, dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_bmhk("lse", lse, (B, heads, Nn), torch.float32)
+    _check(lib.lc_bsa_forward_cached(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k),
+                                     _ptr(cond_v), out.data_ptr(), _ptr(lse), B, heads, hd,
+                                     _dtype_code(q), float(softmax_scale), plan.handle,
+                                     rope.handle, _stream(stream)), "lc_bsa_forward_cached")
+    return (out, lse) if (return_lse or lse is not None) else out
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status word as a status code."""
+    return int(lib.lc_last_device_status(_stream(stream)))
+
+
+def watchdog_selftest(timeout_us: int = 20000, stream=None) -> int:
+    return int(lib.lc_debug_watchdog_selftest(int(timeout_us), _stream(stream)))

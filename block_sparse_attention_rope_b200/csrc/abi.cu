@@ -1,0 +1,139 @@
+// abi.cu -- argument checking and dispatch of the attention entry points,
+// the per-device status word, status strings.
+#include <mutex>
+
+#include "lc_internal.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int *g_status[kMaxDevices] = {nullptr};
+
+bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+lc_status check_common(const lc_bsa_plan_s *plan, const lc_rope3d_s *rope, int batch, int heads,
+                       int head_dim, lc_dtype dtype) {
+  if (!plan || !rope || batch <= 0 || heads <= 0 || head_dim <= 0)
+    return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
+  if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
+  if (plan->T != rope->T || plan->H != rope->H || plan->W != rope->W)
+    return LC_ERR_INVALID_ARGUMENT;
+  long long rows = (long long)batch * (plan->Nc + plan->Nn) * heads;
+  if (rows * LC_HEAD_DIM >= (1LL << 40)) return LC_ERR_UNSUPPORTED;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return LC_ERR_CUDA;
+  if (dev != plan->device || dev != rope->device) return LC_ERR_INVALID_ARGUMENT;
+  return LC_OK;
+}
+
+lc_status run_forward(const void *q, const void *k, const void *v, const void *cond_k,
+                      const void *cond_v, void *out, float *lse, int batch, int heads, int head_dim,
+                      lc_dtype dtype, float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
+                      void *stream, bool cached) {
+  lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
+  if (s != LC_OK) return s;
+  if (!q || !k || !v || !out) return LC_ERR_INVALID_ARGUMENT;
+  if (cached && plan->Nc > 0 && (!cond_k || !cond_v)) return LC_ERR_INVALID_ARGUMENT;
+  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
+      (cached && plan->Nc > 0 && (misaligned(cond_k) || misaligned(cond_v))) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return LC_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;  // NaN
+  float scale = softmax_scale > 0.f ? softmax_scale : 0.125f;  // 1/sqrt(64)
+  int *dev_status = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == LC_DTYPE_F32)
+    return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
+                                 static_cast<const float *>(v), static_cast<const float *>(cond_k),
+                                 static_cast<const float *>(cond_v), static_cast<float *>(out),
+                                 lse, batch, heads, scale, cached, plan, rope, dev_status, st);
+  return lc_launch_forward_sm100(q, k, v, cond_k, cond_v, out, lse, batch, heads, scale, cached,
+                                 plan, rope, dev_status, st);
+}
+
+}  // namespace
+
+int *lc_device_status_ptr(lc_status *st) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = LC_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status[dev]) {
+    int *p = nullptr;
+    e = cudaMalloc(&p, sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(int));
+    if (e != cudaSuccess) {
+      *st = lc_from_cuda(e);
+      return nullptr;
+    }
+    g_status[dev] = p;
+  }
+  *st = LC_OK;
+  return g_status[dev];
+}
+
+extern "C" lc_status lc_bsa_forward(const void *q, const void *k, const void *v, void *out,
+                                    float *lse, int batch, int heads, int head_dim, lc_dtype dtype,
+                                    float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
+                                    void *stream) {
+  return run_forward(q, k, v, nullptr, nullptr, out, lse, batch, heads, head_dim, dtype,
+                     softmax_scale, plan, rope, stream, false);
+}
+
+extern "C" lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
+                                           const void *cond_k, const void *cond_v, void *out,
+                                           float *lse, int batch, int heads, int head_dim,
+                                           lc_dtype dtype, float softmax_scale, lc_bsa_plan plan,
+                                           lc_rope3d rope, void *stream) {
+  return run_forward(q, k, v, cond_k, cond_v, out, lse, batch, heads, head_dim, dtype,
+                     softmax_scale, plan, rope, stream, true);
+}
+
+extern "C" lc_status lc_last_device_status(void *stream) {
+  lc_status s;
+  int *p = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LC_CUDA_TRY(cudaStreamSynchronize(st));
+  int word = 0;
+  LC_CUDA_TRY(cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost));
+  LC_CUDA_TRY(cudaMemset(p, 0, sizeof(int)));
+  if (word & LC_DEVSTAT_TIMEOUT) return LC_ERR_TIMEOUT;
+  if (word & LC_DEVSTAT_CHECK) return LC_ERR_DEVICE_CHECK;
+  return LC_OK;
+}
+
+extern "C" lc_status lc_debug_watchdog_selftest(int timeout_us, void *stream) {
+  if (timeout_us <= 0 || timeout_us > 10 * 1000 * 1000) return LC_ERR_INVALID_ARGUMENT;
+  lc_status s;
+  int *p = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LC_CUDA_TRY(cudaStreamSynchronize(st));
+  LC_CUDA_TRY(cudaMemset(p, 0, sizeof(int)));
+  s = lc_launch_watchdog_selftest(p, (long long)timeout_us * 1000LL, st);
+  if (s != LC_OK) return s;
+  return lc_last_device_status(stream);
+}
+
+extern "C" const char *lc_status_string(lc_status s) {
+  switch (s) {
+    case LC_OK: return "ok";
+    case LC_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case LC_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LC_ERR_CUDA: return "CUDA error";
+    case LC_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case LC_ERR_TIMEOUT: return "a bounded in-kernel wait timed out";
+    case LC_ERR_DEVICE_CHECK: return "an in-kernel consistency check failed";
+  }
+  return "unknown status";
+}
+
+extern "C" const char *lc_version(void) { return "0.1.0"; }

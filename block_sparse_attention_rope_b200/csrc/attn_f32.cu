@@ -1,0 +1,166 @@
+// attn_f32.cu -- fp32 SIMT block-sparse 3D-RoPE attention.
+//
+// One CTA per (query block, head, batch), one thread per query row.  The CTA
+// walks the query block's key-block list (the plan's CSR row), stages each key
+// block in shared memory with the 3D-RoPE applied on load ("longcat-video-rs"
+// section 03-01; section 03-03 for the block list), and keeps an online
+// softmax in fp32 registers.  Accuracy path for fp32 inputs; the bf16 path is
+// the tcgen05 kernel in attn_sm100.cu.
+#include <math.h>
+
+#include "lc_internal.cuh"
+
+namespace {
+
+struct F32Args {
+  const float *q, *k, *v, *cond_k, *cond_v;
+  float *out, *lse;
+  const int *row_ptr, *col_idx;
+  const float *tab;
+  int T, H, W;
+  lc_divmod div_hw, div_w;
+  int Nc, Nn, Cb, heads;
+  int q_block0;    // first CSR row processed (Cb when only noisy queries)
+  int cached;
+  float scale;
+};
+
+__device__ __forceinline__ void rope_row(float *x, int n, const F32Args &a) {
+  int t = lc_div(n, a.div_hw);
+  int rem = n - t * a.div_hw.d;
+  int h = lc_div(rem, a.div_w);
+  int w = rem - h * a.div_w.d;
+  const float *cT = a.tab, *sT = cT + a.T * 8;
+  const float *cH = sT + a.T * 8, *sH = cH + a.H * 12;
+  const float *cW = sH + a.H * 12, *sW = cW + a.W * 12;
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    float c, s;
+    if (p < 8) { c = cT[t * 8 + p]; s = sT[t * 8 + p]; }
+    else if (p < 20) { c = cH[h * 12 + p - 8]; s = sH[h * 12 + p - 8]; }
+    else { c = cW[w * 12 + p - 20]; s = sW[w * 12 + p - 20]; }
+    float x0 = x[2 * p], x1 = x[2 * p + 1];
+    x[2 * p] = x0 * c - x1 * s;
+    x[2 * p + 1] = x0 * s + x1 * c;
+  }
+}
+
+// Address of head `h` of sequence token m (full-sequence index) for K or V.
+__device__ __forceinline__ const float *kv_row(const float *full, const float *cond, int b, int m,
+                                               int h, const F32Args &a) {
+  if (!a.cached) {
+    long long N = (long long)a.Nc + a.Nn;
+    return full + (((long long)b * N + m) * a.heads + h) * LC_HEAD_DIM;
+  }
+  if (m < a.Nc) return cond + (((long long)b * a.Nc + m) * a.heads + h) * LC_HEAD_DIM;
+  return full + (((long long)b * a.Nn + (m - a.Nc)) * a.heads + h) * LC_HEAD_DIM;
+}
+
+__global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
+  __shared__ float sK[64][LC_HEAD_DIM + 1];
+  __shared__ float sV[64][LC_HEAD_DIM + 1];
+  const int r = a.q_block0 + blockIdx.x;  // CSR row = query block id
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  // Query tokens of block r (full-sequence indices).
+  int q_lo, q_hi;
+  if (r < a.Cb) { q_lo = 64 * r; q_hi = min(a.Nc, q_lo + 64); }
+  else { q_lo = a.Nc + 64 * (r - a.Cb); q_hi = min(a.Nc + a.Nn, q_lo + 64); }
+  const int n = q_lo + tid;
+  const bool valid = n < q_hi;
+  // Row of the q / out tensors that holds token n.
+  const int q_row = a.cached ? n - a.Nc : n;
+  const long long Nq = a.cached ? a.Nn : (long long)a.Nc + a.Nn;
+
+  float q[LC_HEAD_DIM], o[LC_HEAD_DIM];
+  if (valid) {
+    const float *src = a.q + (((long long)b * Nq + q_row) * a.heads + h) * LC_HEAD_DIM;
+#pragma unroll
+    for (int d = 0; d < LC_HEAD_DIM; ++d) q[d] = src[d];
+    rope_row(q, n, a);
+  } else {
+#pragma unroll
+    for (int d = 0; d < LC_HEAD_DIM; ++d) q[d] = 0.f;
+  }
+#pragma unroll
+  for (int d = 0; d < LC_HEAD_DIM; ++d) {
+    q[d] *= a.scale;
+    o[d] = 0.f;
+  }
+  float m_run = -INFINITY, l_run = 0.f;
+
+  for (int e = a.row_ptr[r]; e < a.row_ptr[r + 1]; ++e) {
+    const int c = a.col_idx[e];
+    int k_lo, k_hi;
+    if (c < a.Cb) { k_lo = 64 * c; k_hi = min(a.Nc, k_lo + 64); }
+    else { k_lo = a.Nc + 64 * (c - a.Cb); k_hi = min(a.Nc + a.Nn, k_lo + 64); }
+    const int kn = k_hi - k_lo;
+    __syncthreads();
+    if (tid < kn) {
+      const int m = k_lo + tid;
+      float kr[LC_HEAD_DIM];
+      const float *ks = kv_row(a.k, a.cond_k, b, m, h, a);
+      const float *vs = kv_row(a.v, a.cond_v, b, m, h, a);
+#pragma unroll
+      for (int d = 0; d < LC_HEAD_DIM; ++d) kr[d] = ks[d];
+      rope_row(kr, m, a);
+#pragma unroll
+      for (int d = 0; d < LC_HEAD_DIM; ++d) {
+        sK[tid][d] = kr[d];
+        sV[tid][d] = vs[d];
+      }
+    }
+    __syncthreads();
+    for (int j = 0; j < kn; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int d = 0; d < LC_HEAD_DIM; ++d) s = fmaf(q[d], sK[j][d], s);
+      if (s > m_run) {
+        float corr = expf(m_run - s);  // 0 on the first key
+        l_run = l_run * corr + 1.f;
+#pragma unroll
+        for (int d = 0; d < LC_HEAD_DIM; ++d) o[d] = fmaf(o[d], corr, sV[j][d]);
+        m_run = s;
+      } else {
+        float p = expf(s - m_run);
+        l_run += p;
+#pragma unroll
+        for (int d = 0; d < LC_HEAD_DIM; ++d) o[d] = fmaf(p, sV[j][d], o[d]);
+      }
+    }
+  }
+  if (!valid) return;
+  const float inv = 1.f / l_run;
+  float *dst = a.out + (((long long)b * Nq + q_row) * a.heads + h) * LC_HEAD_DIM;
+#pragma unroll
+  for (int d = 0; d < LC_HEAD_DIM; ++d) dst[d] = o[d] * inv;
+  if (a.lse) a.lse[((long long)b * a.heads + h) * Nq + q_row] = m_run + logf(l_run);
+}
+
+}  // namespace
+
+lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
+                                const float *cond_k, const float *cond_v, float *out, float *lse,
+                                int batch, int heads, float scale, bool cached,
+                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                int * /*dev_status*/, cudaStream_t stream) {
+  F32Args a;
+  a.q = q; a.k = k; a.v = v; a.cond_k = cond_k; a.cond_v = cond_v;
+  a.out = out; a.lse = lse;
+  a.row_ptr = plan->row_ptr; a.col_idx = plan->col_idx;
+  a.tab = rope->tab;
+  a.T = rope->T; a.H = rope->H; a.W = rope->W;
+  a.div_hw = lc_make_divmod(rope->H * rope->W);
+  a.div_w = lc_make_divmod(rope->W);
+  a.Nc = plan->Nc; a.Nn = plan->Nn; a.Cb = plan->Cb; a.heads = heads;
+  a.cached = cached ? 1 : 0;
+  a.q_block0 = cached ? plan->Cb : 0;
+  a.scale = scale;
+  int nrows = cached ? plan->Nb : plan->nq;
+  if (nrows == 0) return LC_OK;
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
+  dim3 grid(nrows, heads, batch);
+  attn_f32_kernel<<<grid, 64, 0, stream>>>(a);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}

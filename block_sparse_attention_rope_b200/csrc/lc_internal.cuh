@@ -1,0 +1,101 @@
+// lc_internal.cuh -- definitions shared by the translation units of liblcbsa.so
+// (plan and rope handles, status plumbing, launch helpers).  Not installed.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/lc_bsa.h"
+
+// Device status bits written by kernels (see lc_last_device_status).
+#define LC_DEVSTAT_TIMEOUT 0x1
+#define LC_DEVSTAT_CHECK 0x2
+
+// Tokens of one block, head dimension and RoPE split supported by v1.
+#define LC_BLOCK 64
+#define LC_HEAD_DIM 64
+
+// Block-sparse plan.  All arrays live in one device allocation `mem`.
+//
+// Block ids: 0..Cb-1 are condition blocks (tokens [64c, min(Nc, 64c+64)) of the
+// condition segment), Cb..Cb+Nb-1 noisy blocks (tokens [64j, ...) of the noisy
+// segment).  A "group" is up to 4 consecutive query blocks of one segment,
+// the unit of work of the tensor-core kernel (two 128-row query tiles); its
+// entry list is the sorted union of its members' key blocks, each entry
+// holding (key block id) | (member mask << 24).
+struct lc_bsa_plan_s {
+  int T, H, W, block, local, stride, n_cond;
+  int Nc, Nn, Cb, Nb, nq;
+  int gc, gn, G;            // groups in the condition / noisy segment, total
+  long long nnz;            // CSR entries (host closed form, checked on device)
+  int device;
+  cudaEvent_t ready;        // recorded after the planner kernels
+  void *mem;
+  int *row_ptr;             // [nq + 1]
+  int *col_idx;             // [nnz]
+  int *row_cnt;             // [nq]      planner work array
+  int *grp_ptr;             // [G + 1]
+  int *grp_cnt;             // [G]       planner work array
+  uint32_t *grp_ent;        // [nnz]     (upper bound of the union lists)
+  int *grp_order;           // [G]       groups by entry count, longest first
+  unsigned long long *pairs;  // [2] attended token pairs: all rows, noisy rows
+  int *err;                 // [1] planner consistency flag
+  long long pairs_host[2];
+  bool info_cached;
+};
+
+// RoPE tables: fp32 [cos_t T*dt/2][sin_t][cos_h H*dh/2][sin_h][cos_w W*dw/2][sin_w].
+struct lc_rope3d_s {
+  int T, H, W;
+  double theta;
+  int dt, dh, dw;
+  int device;
+  long long n_floats;
+  float *tab;
+};
+
+// Per-device library state: the status word kernels report into.
+int *lc_device_status_ptr(lc_status *st);
+
+// Map a CUDA error to a status (out-of-memory gets its own code).
+static inline lc_status lc_from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return LC_OK;
+  if (e == cudaErrorMemoryAllocation) return LC_ERR_OUT_OF_MEMORY;
+  return LC_ERR_CUDA;
+}
+
+#define LC_CUDA_TRY(expr)                                   \
+  do {                                                      \
+    cudaError_t _e = (expr);                                \
+    if (_e != cudaSuccess) return lc_from_cuda(_e);         \
+  } while (0)
+
+// Fast exact division of non-negative n < 2^24 by a constant d < 2^16:
+// q = (n * m) >> 40 with m = ceil(2^40 / d).  Exact because the rounding
+// error n*(m*d - 2^40) < n*d <= 2^40 keeps the quotient's integer part.
+struct lc_divmod {
+  unsigned long long m;
+  int d;
+};
+static inline lc_divmod lc_make_divmod(int d) {
+  lc_divmod r;
+  r.d = d;
+  r.m = ((1ull << 40) + (unsigned long long)d - 1ull) / (unsigned long long)d;
+  return r;
+}
+__device__ __forceinline__ int lc_div(int n, lc_divmod dm) {
+  return (int)(((unsigned long long)(unsigned)n * dm.m) >> 40);
+}
+
+// Launch helpers implemented by the kernel translation units.
+lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
+                                const float *cond_k, const float *cond_v, float *out,
+                                float *lse, int batch, int heads, float scale, bool cached,
+                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                int *dev_status, cudaStream_t stream);
+lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
+                                  const void *cond_k, const void *cond_v, void *out,
+                                  float *lse, int batch, int heads, float scale, bool cached,
+                                  const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                  int *dev_status, cudaStream_t stream);
+lc_status lc_launch_watchdog_selftest(int *dev_status, long long timeout_ns, cudaStream_t stream);

@@ -1,0 +1,168 @@
+// rope.cu -- partitioned 3D-RoPE tables and the standalone rotation kernel.
+//
+// "longcat-video-rs" header card ("16T + 24H + 24W ... norm-conserving
+// spatiotemporal rotary pairs") and section 03-01: a 64-D head is split into
+// a temporal slice (channels [0,16)), a height slice ([16,40)) and a width
+// slice ([40,64)); pair (c, c+1) of a slice of width d, pair index k, turns by
+// pos * theta^(-2k/d) with pos the token's t, h or w.
+#include <math.h>
+
+#include <new>
+
+#include "lc_internal.cuh"
+#include <cuda_bf16.h>
+
+namespace {
+
+// One thread per table entry; angles and cos/sin in fp64, stored fp32.
+__global__ void rope_tables_kernel(float *tab, int T, int H, int W, double theta, int dt, int dh,
+                                   int dw) {
+  long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const int npos[3] = {T, H, W};
+  const int dims[3] = {dt, dh, dw};
+  long long base = 0;
+  for (int a = 0; a < 3; ++a) {
+    long long half = (long long)npos[a] * (dims[a] / 2);
+    if (i < base + 2 * half) {
+      long long j = i - base;
+      bool is_sin = j >= half;
+      if (is_sin) j -= half;
+      int pos = (int)(j / (dims[a] / 2));
+      int k = (int)(j % (dims[a] / 2));
+      double omega = pow(theta, -2.0 * (double)k / (double)dims[a]);
+      double phi = (double)pos * omega;
+      tab[i] = (float)(is_sin ? sin(phi) : cos(phi));
+      return;
+    }
+    base += 2 * half;
+  }
+}
+
+// Rotate the 4 channel pairs of 8-channel chunk `ch` (0..7) of a 64-D head.
+__device__ __forceinline__ void rotate_chunk(float (&x)[8], int ch, int t, int h, int w,
+                                             const float *tab, int T, int H, int W) {
+  const float *c, *s;
+  if (ch < 2) {
+    c = tab + t * 8 + 4 * ch;
+    s = c + T * 8;
+  } else if (ch < 5) {
+    c = tab + T * 16 + h * 12 + 4 * (ch - 2);
+    s = c + H * 12;
+  } else {
+    c = tab + T * 16 + H * 24 + w * 12 + 4 * (ch - 5);
+    s = c + W * 12;
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    float a = x[2 * p], b = x[2 * p + 1];
+    float cc = c[p], ss = s[p];
+    x[2 * p] = a * cc - b * ss;
+    x[2 * p + 1] = a * ss + b * cc;
+  }
+}
+
+template <typename Tin>
+__global__ void rope_apply_kernel(const Tin *x, Tin *out, long long n_chunks, int heads,
+                                  long long ntok, long long tok_offset, const float *tab, int T,
+                                  int H, int W, lc_divmod div_hw, lc_divmod div_w) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_chunks;
+       i += (long long)gridDim.x * blockDim.x) {
+    int ch = (int)(i & 7);
+    long long tokhead = i >> 3;
+    long long tok = (tokhead / heads) % ntok;
+    int n = (int)(tok + tok_offset);
+    int t = lc_div(n, div_hw);
+    int rem = n - t * div_hw.d;
+    int h = lc_div(rem, div_w);
+    int w = rem - h * div_w.d;
+    float v[8];
+    const Tin *src = x + i * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (float)src[e];
+    rotate_chunk(v, ch, t, h, w, tab, T, H, W);
+    Tin *dst = out + i * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[e] = (Tin)v[e];
+  }
+}
+
+}  // namespace
+
+extern "C" lc_status lc_rope3d_tables(lc_rope3d *out, int T, int H, int W, double theta, int dim_t,
+                                      int dim_h, int dim_w, void *stream) {
+  if (!out || T <= 0 || H <= 0 || W <= 0 || !(theta > 0.0) || dim_t <= 0 || dim_h <= 0 ||
+      dim_w <= 0 || (dim_t & 1) || (dim_h & 1) || (dim_w & 1))
+    return LC_ERR_INVALID_ARGUMENT;
+  if (dim_t != 16 || dim_h != 24 || dim_w != 24) return LC_ERR_UNSUPPORTED;
+  if ((long long)T * H * W >= (1LL << 24) || (long long)H * W >= (1LL << 16))
+    return LC_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  lc_rope3d_s *r = new (std::nothrow) lc_rope3d_s();
+  if (!r) return LC_ERR_OUT_OF_MEMORY;
+  r->T = T; r->H = H; r->W = W; r->theta = theta;
+  r->dt = dim_t; r->dh = dim_h; r->dw = dim_w;
+  r->n_floats = (long long)T * dim_t + (long long)H * dim_h + (long long)W * dim_w;
+  lc_status s = lc_from_cuda(cudaGetDevice(&r->device));
+  if (s != LC_OK) { delete r; return s; }
+  cudaError_t e = cudaMallocAsync(&r->tab, sizeof(float) * r->n_floats, st);
+  if (e != cudaSuccess) { delete r; return lc_from_cuda(e); }
+  int tpb = 256;
+  int nb = (int)((r->n_floats + tpb - 1) / tpb);
+  rope_tables_kernel<<<nb, tpb, 0, st>>>(r->tab, T, H, W, theta, dim_t, dim_h, dim_w);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    cudaFreeAsync(r->tab, st);
+    delete r;
+    return lc_from_cuda(e);
+  }
+  *out = r;
+  return LC_OK;
+}
+
+extern "C" lc_status lc_rope3d_destroy(lc_rope3d rope, void *stream) {
+  if (!rope) return LC_OK;
+  cudaError_t e = cudaFreeAsync(rope->tab, static_cast<cudaStream_t>(stream));
+  delete rope;
+  return lc_from_cuda(e);
+}
+
+extern "C" lc_status lc_rope3d_copy_tables(lc_rope3d rope, float *host, void *stream) {
+  if (!rope || !host) return LC_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LC_CUDA_TRY(cudaMemcpyAsync(host, rope->tab, sizeof(float) * rope->n_floats,
+                              cudaMemcpyDeviceToHost, st));
+  LC_CUDA_TRY(cudaStreamSynchronize(st));
+  return LC_OK;
+}
+
+extern "C" lc_status lc_rope3d_apply(const void *x, void *out, int batch, long long ntok, int heads,
+                                     int head_dim, long long tok_offset, lc_dtype dtype,
+                                     lc_rope3d rope, void *stream) {
+  if (!x || !out || !rope || batch <= 0 || ntok <= 0 || heads <= 0 || tok_offset < 0)
+    return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
+  if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
+  if (tok_offset + ntok > (long long)rope->T * rope->H * rope->W) return LC_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return LC_ERR_INVALID_ARGUMENT;
+  int dev = -1;
+  LC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != rope->device) return LC_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  long long n_chunks = (long long)batch * ntok * heads * (LC_HEAD_DIM / 8);
+  int tpb = 256;
+  long long want = (n_chunks + tpb - 1) / tpb;
+  int nb = (int)(want < 148LL * 16 ? want : 148LL * 16);
+  lc_divmod dhw = lc_make_divmod(rope->H * rope->W), dw = lc_make_divmod(rope->W);
+  if (dtype == LC_DTYPE_F32)
+    rope_apply_kernel<float><<<nb, tpb, 0, st>>>(static_cast<const float *>(x),
+                                                 static_cast<float *>(out), n_chunks, heads, ntok,
+                                                 tok_offset, rope->tab, rope->T, rope->H, rope->W,
+                                                 dhw, dw);
+  else
+    rope_apply_kernel<__nv_bfloat16><<<nb, tpb, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(out), n_chunks,
+        heads, ntok, tok_offset, rope->tab, rope->T, rope->H, rope->W, dhw, dw);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}

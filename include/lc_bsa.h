@@ -1,0 +1,206 @@
+/*
+ * lc_bsa.h -- C ABI of liblcbsa.so: block-sparse 3D-RoPE self-attention over
+ * video latent tokens (the 3D self-attention of the LongCat-Video diffusion
+ * transformer), for NVIDIA B200 (sm_100a).
+ *
+ * What the operation is (sources are the pages the method is described on):
+ *   - "longcat-video-rs" (code.brandonhubbard.com), header card and section
+ *     03-01 "Partitioned 3D-RoPE (16T+24H+24W)": every 64-D head is split into
+ *     16 temporal, 24 height and 24 width channels, rotated as complex pairs
+ *     by the token's (t, h, w) position.
+ *   - same page, section 03-03 "Block-Sparse & Multi-Audio" and the section 02
+ *     table row "Block-Sparse Self-Attention (block=64, local=2, stride=4)":
+ *     a query block attends a local window of key blocks plus strided global
+ *     key blocks.
+ *   - "美团视频生成模型来了！一出手就是开源 SOTA" (myzaker / QbitAI), section
+ *     "背后技术原理": condition frames precede the noisy frames on the time
+ *     axis; condition tokens are not affected by noise tokens and their K/V
+ *     can be cached and reused.
+ *
+ * Readings where the pages are silent (same as the test oracle's):
+ *   token n of the full sequence sits at t = n/(H*W), h = (n/W)%H, w = n%W;
+ *   RoPE pair k of an axis of width d turns by pos*theta^(-2k/d), pairs are
+ *   adjacent channels (c, c+1), axes in the order T, H, W;
+ *   a block is 64 consecutive tokens of one segment (the first Nc = n_cond*H*W
+ *   tokens are the condition segment, the rest the noisy segment; the last
+ *   block of a segment may be short);
+ *   noisy block i attends noisy block j iff |i-j| <= local or
+ *   (stride > 0 and j % stride == 0); stride == 1 is dense, stride <= 0 means
+ *   no global blocks;
+ *   condition queries attend every condition key and no noisy key; noisy
+ *   queries attend every condition key plus their noisy blocks;
+ *   softmax scale 1/sqrt(head_dim) unless given.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are contiguous [B, N, heads, head_dim] ("BMHK"), tokens ordered
+ *     t-major, then h, then w.  Device pointers, 16-byte aligned.  LSE is
+ *     [B, heads, Nq] fp32, natural log.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Every call is stream ordered and returns without waiting for the GPU,
+ *     except lc_bsa_plan_info, lc_bsa_plan_copy_csr, lc_rope3d_copy_tables and
+ *     lc_last_device_status, which synchronise the stream.
+ *   - Errors are returned as lc_status; argument errors are detected before any
+ *     GPU work is queued.  No C++ exception crosses this boundary.
+ *   - The caller owns q/k/v/out/lse.  The library owns the memory behind plan
+ *     and rope handles (allocated stream-ordered on the given stream, released
+ *     by the matching *_destroy on its stream).
+ *   - There is no CPU fallback: on a machine without a usable sm_100 GPU the
+ *     calls that need one return LC_ERR_CUDA.
+ *   - v1 supports block = 64 and head_dim = 64 with RoPE channel split
+ *     16/24/24; other values return LC_ERR_UNSUPPORTED.
+ */
+#ifndef LC_BSA_H
+#define LC_BSA_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LC_OK = 0,
+    LC_ERR_INVALID_ARGUMENT = 1,  /* null pointer, bad size, misaligned pointer, mismatch */
+    LC_ERR_UNSUPPORTED = 2,       /* valid but not implemented (block or head_dim != 64 ...) */
+    LC_ERR_CUDA = 3,              /* a CUDA runtime/driver call failed (incl. no device) */
+    LC_ERR_OUT_OF_MEMORY = 4,     /* device allocation failed */
+    LC_ERR_TIMEOUT = 5,           /* a bounded in-kernel wait gave up (device status) */
+    LC_ERR_DEVICE_CHECK = 6       /* an in-kernel bounds/consistency check failed (device status) */
+} lc_status;
+
+typedef enum {
+    LC_DTYPE_BF16 = 0,   /* tcgen05 tensor-core kernel, fp32 accumulation */
+    LC_DTYPE_F32 = 1     /* fp32 SIMT kernel (exact-arithmetic reference speed path) */
+} lc_dtype;
+
+typedef struct lc_bsa_plan_s *lc_bsa_plan;   /* opaque, device resident, read-only once built */
+typedef struct lc_rope3d_s *lc_rope3d;       /* opaque, device resident */
+
+/* Summary of a plan; returned by lc_bsa_plan_info. */
+typedef struct {
+    int num_q_blocks;          /* Cb + Nb: rows of the block CSR */
+    int num_cond_blocks;       /* Cb = ceil(Nc / block) */
+    int num_noisy_blocks;      /* Nb = ceil(Nn / block) */
+    long long nnz;             /* entries of the block CSR */
+    int n_cond_tokens;         /* Nc = n_cond_frames * H * W */
+    int n_noisy_tokens;        /* Nn = (T - n_cond_frames) * H * W */
+    long long attended_token_pairs;        /* per head, all queries (lc_bsa_forward) */
+    long long attended_token_pairs_noisy;  /* per head, noisy queries (lc_bsa_forward_cached) */
+} lc_bsa_plan_info_t;
+
+/*
+ * lc_bsa_plan_create -- build, on the device, the block-sparse pattern of a
+ * (T, H, W) latent video with n_cond_frames condition frames: for each query
+ * block the sorted list of attended key blocks (block CSR, key ids 0..Cb-1 for
+ * condition blocks then Cb+j for noisy block j), plus the kernel's internal
+ * work lists.  Source: "longcat-video-rs" section 03-03 and the section 02
+ * table row (local window + strided global blocks, block=64); myzaker / QbitAI
+ * "背后技术原理" (condition frames first, isolated from noise).
+ *   T: latent frames including condition frames (T > n_cond_frames >= 0);
+ *   block: 64; local >= 0; stride: <= 0 none, 1 dense, > 1 strided globals.
+ * Errors: LC_ERR_INVALID_ARGUMENT (out NULL, T/H/W <= 0, local < 0,
+ * n_cond_frames outside [0, T), token count >= 2^31), LC_ERR_UNSUPPORTED
+ * (block != 64), LC_ERR_OUT_OF_MEMORY, LC_ERR_CUDA.  *out is set only on LC_OK.
+ */
+lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, int block, int local,
+                             int stride, int n_cond_frames, void *stream);
+
+/* Release a plan (stream ordered on `stream`).  NULL is accepted. */
+lc_status lc_bsa_plan_destroy(lc_bsa_plan plan, void *stream);
+
+/* Sizes of a plan.  Waits for the plan's construction to finish. */
+lc_status lc_bsa_plan_info(lc_bsa_plan plan, lc_bsa_plan_info_t *info);
+
+/* Copy the block CSR to host memory: row_ptr_host[num_q_blocks + 1],
+ * col_idx_host[nnz] (int32).  Synchronises `stream`.  For checking the plan. */
+lc_status lc_bsa_plan_copy_csr(lc_bsa_plan plan, int *row_ptr_host, int *col_idx_host,
+                               void *stream);
+
+/*
+ * lc_rope3d_tables -- per-axis cos/sin tables of the partitioned 3D-RoPE
+ * ("longcat-video-rs" header card and section 03-01): for axis a in (T, H, W)
+ * of width dim_a and pair k < dim_a/2, angle = pos * theta^(-2k/dim_a), pos in
+ * [0, T), [0, H), [0, W).  Computed in fp64 on the device, stored fp32.
+ * dim_t + dim_h + dim_w is the head dimension; v1 needs (16, 24, 24).
+ * Errors: LC_ERR_INVALID_ARGUMENT (out NULL, sizes <= 0, odd dims, theta <= 0),
+ * LC_ERR_UNSUPPORTED (dims other than 16/24/24), LC_ERR_OUT_OF_MEMORY, LC_ERR_CUDA.
+ */
+lc_status lc_rope3d_tables(lc_rope3d *out, int T, int H, int W, double theta,
+                           int dim_t, int dim_h, int dim_w, void *stream);
+
+/* Release rope tables (stream ordered).  NULL is accepted. */
+lc_status lc_rope3d_destroy(lc_rope3d rope, void *stream);
+
+/* Copy the tables to host memory as fp32, in this order: cos_t[T][dim_t/2],
+ * sin_t[T][dim_t/2], cos_h[H][dim_h/2], sin_h[H][dim_h/2], cos_w[W][dim_w/2],
+ * sin_w[W][dim_w/2].  `host` holds (T*dim_t + H*dim_h + W*dim_w) floats.
+ * Synchronises `stream`. */
+lc_status lc_rope3d_copy_tables(lc_rope3d rope, float *host, void *stream);
+
+/*
+ * lc_rope3d_apply -- rotate x [B, ntok, heads, head_dim] by the partitioned
+ * 3D-RoPE into out (same shape and dtype; out == x is allowed).  Token n of x is
+ * token n + tok_offset of the full sequence.  The standalone form of the
+ * rotation that the attention entry points fuse into their Q/K tile loads
+ * ("longcat-video-rs" section 02 row "3D-RoPE Spatiotemporal Frequency & Token
+ * Rotation", section 03-01).  Requires tok_offset + ntok <= T*H*W of the tables.
+ */
+lc_status lc_rope3d_apply(const void *x, void *out, int batch, long long ntok, int heads,
+                          int head_dim, long long tok_offset, lc_dtype dtype,
+                          lc_rope3d rope, void *stream);
+
+/*
+ * lc_bsa_forward -- out = softmax(mask(scale * R(q) R(k)^T)) v over the whole
+ * sequence of N = T*H*W tokens, with R the 3D-RoPE of `rope` and the mask of
+ * `plan`; optionally lse (nullable).  q, k, v, out: [batch, N, heads, head_dim]
+ * of `dtype`; lse: [batch, heads, N] fp32.  softmax_scale <= 0 means
+ * 1/sqrt(head_dim).  plan and rope must describe the same (T, H, W).
+ * Errors: LC_ERR_INVALID_ARGUMENT (NULL tensors or handles, batch/heads <= 0,
+ * pointers not 16-byte aligned, plan/rope grid mismatch), LC_ERR_UNSUPPORTED
+ * (head_dim != 64), LC_ERR_CUDA (launch failure).  In-kernel faults of the
+ * bounded waits or checks are reported by lc_last_device_status.
+ */
+lc_status lc_bsa_forward(const void *q, const void *k, const void *v, void *out, float *lse,
+                         int batch, int heads, int head_dim, lc_dtype dtype,
+                         float softmax_scale, lc_bsa_plan plan, lc_rope3d rope, void *stream);
+
+/*
+ * lc_bsa_forward_cached -- the same attention for the noisy queries only, with
+ * the condition tokens' K/V supplied separately (the KV-cache form of myzaker /
+ * QbitAI "背后技术原理").  q, k, v, out: [batch, Nn, heads, head_dim] (noisy
+ * tokens); cond_k, cond_v: [batch, Nc, heads, head_dim], pre-RoPE like k (they
+ * are rotated with t in [0, n_cond_frames)); lse: [batch, heads, Nn] or NULL.
+ * With n_cond_frames == 0, cond_k/cond_v may be NULL.  Errors as lc_bsa_forward.
+ */
+lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
+                                const void *cond_k, const void *cond_v, void *out,
+                                float *lse, int batch, int heads, int head_dim,
+                                lc_dtype dtype, float softmax_scale, lc_bsa_plan plan,
+                                lc_rope3d rope, void *stream);
+
+/*
+ * lc_last_device_status -- synchronise `stream`, then report and clear the
+ * current device's status word, which the kernels set when a bounded wait
+ * timed out (LC_ERR_TIMEOUT) or an in-kernel check failed
+ * (LC_ERR_DEVICE_CHECK).  LC_OK when nothing was flagged.
+ */
+lc_status lc_last_device_status(void *stream);
+
+/*
+ * lc_debug_watchdog_selftest -- launch one CTA that waits, with the same
+ * bounded wait the attention kernel uses, on a barrier that nothing ever
+ * arrives on; the wait gives up after timeout_us microseconds and the kernel
+ * returns normally.  Returns the device status that run left
+ * (LC_ERR_TIMEOUT when the watchdog works).  For tests of failure detection.
+ */
+lc_status lc_debug_watchdog_selftest(int timeout_us, void *stream);
+
+/* Static description of a status code. */
+const char *lc_status_string(lc_status s);
+
+/* Library version, "major.minor.patch". */
+const char *lc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LC_BSA_H */

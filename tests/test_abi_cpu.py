@@ -1,0 +1,90 @@
+"""The C-ABI library loads, exports every symbol its header declares, and
+rejects bad arguments before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lc_bsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_rope_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(lc_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ["lc_bsa_plan_create", "lc_bsa_plan_destroy", "lc_bsa_plan_info",
+                 "lc_bsa_plan_copy_csr", "lc_rope3d_tables", "lc_rope3d_destroy",
+                 "lc_bsa_forward", "lc_bsa_forward_cached", "lc_last_device_status",
+                 "lc_status_string"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    lib.lc_status_string.restype = ctypes.c_char_p
+    seen = set()
+    for code in range(7):
+        s = lib.lc_status_string(code).decode()
+        assert s and s != "unknown status"
+        seen.add(s)
+    assert len(seen) == 7
+    assert lib.lc_status_string(99).decode() == "unknown status"
+
+
+def test_plan_argument_errors_before_any_gpu_work(lib):
+    h = ctypes.c_void_p()
+    f = lib.lc_bsa_plan_create
+    f.argtypes = [ctypes.POINTER(ctypes.c_void_p)] + [ctypes.c_int] * 7 + [ctypes.c_void_p]
+    assert f(None, 4, 8, 16, 64, 2, 4, 0, None) == 1
+    assert f(ctypes.byref(h), 0, 8, 16, 64, 2, 4, 0, None) == 1        # T <= 0
+    assert f(ctypes.byref(h), 4, 8, 16, 64, -1, 4, 0, None) == 1       # local < 0
+    assert f(ctypes.byref(h), 4, 8, 16, 64, 2, 4, 4, None) == 1        # n_cond >= T
+    assert f(ctypes.byref(h), 4, 8, 16, 32, 2, 4, 0, None) == 2        # block != 64
+    assert f(ctypes.byref(h), 4096, 64, 64, 64, 2, 4, 0, None) == 2    # > 2^24 tokens
+    assert h.value is None
+
+
+def test_rope_argument_errors(lib):
+    h = ctypes.c_void_p()
+    f = lib.lc_rope3d_tables
+    f.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+    assert f(ctypes.byref(h), 4, 8, 16, 0.0, 16, 24, 24, None) == 1    # theta
+    assert f(ctypes.byref(h), 4, 8, 16, 1e4, 15, 25, 24, None) == 1    # odd dims
+    assert f(ctypes.byref(h), 4, 8, 16, 1e4, 32, 16, 16, None) == 2    # other split
+    assert h.value is None
+
+
+def test_forward_rejects_null_handles(lib):
+    f = lib.lc_bsa_forward
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 3
+    assert f(None, None, None, None, None, 1, 2, 64, 0, 0.0, None, None, None) == 1
+    g = lib.lc_bsa_forward_cached
+    g.argtypes = [ctypes.c_void_p] * 7 + [ctypes.c_int] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 3
+    assert g(None, None, None, None, None, None, None, 1, 2, 64, 0, 0.0, None, None, None) == 1
+
+
+def test_python_binding_imports_only_the_library():
+    """The binding module must not reach the oracle (no CPU fallback)."""
+    src = open(os.path.join(ROOT, "block_sparse_attention_rope_b200", "api.py")).read()
+    assert "oracle" not in src.replace("no CPU fallback", "")
+    for f in os.listdir(os.path.join(ROOT, "block_sparse_attention_rope_b200", "csrc")):
+        assert "oracle" not in open(os.path.join(ROOT, "block_sparse_attention_rope_b200",
+                                                 "csrc", f)).read().lower()

@@ -1,0 +1,191 @@
+"""GPU attention (fp32 SIMT and bf16 tcgen05 kernels) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+from block_sparse_attention_rope_b200 import synthetic
+from block_sparse_attention_rope_b200.synthetic import Workload
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    # several 256-row groups, a condition frame, ragged nothing
+    "small_i2v": Workload("small_i2v", T=4, H=16, W=40, n_cond=1, heads=4, local=2, stride=4,
+                          dtype="bf16"),
+    # partial blocks at the end of both segments (273 tokens per frame)
+    "ragged": Workload("ragged", T=6, H=13, W=21, n_cond=1, heads=3, local=1, stride=3,
+                       dtype="bf16"),
+    "dense_small": Workload("dense_small", T=3, H=16, W=32, n_cond=0, heads=2, local=0, stride=1,
+                            dtype="bf16"),
+    "local_only": Workload("local_only", T=2, H=10, W=30, n_cond=0, heads=2, local=0, stride=0,
+                           dtype="bf16"),
+    "batch2": Workload("batch2", T=3, H=8, W=24, n_cond=1, heads=2, local=1, stride=2,
+                       dtype="bf16", batch=2),
+    "many_heads": Workload("many_heads", T=2, H=8, W=32, n_cond=0, heads=32, local=2, stride=4,
+                           dtype="bf16"),
+    "one_block": Workload("one_block", T=1, H=5, W=12, n_cond=0, heads=2, local=2, stride=4,
+                          dtype="bf16"),
+    "cached_small": Workload("cached_small", T=5, H=8, W=20, n_cond=2, heads=2, local=1,
+                             stride=3, dtype="bf16", cached=True),
+    "cached_ragged": Workload("cached_ragged", T=4, H=7, W=19, n_cond=1, heads=2, local=2,
+                              stride=4, dtype="bf16", cached=True),
+    "ragged_f32": Workload("ragged_f32", T=6, H=13, W=21, n_cond=1, heads=3, local=1, stride=3,
+                           dtype="f32"),
+    "cached_f32": Workload("cached_f32", T=5, H=8, W=20, n_cond=2, heads=2, local=1, stride=3,
+                           dtype="f32", cached=True),
+}
+
+
+@pytest.fixture(scope="module")
+def api():
+    from block_sparse_attention_rope_b200 import build
+    build.build()
+    from block_sparse_attention_rope_b200 import api as a
+    return a
+
+
+def run_gpu(api, w, inputs):
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    d = {k: v.cuda() for k, v in inputs.items()}
+    if w.cached:
+        out, lse = api.forward_cached(d["q"], d["k"], d["v"], d.get("cond_k"), d.get("cond_v"),
+                                      plan, rope, return_lse=True)
+    else:
+        out, lse = api.forward(d["q"], d["k"], d["v"], plan, rope, return_lse=True)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    return out.cpu(), lse.cpu()
+
+
+def full_oracle(w, inputs):
+    kw = dict(T=w.T, H=w.H, W=w.W, n_cond=w.n_cond, local=w.local, stride=w.stride)
+    if w.cached:
+        return oracle.forward_cached(inputs["q"], inputs["k"], inputs["v"], inputs["cond_k"],
+                                     inputs["cond_v"], **kw)
+    return oracle.forward(inputs["q"], inputs["k"], inputs["v"], **kw)
+
+
+def check_all_rows(w, out, lse, ref_out, ref_lse):
+    g = out.float().numpy().astype(np.float64)
+    err = np.abs(g - ref_out)
+    lerr = np.abs(lse.numpy().astype(np.float64) - ref_lse).max()
+    if w.dtype == "f32":
+        assert err.max() <= parity.F32_MAX_ABS, err.max()
+        assert lerr <= parity.F32_LSE_ABS, lerr
+    else:
+        assert err.max() <= parity.BF16_MAX_ABS, (err.max(), err.mean())
+        assert err.mean() <= parity.BF16_MEAN_ABS, (err.max(), err.mean())
+        assert lerr <= parity.BF16_LSE_ABS, lerr
+    return err.max(), err.mean(), lerr
+
+
+def test_tiny_f32_all_rows(api):
+    w = synthetic.get("tiny_f32")
+    inputs = synthetic.make_inputs(w)
+    out, lse = run_gpu(api, w, inputs)
+    ref_out, ref_lse = full_oracle(w, inputs)
+    mx, mean, lerr = check_all_rows(w, out, lse, ref_out, ref_lse)
+    print("tiny_f32 max %.3g mean %.3g lse %.3g" % (mx, mean, lerr))
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_all_rows(api, name):
+    w = SMALL[name]
+    inputs = synthetic.make_inputs(w)
+    out, lse = run_gpu(api, w, inputs)
+    assert torch.isfinite(out.float()).all()
+    ref_out, ref_lse = full_oracle(w, inputs)
+    mx, mean, lerr = check_all_rows(w, out, lse, ref_out, ref_lse)
+    print("%s max %.3g mean %.3g lse %.3g" % (name, mx, mean, lerr))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_cached_equals_noisy_rows_of_forward(api, dtype):
+    w = Workload("x", T=5, H=8, W=24, n_cond=2, heads=3, local=1, stride=3, dtype=dtype)
+    full = synthetic.make_inputs(w)
+    out_full, lse_full = run_gpu(api, w, full)
+    Nc = w.n_cond_tokens
+    cin = {"q": full["q"][:, Nc:].contiguous(), "k": full["k"][:, Nc:].contiguous(),
+           "v": full["v"][:, Nc:].contiguous(), "cond_k": full["k"][:, :Nc].contiguous(),
+           "cond_v": full["v"][:, :Nc].contiguous()}
+    wc = Workload("xc", T=5, H=8, W=24, n_cond=2, heads=3, local=1, stride=3, dtype=dtype,
+                  cached=True)
+    out_c, lse_c = run_gpu(api, wc, cin)
+    assert torch.equal(out_c, out_full[:, Nc:])
+    assert torch.equal(lse_c, lse_full[:, :, Nc:])
+
+
+def test_condition_rows_ignore_noise_tokens(api):
+    w = SMALL["small_i2v"]
+    inputs = synthetic.make_inputs(w)
+    out1, lse1 = run_gpu(api, w, inputs)
+    Nc = w.n_cond_tokens
+    g = torch.Generator().manual_seed(77)
+    pert = {k: v.clone() for k, v in inputs.items()}
+    for k in ("q", "k", "v"):
+        pert[k][:, Nc:] = torch.randn(pert[k][:, Nc:].shape, generator=g).to(pert[k].dtype)
+    out2, lse2 = run_gpu(api, w, pert)
+    assert torch.equal(out1[:, :Nc], out2[:, :Nc])
+    assert torch.equal(lse1[:, :, :Nc], lse2[:, :, :Nc])
+    assert not torch.equal(out1[:, Nc:], out2[:, Nc:])
+
+
+def test_deterministic(api):
+    w = SMALL["ragged"]
+    inputs = synthetic.make_inputs(w)
+    a, la = run_gpu(api, w, inputs)
+    b, lb = run_gpu(api, w, inputs)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+FULL = ["i2v_480p", "refine_720p", "continuation_cached", "sweep_l2s8", "sweep_l1s32",
+        "sweep_dense"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_rows(api, name):
+    """Full-size workloads in the benchmark's launch configuration; every head
+    on a fixed sample of query rows (see parity.sample_rows)."""
+    w = synthetic.get(name)
+    inputs = synthetic.make_inputs(w)
+    out, lse = run_gpu(api, w, inputs)
+    assert torch.isfinite(out.float()).all() and torch.isfinite(lse).all()
+    nrand = 8 if name == "sweep_dense" else 64
+    rows = parity.sample_rows(w, n_random_blocks=nrand)
+    ref_out, ref_lse = parity.oracle_rows(w, inputs, rows)
+    mx, mean, lerr = parity.compare(w, out, lse, ref_out, ref_lse, rows)
+    print("%s rows=%d x %d heads: max %.3g mean %.3g lse %.3g" % (name, len(rows), w.heads, mx,
+                                                                  mean, lerr))
+
+
+def test_argument_errors_on_gpu(api):
+    w = SMALL["small_i2v"]
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    other = api.Rope3D(w.T, w.H, w.W + 1)
+    q = torch.randn(1, w.n_tokens, w.heads, 64, device="cuda").bfloat16()
+    with pytest.raises(api.LcError) as e:
+        api.forward(q, q, q, plan, other)
+    assert e.value.status == api.LC_ERR_INVALID_ARGUMENT
+    # a pointer that is not 16-byte aligned
+    buf = torch.empty(w.n_tokens * w.heads * 64 + 8, device="cuda", dtype=torch.bfloat16)
+    mis = buf[1:1 + w.n_tokens * w.heads * 64].view(1, w.n_tokens, w.heads, 64)
+    with pytest.raises(api.LcError) as e:
+        api.forward(mis, q, q, plan, rope)
+    assert e.value.status == api.LC_ERR_INVALID_ARGUMENT
+    assert api.last_device_status() == 0
+
+
+def test_watchdog_gives_up_and_context_survives(api):
+    """A bounded wait on a barrier that nothing arrives on reports a timeout
+    instead of hanging; the context keeps working afterwards."""
+    assert api.watchdog_selftest(20000) == api.LC_ERR_TIMEOUT
+    assert api.last_device_status() == 0
+    w = SMALL["one_block"]
+    inputs = synthetic.make_inputs(w)
+    out, lse = run_gpu(api, w, inputs)
+    ref_out, ref_lse = full_oracle(w, inputs)
+    check_all_rows(w, out, lse, ref_out, ref_lse)

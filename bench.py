@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of block-sparse 3D-RoPE attention (one attention layer per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload i2v_480p] [--sweep] [--no-cpu-baseline]
+
+One step = one lc_bsa_forward call over one layer: B=1 per GPU, 32 heads x 64,
+the 480x832 93-frame image-to-video latent (24x30x52 = 37,440 tokens, first
+frame = condition, local=2, stride=4) unless --workload says otherwise.  The
+metric is attended TFLOP/s (4 * head_dim * heads * attended token pairs per
+second) with ms per layer and the fraction of the measured bf16 dense tensor
+peak.  Inputs (q, k, v: 153 MB each) are larger than the 126 MB L2, so no
+flush is needed between steps.  With N > 1 (torchrun) every rank runs its own
+batch element (weak scaling, no collective on the data path); the time is the
+max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+project) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn ms/layer, attended TFLOP/s, % bf16 tensor peak @37k/86k tok"
+UNIT = "attended TFLOP/s"
+KERNEL_SRC = os.path.join(ROOT, "block_sparse_attention_rope_b200", "csrc", "attn_sm100.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAK_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="i2v_480p")
+    ap.add_argument("--sweep", action="store_true", help="also time the sparsity sweep")
+    ap.add_argument("--no-extra", action="store_true", help="skip the 86,400-token line")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    return FALLBACK_PEAK_TFLOPS, "fallback 1.59 PFLOP/s"
+
+
+def kernel_hash() -> str:
+    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+
+
+def traffic_for(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    e = d.get(workload)
+    if not e or e.get("kernel_sha") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every 10 ms."""
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover
+            self.nv, self.err = None, str(e)
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+            "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for n, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ----------------------------------------------------------------------------- ours
+def time_forward(api, torch, w, d, plan, rope, steps, warmup, dist, stream):
+    """Device time of `steps` back-to-back forward calls, bracketed by a
+    barrier and synchronisations; per-launch CUDA events on the launching
+    stream.  Returns (max-over-ranks total ms, mean per-launch ms)."""
+    out = torch.empty_like(d["q"])
+    call = (lambda: api.forward_cached(d["q"], d["k"], d["v"], d["cond_k"], d["cond_v"], plan,
+                                       rope, out=out, stream=stream)) if w.cached else \
+        (lambda: api.forward(d["q"], d["k"], d["v"], plan, rope, out=out, stream=stream))
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            call()
+    torch.cuda.synchronize()
+    if api.last_device_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i in range(steps):
+            call()
+            evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+    total = evs[0].elapsed_time(evs[-1])
+    if dist is not None:
+        t = torch.tensor([total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    st = api.last_device_status()
+    if st != 0:
+        raise RuntimeError("device status %d after the timed region" % st)
+    return total, sum(per) / len(per), out
+
+
+def time_e2e(api, torch, w, host, plan, rope, steps, stream):
+    """End to end through the public API: pinned host inputs -> device ->
+    forward -> result back to pinned host memory, every step."""
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    out_h = torch.empty_like(host["q"]).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for k, v in host.items():
+            dev[k].copy_(v, non_blocking=True)
+        if w.cached:
+            o = api.forward_cached(dev["q"], dev["k"], dev["v"], dev["cond_k"], dev["cond_v"],
+                                   plan, rope, stream=stream)
+        else:
+            o = api.forward(dev["q"], dev["k"], dev["v"], plan, rope, stream=stream)
+        out_h.copy_(o, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, stream, e2e_steps=0):
+    w = synthetic.get(name)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    info = plan.info()
+    pairs = info.attended_token_pairs_noisy if w.cached else info.attended_token_pairs
+    flops = 4.0 * w.head_dim * w.heads * w.batch * pairs
+    host = synthetic.make_inputs(w, seed_offset=rank)
+    host = {k: v.pin_memory() for k, v in host.items()}
+    d = {k: v.cuda() for k, v in host.items()}
+    total_ms, launch_ms, out = time_forward(api, torch, w, d, plan, rope, steps, warmup, dist,
+                                            stream)
+    res = {"w": w, "flops": flops, "pairs": pairs, "total_ms": total_ms, "launch_ms": launch_ms,
+           "nnz": info.nnz}
+    if e2e_steps:
+        del d, out
+        torch.cuda.empty_cache()
+        res["e2e_ms"], res["h2d"], res["d2h"] = time_e2e(api, torch, w, host, plan, rope,
+                                                         e2e_steps, stream)
+    return res
+
+
+def oracle_sample(w, x, heads, row_stride):
+    """Time the fp64 oracle, as it stands, on `heads` (one at a time: a head
+    is an independent unit of the layer) x every `row_stride`-th query row.
+    The oracle's own RoPE of that head's q and k is inside the timed region.
+    Returns (attended TFLOP/s, seconds, threads, attended pairs)."""
+    import numpy as np
+
+    import oracle
+    Nc, Nn, Cb, Nb = oracle.segment_sizes(w.T, w.H, w.W, w.n_cond)
+    if w.cached:
+        k = np.concatenate([oracle._f64(x["cond_k"]), oracle._f64(x["k"])], axis=1)
+        v = np.concatenate([oracle._f64(x["cond_v"]), oracle._f64(x["v"])], axis=1)
+        q, q_off, nq = oracle._f64(x["q"]), Nc, Nn
+    else:
+        q, k, v = oracle._f64(x["q"]), oracle._f64(x["k"]), oracle._f64(x["v"])
+        q_off, nq = 0, w.n_tokens
+    rows = np.arange(0, nq, row_stride)
+    trip = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1)
+    # attended keys of the sampled rows, from the oracle's block CSR
+    rp, ci = oracle.block_csr(w.T, w.H, w.W, w.block, w.local, w.stride, w.n_cond)
+    bsize = np.array([min(64, Nc - 64 * b) for b in range(Cb)] +
+                     [min(64, Nn - 64 * j) for j in range(Nb)], dtype=np.int64)
+    keys = np.array([bsize[ci[rp[i]:rp[i + 1]]].sum() for i in range(Cb + Nb)])
+    tok = rows + q_off
+    qb = np.where(tok < Nc, tok // 64, Cb + (tok - Nc) // 64)
+    pairs = int(keys[qb].sum()) * len(heads)
+    sec = 0.0
+    for h in heads:
+        qh, kh, vh = (np.ascontiguousarray(a[:, :, h:h + 1]) for a in (q, k, v))
+        t0 = time.perf_counter()
+        oracle.attention_rows(qh, kh, vh, H=w.H, W=w.W, Nc=Nc, block=w.block, local=w.local,
+                              stride=w.stride, rows=trip, q_offset=q_off)
+        sec += time.perf_counter() - t0
+    return 4.0 * w.head_dim * pairs / sec / 1e12, sec, oracle.max_threads(), pairs
+
+
+def cpu_baseline(name: str):
+    """The oracle on a bounded sample of the workload (about 10-30 s of CPU
+    work on the benchmark host): 8 heads x every 6th query row."""
+    from block_sparse_attention_rope_b200 import synthetic
+    w = synthetic.get(name)
+    x = synthetic.make_inputs(w)
+    heads, stride = list(range(8)), 6
+    tf, sec, threads, pairs = oracle_sample(w, x, heads, stride)
+    sample = ("fp64 oracle (C, OpenMP) on heads 0-7 x every %dth query row of %s "
+              "(%.3g attended token pairs, RoPE of those heads included), %.1f s" %
+              (stride, name, pairs, sec))
+    return tf, sec, threads, sample
+
+
+def run_ours(a):
+    import torch
+    world, rank, local = dist_env()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    from block_sparse_attention_rope_b200 import api, synthetic
+    stream = torch.cuda.Stream()
+    peak, peak_src = peaks()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    nvml_index = int(vis.split(",")[local]) if vis else local
+    with ClockSampler(nvml_index) as clk:
+        main = measure_workload(api, synthetic, torch, a.workload, a.steps, a.warmup, dist, rank,
+                                stream)
+    clocks = clk.summary()
+    e2e = None
+    if a.e2e_steps > 0:
+        w = main["w"]
+        res = measure_workload(api, synthetic, torch, a.workload, 1, 1, dist, rank, stream,
+                               e2e_steps=a.e2e_steps)
+        e2e_ms = res["e2e_ms"]
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": round(world * res["flops"] / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": res["h2d"],
+               "d2h_bytes_per_step": res["d2h"],
+               "path": "pinned host q/k/v -> device, lc_bsa_forward, out -> pinned host"}
+    extra = {}
+    names = [] if a.no_extra else ["refine_720p"]
+    if a.sweep:
+        names += ["continuation_cached"] + ["sweep_" + s for s in
+                                            ("dense", "l2s4", "l2s8", "l1s16", "l1s32")]
+    for n in names:
+        if n == a.workload:
+            continue
+        r = measure_workload(api, synthetic, torch, n, max(10, a.steps // 2), a.warmup, dist, rank,
+                             stream)
+        ms = r["total_ms"] / max(10, a.steps // 2)
+        extra[n] = {"tokens": r["w"].n_tokens, "ms_per_layer": round(ms, 4),
+                    "attended_tflops": round(r["flops"] / (ms * 1e-3) / 1e12, 2),
+                    "pct_bf16_peak": round(100.0 * r["flops"] / (r["launch_ms"] * 1e-3) / 1e12 / peak, 2),
+                    "attended_pairs_per_head": r["pairs"]}
+    w = main["w"]
+    ms = main["total_ms"] / a.steps
+    value = world * main["flops"] * a.steps / (main["total_ms"] * 1e-3) / 1e12
+    achieved = main["flops"] / (main["launch_ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) q/k/v, bf16)",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "n_cond_frames": w.n_cond,
+                   "tokens": w.n_tokens, "heads": w.heads, "head_dim": w.head_dim, "block": w.block,
+                   "local": w.local, "stride": w.stride, "batch_per_gpu": w.batch,
+                   "global_batch": w.batch * world,
+                   "parallelism": "replicas: one batch element per GPU, no data-path collective",
+                   "l2": "inputs larger than L2 (q, k, v 153 MB each); no flush"},
+        "pct_bf16_peak": round(100.0 * achieved / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src, "traffic": traffic_for(w.name),
+                     "kernel": "bsa_sm100_kernel",
+                     "algorithmic": "4*64*32*%d FLOP per launch" % main["pairs"]},
+        "gpu_launches": a.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "extra": extra,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        tf, sec, threads, sample = cpu_baseline(a.workload)
+        line["cpu_baseline"] = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": sample, "seconds": round(sec, 2)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(a):
+    """The project's reference arm: the fp64 oracle on the host cores.  Each
+    step is one head of the workload (cycling through the heads), every 16th
+    query row, so that --steps K finishes in a few minutes.  Under torchrun
+    only rank 0 works."""
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    from block_sparse_attention_rope_b200 import synthetic
+    w = synthetic.get(a.workload)
+    x = synthetic.make_inputs(w)
+    for i in range(a.warmup):
+        oracle_sample(w, x, [i % w.heads], 64)
+    secs, pairs_tot, threads = 0.0, 0, 1
+    for i in range(a.steps):
+        tf, sec, threads, pairs = oracle_sample(w, x, [i % w.heads], 16)
+        secs += sec
+        pairs_tot += pairs
+    tf = 4.0 * w.head_dim * pairs_tot / secs / 1e12
+    sample = ("fp64 oracle (C, OpenMP): %d steps of one head x every 16th query row of %s, "
+              "RoPE of the head included" % (a.steps, w.name))
+    line = {"metric": METRIC, "value": tf, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": round(1e3 * secs / a.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) q/k/v, bf16 values upcast to f64)",
+            "impl": "reference",
+            "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W,
+                       "n_cond_frames": w.n_cond, "tokens": w.n_tokens, "heads": w.heads,
+                       "head_dim": w.head_dim, "local": w.local, "stride": w.stride},
+            "cpu_baseline": {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -53,6 +53,7 @@ def _load():
         "lc_rope3d_apply": (S, [vp, vp, I, LL, I, I, LL, I, vp, vp]),
         "lc_bsa_forward": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_bsa_forward_cached": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_bsa_forward_noalloc": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
         "lc_status_string": (ctypes.c_char_p, [S]),
@@ -250,6 +251,28 @@ def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Op
                                      _dtype_code(q), float(softmax_scale), plan.handle,
                                      rope.handle, _stream(stream)), "lc_bsa_forward_cached")
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D,
+                    *, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                    softmax_scale: float = 0.0, stream=None):
+    """lc_bsa_forward_noalloc: the same attention as `forward` for callers
+    that must not allocate device memory during the call; the caller passes
+    `out` (and `lse` if wanted).  The library's scheduler counter lives in a
+    fixed per-device array, so calls on one device must not overlap on the
+    GPU; the first call on a device should come before any stream capture."""
+    B, N, heads, hd = q.shape
+    for name, t in (("k", k), ("v", v)):
+        _check_bmhk(name, t, q.shape, q.dtype)
+    _check_bmhk("q", q, (B, plan.n_tokens, heads, hd), q.dtype)
+    _check_bmhk("out", out, q.shape, q.dtype)
+    if lse is not None:
+        _check_bmhk("lse", lse, (B, heads, N), torch.float32)
+    _check(lib.lc_bsa_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                      _ptr(lse), B, heads, hd, _dtype_code(q),
+                                      float(softmax_scale), plan.handle, rope.handle,
+                                      _stream(stream)), "lc_bsa_forward_noalloc")
+    return out
 
 
 def last_device_status(stream=None) -> int:

@@ -96,15 +96,47 @@ extern "C" lc_status lc_bsa_forward_cached(const void *q, const void *k, const v
                      softmax_scale, plan, rope, stream, true);
 }
 
+extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const void *v,
+                                            void *out, float *lse, int batch, int heads,
+                                            int head_dim, lc_dtype dtype, float softmax_scale,
+                                            lc_bsa_plan plan, lc_rope3d rope, void *stream) {
+  lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
+  if (s != LC_OK) return s;
+  if (!q || !k || !v || !out) return LC_ERR_INVALID_ARGUMENT;
+  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return LC_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;
+  // The scheduler counter in the fixed scratch is a 32-bit int: one launch
+  // may hand out at most 2^31 - 1 work items (batch x heads x query groups).
+  if ((long long)batch * heads * plan->G >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
+  float scale = softmax_scale > 0.f ? softmax_scale : 0.125f;
+  int *scratch = lc_noalloc_scratch(&s);  // first call on a device: symbol lookup
+  if (s != LC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == LC_DTYPE_F32)  // the fp32 kernel needs no scratch
+    return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
+                                 static_cast<const float *>(v), nullptr, nullptr,
+                                 static_cast<float *>(out), lse, batch, heads, scale, false, plan,
+                                 rope, scratch + 1, st);
+  return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale, false,
+                                 plan, rope, scratch + 1, st, scratch);
+}
+
 extern "C" lc_status lc_last_device_status(void *stream) {
   lc_status s;
   int *p = lc_device_status_ptr(&s);
   if (s != LC_OK) return s;
+  int *na = lc_noalloc_scratch(&s);
+  if (s != LC_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   LC_CUDA_TRY(cudaStreamSynchronize(st));
-  int word = 0;
+  int word = 0, word_na = 0;
   LC_CUDA_TRY(cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost));
+  LC_CUDA_TRY(cudaMemcpy(&word_na, na + 1, sizeof(int), cudaMemcpyDeviceToHost));
   LC_CUDA_TRY(cudaMemset(p, 0, sizeof(int)));
+  LC_CUDA_TRY(cudaMemset(na + 1, 0, sizeof(int)));
+  word |= word_na;
   if (word & LC_DEVSTAT_TIMEOUT) return LC_ERR_TIMEOUT;
   if (word & LC_DEVSTAT_CHECK) return LC_ERR_DEVICE_CHECK;
   return LC_OK;

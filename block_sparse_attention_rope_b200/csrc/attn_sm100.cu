@@ -750,10 +750,46 @@ __global__ void watchdog_selftest_kernel(int *status, long long timeout_ns) {
 
 }  // namespace
 
+// ------------------------------------------------------------ no-alloc scratch
+// Fixed device scratch for lc_bsa_forward_noalloc, for callers that must not
+// allocate device memory.  Word 0 is the work-item counter of the persistent
+// scheduler, word 1 the status word the bounded waits report into; the rest
+// is reserved.  Every GPU that loads the library holds these 256 bytes until
+// the process exits.  In host code the symbol is only a stand-in, so its
+// device address is looked up once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) int g_lc_noalloc_scratch[LC_NOALLOC_SCRATCH_INTS];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+int *g_noalloc_ptr[kNoallocMaxDevices] = {nullptr};
+}  // namespace
+
+int *lc_noalloc_scratch(lc_status *st) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) {
+    *st = LC_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_lc_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      *st = LC_ERR_CUDA;
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = static_cast<int *>(p);
+  }
+  *st = LC_OK;
+  return g_noalloc_ptr[dev];
+}
+
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, const void *cond_k,
                                   const void *cond_v, void *out, float *lse, int batch, int heads,
                                   float scale, bool cached, const lc_bsa_plan_s *plan,
-                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream) {
+                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
+                                  int *counter_scratch) {
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
   const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
@@ -820,6 +856,16 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
   const int grid = (int)(total < n_sm ? total : n_sm);
 
+  if (counter_scratch) {  // caller-provided scratch: nothing is allocated
+    prm.work_counter = counter_scratch;
+    cudaError_t e = cudaMemsetAsync(counter_scratch, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
+    if (e == cudaSuccess) {
+      bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+      e = cudaGetLastError();
+    }
+    return lc_from_cuda(e);
+  }
   int *counter = nullptr;
   LC_CUDA_TRY(cudaMallocAsync(&counter, sizeof(int), stream));
   prm.work_counter = counter;

@@ -93,9 +93,17 @@ lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 float *lse, int batch, int heads, float scale, bool cached,
                                 const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
                                 int *dev_status, cudaStream_t stream);
+// counter_scratch: NULL = allocate the scheduler counter stream-ordered for
+// this launch; else a device int the caller provides (lc_bsa_forward_noalloc).
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
                                   const void *cond_k, const void *cond_v, void *out,
                                   float *lse, int batch, int heads, float scale, bool cached,
                                   const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                  int *dev_status, cudaStream_t stream);
+                                  int *dev_status, cudaStream_t stream,
+                                  int *counter_scratch = nullptr);
+
+// Fixed scratch of lc_bsa_forward_noalloc (attn_sm100.cu): device address of
+// g_lc_noalloc_scratch on the current device, looked up once per device.
+#define LC_NOALLOC_SCRATCH_INTS 64
+int *lc_noalloc_scratch(lc_status *st);
 lc_status lc_launch_watchdog_selftest(int *dev_status, long long timeout_ns, cudaStream_t stream);

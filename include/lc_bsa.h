@@ -177,6 +177,32 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
                                 lc_rope3d rope, void *stream);
 
 /*
+ * lc_bsa_forward_noalloc -- lc_bsa_forward for callers that cannot allocate
+ * device memory during the call: an application whose allocator owns all of
+ * the GPU's memory up front, a serving loop that forbids allocations after
+ * warm-up, or code that must not add memory operations to a stream.  (The
+ * pages describe no such entry point; it is an addition of this library.)
+ * Same arguments, layouts, results and errors as lc_bsa_forward.  It allocates
+ * nothing: the tensor-core kernel's scheduler counter and status word live in
+ * a fixed 256-byte device array inside the library (64 ints, of which a call
+ * uses 2), which every GPU that loads the library keeps until the process
+ * exits.  One launch can hand out at most 2^31 - 1 work items (batch x heads
+ * x groups of 4 query blocks); larger requests return LC_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share that device's array, which keeps the last
+ *     call's contents; each call clears the counter on its stream before its
+ *     kernel starts.  Calls on one device that overlap on the GPU (for
+ *     example on two streams) race on the counter: serialise them.
+ *   - In-kernel timeouts are reported by lc_last_device_status like the
+ *     other entry points'.
+ */
+lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const void *v, void *out,
+                                 float *lse, int batch, int heads, int head_dim, lc_dtype dtype,
+                                 float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
+                                 void *stream);
+
+/*
  * lc_last_device_status -- synchronise `stream`, then report and clear the
  * current device's status word, which the kernels set when a bounded wait
  * timed out (LC_ERR_TIMEOUT) or an in-kernel check failed

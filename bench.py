@@ -171,6 +171,7 @@ def time_forward(api, torch, w, d, plan, rope, steps, warmup, dist, stream):
     st = api.last_device_status()
     if st != 0:
         raise RuntimeError("device status %d after the timed region" % st)
+    time_forward.last_spread = (min(per), statistics.median(per), max(per))
     return total, sum(per) / len(per), out
 
 
@@ -217,6 +218,7 @@ def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, str
     total_ms, launch_ms, out = time_forward(api, torch, w, d, plan, rope, steps, warmup, dist,
                                             stream)
     res = {"w": w, "flops": flops, "pairs": pairs, "total_ms": total_ms, "launch_ms": launch_ms,
+           "spread": [round(x, 4) for x in time_forward.last_spread],
            "nnz": info.nnz}
     if e2e_steps:
         del d, out
@@ -325,7 +327,8 @@ def run_ours(a):
         extra[n] = {"tokens": r["w"].n_tokens, "ms_per_layer": round(ms, 4),
                     "attended_tflops": round(r["flops"] / (ms * 1e-3) / 1e12, 2),
                     "pct_bf16_peak": round(100.0 * r["flops"] / (r["launch_ms"] * 1e-3) / 1e12 / peak, 2),
-                    "attended_pairs_per_head": r["pairs"]}
+                    "attended_pairs_per_head": r["pairs"],
+                    "launch_ms_min_median_max": r["spread"]}
     w = main["w"]
     ms = main["total_ms"] / a.steps
     value = world * main["flops"] * a.steps / (main["total_ms"] * 1e-3) / 1e12
@@ -342,6 +345,7 @@ def run_ours(a):
                    "parallelism": "replicas: one batch element per GPU, no data-path collective",
                    "l2": "inputs larger than L2 (q, k, v 153 MB each); no flush"},
         "pct_bf16_peak": round(100.0 * achieved / peak, 2),
+        "launch_ms_min_median_max": main["spread"],
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": peak_src, "traffic": traffic_for(w.name),

@@ -15,7 +15,8 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "liblcbsa.so")
+# LC_BSA_LIB may name another build of the same library (same ABI).
+LIB_PATH = os.environ.get("LC_BSA_LIB") or os.path.join(_HERE, "liblcbsa.so")
 
 LC_OK, LC_ERR_INVALID_ARGUMENT, LC_ERR_UNSUPPORTED, LC_ERR_CUDA = 0, 1, 2, 3
 LC_ERR_OUT_OF_MEMORY, LC_ERR_TIMEOUT, LC_ERR_DEVICE_CHECK = 4, 5, 6

@@ -14,17 +14,19 @@
 //               its two 128-row query tiles Q0, Q1 share one key list, the
 //               sorted union of the member blocks' lists, walked two key
 //               blocks (128 keys) at a time.
-//   warp 8      TMA producer: Q tiles, then the listed K and V blocks into a
-//               3-stage ring (missing second block = out-of-range box, which
-//               TMA fills with zeros).
-//   warps 10-11 RoPE: rotate every freshly loaded Q and K tile in shared
-//               memory (128-byte swizzled rows, cos/sin tables in smem).
+//   warp 8      TMA producer: Q tiles (double-buffered across items), then the
+//               listed K and V blocks into a 3-stage ring (a missing second
+//               block is an out-of-range box, which TMA fills with zeros).
+//   warps 10-11 RoPE: rotate every freshly loaded Q tile, and K tile unless K
+//               was rotated beforehand, in shared memory (128-byte swizzled
+//               rows, cos/sin tables in smem), one token row per thread.
 //   warp 9      MMA issuer (one thread): S_i = Q_i K^T (M=128, N=128, K=64)
 //               into TMEM, O_i += P_i V (A = P from TMEM, M=128, N=64).
 //   warps 0-3 / 4-7  softmax of Q0 / Q1, one TMEM lane (= query row) per
 //               thread: mask, running max with lazy rescaling (threshold 2^8),
-//               exp2, row sum, P as bf16 into TMEM; at the end O / l through
-//               shared memory to a TMA store, plus the log-sum-exp.
+//               exp2 (part on the MUFU unit, part as a polynomial on the FMA
+//               pipe), packed f32x2 sums, P as bf16 into TMEM; at the end
+//               O / l through shared memory to a TMA store, plus the LSE.
 //   TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384)
 //               P0 [384,448) P1 [448,512).
 // Every wait on an mbarrier is bounded (globaltimer); on expiry the kernel
@@ -34,7 +36,6 @@
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
-
 #include <string.h>
 
 #include <mutex>
@@ -58,6 +59,20 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 320, kColP0 
 constexpr uint32_t kIdescQK = lcptx::idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdescPV = lcptx::idesc_bf16_f32(128, 64, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p stays below 2^8 before a rescale
+#ifndef LC_REGS_SOFTMAX
+#define LC_REGS_SOFTMAX 200
+#define LC_REGS_OTHER 104
+#endif
+constexpr int kRegsSoftmax = LC_REGS_SOFTMAX, kRegsOther = LC_REGS_OTHER;
+static_assert(2 * 128 * LC_REGS_SOFTMAX + 128 * LC_REGS_OTHER <= 65536, "register split");
+// Registers per thread the kernel must be launched with for that split.
+constexpr int kRegsAtLaunchMin = (256 * kRegsSoftmax + 128 * kRegsOther + kThreads - 1) / kThreads;
+// Of every 8 column pairs of a row, the pairs whose bit is set here take the
+// polynomial exp2 on the FMA pipe; the others take MUFU ex2.
+#ifndef LC_POLY_EXP2_MASK
+#define LC_POLY_EXP2_MASK 0x00u
+#endif
+constexpr uint32_t kPolyMask = LC_POLY_EXP2_MASK;
 
 struct __align__(64) Sm100Params {
   CUtensorMap tmQ[2], tmK[2], tmV[2], tmO[2];  // [0] condition segment, [1] noisy segment
@@ -73,16 +88,17 @@ struct __align__(64) Sm100Params {
   int T, H, W;
   int Nc, Nn, Cb, gc;
   int heads, n_groups_active, total_items;
-  int lse_nq;          // rows of the lse tensor per (batch, head)
+  int lse_nq;              // rows of the lse tensor per (batch, head)
   int q_row_offset_noisy;  // row of the q/out/lse tensors holding noisy token 0
   int tab_floats;
+  int k_prerotated;        // K tensors already hold R(k): skip the K rotation
   float scale_log2;
 };
 
 // Shared memory carve-up (offsets from a 1024-aligned base).
 struct SmemOffsets {
-  static constexpr int q = 0;                                  // 2 tiles
-  static constexpr int k = q + 2 * kTileBytes;                 // kStages tiles
+  static constexpr int q = 0;                                  // [2 items][2 tiles]
+  static constexpr int k = q + 4 * kTileBytes;                 // kStages tiles
   static constexpr int v = k + kStages * kTileBytes;           // kStages tiles
   static constexpr int bars = v + kStages * kTileBytes;        // mbarriers
   static constexpr int n_bars = 64;
@@ -92,21 +108,21 @@ struct SmemOffsets {
 
 // Barrier indices.
 enum {
-  B_QFULL = 0,   // [2] TMA Q landed
-  B_QREADY = 2,  // [2] Q rotated
-  B_QEMPTY = 4,  // [2] Q buffer (and O staging) free
-  B_KFULL = 6,   // [kStages]
-  B_KREADY = 6 + kStages,
-  B_KEMPTY = 6 + 2 * kStages,
-  B_VFULL = 6 + 3 * kStages,
-  B_VEMPTY = 6 + 4 * kStages,
-  B_SFULL = 6 + 5 * kStages,  // [2]
-  B_SFREE = B_SFULL + 2,      // [2]
-  B_PFULL = B_SFREE + 2,      // [2]
-  B_ODONE = B_PFULL + 2,      // [2]
-  B_EPI = B_ODONE + 2,        // [2] O rows staged in smem
-  B_SCHED_FULL = B_EPI + 2,   // [2]
-  B_SCHED_EMPTY = B_SCHED_FULL + 2,  // [2]
+  B_QFULL = 0,    // [buf*2 + i] TMA Q landed
+  B_QREADY = 4,   // [buf*2 + i] Q rotated
+  B_QEMPTY = 8,   // [buf*2 + i] Q buffer (and O staging) free
+  B_KFULL = 12,   // [kStages]
+  B_KREADY = B_KFULL + kStages,
+  B_KEMPTY = B_KFULL + 2 * kStages,
+  B_VFULL = B_KFULL + 3 * kStages,
+  B_VEMPTY = B_KFULL + 4 * kStages,
+  B_SFULL = B_KFULL + 5 * kStages,  // [2]
+  B_SFREE = B_SFULL + 2,            // [2]
+  B_PFULL = B_SFREE + 2,            // [2]
+  B_ODONE = B_PFULL + 2,            // [2]
+  B_EPI = B_ODONE + 2,              // [2] O rows staged in smem
+  B_SCHED_FULL = B_EPI + 2,         // [2]
+  B_SCHED_EMPTY = B_SCHED_FULL + 2, // [2]
   B_DRAIN = B_SCHED_EMPTY + 2,
   B_COUNT = B_DRAIN + 1
 };
@@ -123,8 +139,8 @@ struct Ctx {
 
 // Bounded wait: true when the phase of `parity` completed; false when the CTA
 // aborted or this wait timed out (which sets the abort flag and the status).
-__device__ __noinline__ bool wait_bar(const Ctx &c, uint32_t bar, uint32_t parity) {
-  if (lcptx::mbar_try_wait(bar, parity)) return true;
+// (Everything is inlined: register-split regions must not contain calls.)
+__device__ __forceinline__ bool wait_bar_slow(const Ctx &c, uint32_t bar, uint32_t parity) {
   uint64_t t0 = lcptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (lcptx::mbar_try_wait(bar, parity)) return true;
@@ -138,6 +154,11 @@ __device__ __noinline__ bool wait_bar(const Ctx &c, uint32_t bar, uint32_t parit
       }
     }
   }
+}
+
+__device__ __forceinline__ bool wait_bar(const Ctx &c, uint32_t bar, uint32_t parity) {
+  if (lcptx::mbar_try_wait(bar, parity)) return true;
+  return wait_bar_slow(c, bar, parity);
 }
 
 // Warp-uniform form for warps whose lanes then run .sync.aligned tcgen05 ops
@@ -183,43 +204,63 @@ __device__ __forceinline__ void entry_block(const Sm100Params &p, uint32_t e, in
   }
 }
 
+// Entries of an item's list, fetched 32 at a time by a whole warp: lane i
+// holds entry 32*chunk + i; the next chunk is prefetched one chunk ahead.
+struct EntryStream {
+  uint32_t cur, nxt;
+  int len;
+  const uint32_t *ent;
+  __device__ __forceinline__ void start(const uint32_t *e, int n, int lane) {
+    ent = e;
+    len = n;
+    cur = lane < n ? __ldg(e + lane) : 0u;
+    nxt = 32 + lane < n ? __ldg(e + 32 + lane) : 0u;
+  }
+  // Entries 2t and 2t+1 (the second is 0 past the end).
+  __device__ __forceinline__ void pair(int t, int lane, uint32_t &a, uint32_t &b) {
+    const int i = (2 * t) & 31;
+    if (t > 0 && i == 0) {
+      cur = nxt;
+      const int j = 2 * t + 32 + lane;
+      nxt = j < len ? __ldg(ent + j) : 0u;
+    }
+    a = __shfl_sync(0xffffffffu, cur, i);
+    b = __shfl_sync(0xffffffffu, cur, i + 1);
+    if (2 * t + 1 >= len) b = 0u;
+  }
+};
+
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Rotate rows [r_begin, r_end) of a swizzled 64-channel bf16 tile in place;
-// tile row r holds sequence token tok0 + r.  Threads of the RoPE warps split
-// the (row, 16-byte chunk) pairs.
-__device__ __forceinline__ void rope_tile(uint8_t *tile, int r_begin, int r_end, int tok0,
-                                          const float *tab, const Sm100Params &p, int rt) {
-  const float *cT = tab, *sT = tab + p.T * 8;
-  const float *cH = sT + p.T * 8, *sH = cH + p.H * 12;
-  const float *cW = sH + p.H * 12, *sW = cW + p.W * 12;
-  const int jobs = (r_end - r_begin) * 8;
-  for (int j = rt; j < jobs; j += kRopeThreads) {
-    int r = r_begin + (j >> 3), ch = j & 7;
-    int n = tok0 + r;
-    int t = lc_div(n, p.div_hw);
-    int rem = n - t * p.div_hw.d;
-    int hh = lc_div(rem, p.div_w);
-    int w = rem - hh * p.div_w.d;
-    const float *c, *s;
-    if (ch < 2) { c = cT + t * 8 + 4 * ch; s = sT + t * 8 + 4 * ch; }
-    else if (ch < 5) { c = cH + hh * 12 + 4 * (ch - 2); s = sH + hh * 12 + 4 * (ch - 2); }
-    else { c = cW + w * 12 + 4 * (ch - 5); s = sW + w * 12 + 4 * (ch - 5); }
-    float4 cc = *reinterpret_cast<const float4 *>(c);
-    float4 ss = *reinterpret_cast<const float4 *>(s);
-    uint4 *ptr = reinterpret_cast<uint4 *>(tile + swz(r, ch));
+// Rotate one token row (64 bf16 channels, 128-byte swizzled) in place.
+__device__ __forceinline__ void rope_row(uint8_t *tile, int r, int n, const float *tab,
+                                         const Sm100Params &p) {
+  const int t = lc_div(n, p.div_hw);
+  const int rem = n - t * p.div_hw.d;
+  const int hh = lc_div(rem, p.div_w);
+  const int w = rem - hh * p.div_w.d;
+  const float *cT = tab + t * 8, *sT = tab + p.T * 8 + t * 8;
+  const float *cH = tab + p.T * 16 + hh * 12, *sH = cH + p.H * 12;
+  const float *cW = tab + p.T * 16 + p.H * 24 + w * 12, *sW = cW + p.W * 12;
+  uint8_t *rowp = tile + r * 128;
+  const int x = r & 7;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    const float *c = ch < 2 ? cT + 4 * ch : (ch < 5 ? cH + 4 * (ch - 2) : cW + 4 * (ch - 5));
+    const float *s = ch < 2 ? sT + 4 * ch : (ch < 5 ? sH + 4 * (ch - 2) : sW + 4 * (ch - 5));
+    const float4 cc = *reinterpret_cast<const float4 *>(c);
+    const float4 ss = *reinterpret_cast<const float4 *>(s);
+    uint4 *ptr = reinterpret_cast<uint4 *>(rowp + ((ch ^ x) << 4));
     uint4 raw = *ptr;
     uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
     const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 v2 = *reinterpret_cast<__nv_bfloat162 *>(&wds[q]);
-      float2 f = __bfloat1622float2(v2);
-      float a = f.x * cs[q] - f.y * sn[q];
-      float b = f.x * sn[q] + f.y * cs[q];
-      __nv_bfloat162 o2 = __floats2bfloat162_rn(a, b);
+      const float a = __uint_as_float(wds[q] << 16);
+      const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
+      __nv_bfloat162 o2 = __floats2bfloat162_rn(a * cs[q] - b * sn[q], a * sn[q] + b * cs[q]);
       wds[q] = *reinterpret_cast<uint32_t *>(&o2);
     }
     *ptr = make_uint4(wds[0], wds[1], wds[2], wds[3]);
@@ -232,9 +273,99 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x on the FMA pipe, two lanes at once: x = n + f with n = rint(x) (by the
+// 1.5*2^23 rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-3
+// polynomial fitted here by the Remez exchange for least maximum relative
+// error (7.5e-5, far below bf16's 2^-9); 2^n by adding n to the exponent
+// field.  Inputs below -126 are clamped (the result is then < 2^-125).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -126.f);
+  x.y = fmaxf(x.y, -126.f);
+  const float2 rnd = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(x, rnd);
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f,
+                        make_float2(0.242611125f, 0.242611125f));
+  p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
+  p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
+  float2 r;
+  r.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
+  r.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Maximum of a 128-column score row: 8 independent chains of 3-input maxima.
+__device__ __forceinline__ float row_max(const float (&s)[128]) {
+  float mc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) mc[c] = fmaxf(s[2 * c], s[2 * c + 1]);
+#pragma unroll
+  for (int j = 16; j < 128; j += 16)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) mc[c] = max3(mc[c], s[j + 2 * c], s[j + 2 * c + 1]);
+  return max3(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+}
+
+// P = 2^(s * scale_log2 - m) for a 128-column row, written as bf16 pairs to
+// TMEM (64 columns at tP) in four 32-key chunks as they are produced; returns
+// the fp32 row sum of P.
+__device__ __forceinline__ float exp_pass_store(const float (&s)[128], float sl2, float m,
+                                                uint32_t tP) {
+  const float2 sc2 = make_float2(sl2, sl2);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int jj = 16 * c + j;  // column pair
+      const float2 x = __ffma2_rn(make_float2(s[2 * jj], s[2 * jj + 1]), sc2, nm2);
+      float2 e;
+      if (kPolyMask & (1u << (jj & 7))) {
+        e = exp2_poly2(x);
+      } else {
+        e.x = ex2(x.x);
+        e.y = ex2(x.y);
+      }
+      acc[j & 3] = __fadd2_rn(acc[j & 3], e);
+      pk[j] = pack_bf16(e.x, e.y);
+    }
+    lcptx::tmem_st16(tP + 16 * c, pk);
+  }
+  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+  return a.x + a.y;
+}
+
+// Mask limits of tile tt of an item for the rows of query block `qsub`:
+// bits 0-7 = attended tokens of the tile's first key block (0 when the block
+// is not attended), bits 8-15 = same for the second block.
+__device__ __forceinline__ uint32_t tile_limits(const Sm100Params &p, const Item &it, int tt,
+                                                int qsub) {
+  if (2 * tt >= it.len) return 0u;
+  const uint32_t ea = __ldg(it.ent + 2 * tt);
+  int sx, rx, na, nb = 0;
+  entry_block(p, ea, sx, rx, na);
+  if (!((ea >> (24 + qsub)) & 1u)) na = 0;
+  if (2 * tt + 1 < it.len) {
+    const uint32_t eb = __ldg(it.ent + 2 * tt + 1);
+    entry_block(p, eb, sx, rx, nb);
+    if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
+  }
+  return (uint32_t)na | ((uint32_t)nb << 8);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_constant__ Sm100Params p) {
@@ -243,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
                                               ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  uint8_t *sQ = smem + SmemOffsets::q;
+  uint8_t *sQ = smem + SmemOffsets::q;  // tile (buf, i) at sQ + (2*buf + i) * kTileBytes
   uint8_t *sK = smem + SmemOffsets::k;
   uint8_t *sV = smem + SmemOffsets::v;
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SmemOffsets::misc);
@@ -259,10 +390,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   for (int i = tid; i < p.tab_floats; i += kThreads) tab[i] = p.rope_tab[i];
   if (tid == 0) {
     misc[3] = 0;
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       lcptx::mbar_init(ctx.bar(B_QFULL + i), 1);
       lcptx::mbar_init(ctx.bar(B_QREADY + i), kRopeThreads);
       lcptx::mbar_init(ctx.bar(B_QEMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       lcptx::mbar_init(ctx.bar(B_SFULL + i), 1);
       lcptx::mbar_init(ctx.bar(B_SFREE + i), 4);
       lcptx::mbar_init(ctx.bar(B_PFULL + i), 4);
@@ -297,34 +430,45 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   __syncthreads();
   lcptx::tc_fence_after();
   const uint32_t tmem = misc[0];
+  const bool k_rot = p.k_prerotated != 0;
 
+  // Register split: the softmax warpgroups (warps 0-7) hold a 128-column row
+  // of S in registers; the producer / MMA / RoPE warpgroup needs few.
+  // 256 x kRegsSoftmax + 128 x kRegsOther must not exceed the registers the
+  // block was launched with; the host refuses to launch otherwise.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
   if (warp == kWarpProducer) {
     // ======================= TMA producer (one thread) =======================
     if (lane == 0) {
       uint32_t kv_it = 0, item_it = 0;
-      uint32_t k_issued[kStages], v_issued[kStages], q_issued[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};
-      for (int s = 0; s < kStages; ++s) k_issued[s] = v_issued[s] = 0xFFFFFFFFu;
+      // Issued loads, for the drain: bit j of *_valid says barrier j got a
+      // load, bit j of *_par is the parity of its last phase.
+      uint32_t q_valid = 0, q_par = 0, k_valid = 0, k_par = 0, v_valid = 0, v_par = 0;
       for (;;) {
         const int slot = item_it & 1;
-        const uint32_t sph = (item_it >> 1) & 1;
         int item = atomicAdd(p.work_counter, 1);
         if (item >= p.total_items) item = -1;
-        if (!wait_bar(ctx, ctx.bar(B_SCHED_EMPTY + slot), sph ^ 1)) break;
+        if (!wait_bar(ctx, ctx.bar(B_SCHED_EMPTY + slot), ((item_it >> 1) & 1) ^ 1)) break;
         misc[1 + slot] = (uint32_t)item;
         lcptx::mbar_arrive(ctx.bar(B_SCHED_FULL + slot));
         if (item < 0) break;
         const Item it = decode_item(p, item);
+        const int buf = item_it & 1;
+        const uint32_t qph = (item_it >> 1) & 1;
         bool ok = true;
         for (int i = 0; i < 2 && ok; ++i) {
-          ok = wait_bar(ctx, ctx.bar(B_QEMPTY + i), (item_it & 1) ^ 1);
+          const int qi = 2 * buf + i;
+          ok = wait_bar(ctx, ctx.bar(B_QEMPTY + qi), qph ^ 1);
           if (!ok) break;
-          uint32_t bq = ctx.bar(B_QFULL + i);
+          const uint32_t bq = ctx.bar(B_QFULL + qi);
           lcptx::mbar_arrive_expect_tx(bq, kTileBytes);
-          uint32_t dst = lcptx::smem_addr(sQ + i * kTileBytes);
-          int r = it.row0 + 128 * i;
+          const uint32_t dst = lcptx::smem_addr(sQ + qi * kTileBytes);
+          const int r = it.row0 + 128 * i;
           lcptx::tma_load_4d(dst, &p.tmQ[it.seg], bq, 0, it.h, r, it.b);
           lcptx::tma_load_4d(dst + kBoxBytes, &p.tmQ[it.seg], bq, 0, it.h, r + 64, it.b);
-          q_issued[i] = item_it & 1;
+          q_valid |= 1u << qi;
+          q_par = (q_par & ~(1u << qi)) | (qph << qi);
         }
         if (!ok) break;
         const int ntiles = (it.len + 1) >> 1;
@@ -332,145 +476,153 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           const int s = kv_it % kStages;
           const uint32_t ph = (kv_it / kStages) & 1;
           int sa, ra, na, sb, rb, nb;
-          entry_block(p, it.ent[2 * t], sa, ra, na);
+          entry_block(p, __ldg(it.ent + 2 * t), sa, ra, na);
           if (2 * t + 1 < it.len) {
-            entry_block(p, it.ent[2 * t + 1], sb, rb, nb);
+            entry_block(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
           } else {  // no second block: a box entirely past the segment end reads zeros
             sb = 1;
             rb = p.Nn;
           }
           ok = wait_bar(ctx, ctx.bar(B_KEMPTY + s), ph ^ 1);
           if (!ok) break;
-          uint32_t bk = ctx.bar(B_KFULL + s);
+          const uint32_t bk = ctx.bar(B_KFULL + s);
           lcptx::mbar_arrive_expect_tx(bk, kTileBytes);
-          uint32_t dk = lcptx::smem_addr(sK + s * kTileBytes);
+          const uint32_t dk = lcptx::smem_addr(sK + s * kTileBytes);
           lcptx::tma_load_4d(dk, &p.tmK[sa], bk, 0, it.h, ra, it.b);
           lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[sb], bk, 0, it.h, rb, it.b);
-          k_issued[s] = ph;
+          k_valid |= 1u << s;
+          k_par = (k_par & ~(1u << s)) | (ph << s);
           ok = wait_bar(ctx, ctx.bar(B_VEMPTY + s), ph ^ 1);
           if (!ok) break;
-          uint32_t bv = ctx.bar(B_VFULL + s);
+          const uint32_t bv = ctx.bar(B_VFULL + s);
           lcptx::mbar_arrive_expect_tx(bv, kTileBytes);
-          uint32_t dv = lcptx::smem_addr(sV + s * kTileBytes);
+          const uint32_t dv = lcptx::smem_addr(sV + s * kTileBytes);
           lcptx::tma_load_4d(dv, &p.tmV[sa], bv, 0, it.h, ra, it.b);
           lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[sb], bv, 0, it.h, rb, it.b);
-          v_issued[s] = ph;
+          v_valid |= 1u << s;
+          v_par = (v_par & ~(1u << s)) | (ph << s);
         }
         if (!ok) break;
         ++item_it;
       }
       // Drain: every load this thread issued must land before the CTA exits.
-      for (int i = 0; i < 2; ++i) {
-        if (q_issued[i] != 0xFFFFFFFFu) {
-          uint64_t t0 = lcptx::globaltimer_ns();
-          while (!lcptx::mbar_try_wait(ctx.bar(B_QFULL + i), q_issued[i]) &&
-                 (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {}
+      auto drain = [&](uint32_t bar, uint32_t valid, uint32_t par, int j) {
+        if (!((valid >> j) & 1u)) return;
+        const uint32_t ph = (par >> j) & 1u;
+        const uint64_t t0 = lcptx::globaltimer_ns();
+        while (!lcptx::mbar_try_wait(bar, ph) &&
+               (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {
         }
-      }
+      };
+#pragma unroll
+      for (int i = 0; i < 4; ++i) drain(ctx.bar(B_QFULL + i), q_valid, q_par, i);
+#pragma unroll
       for (int s = 0; s < kStages; ++s) {
-        if (k_issued[s] != 0xFFFFFFFFu) {
-          uint64_t t0 = lcptx::globaltimer_ns();
-          while (!lcptx::mbar_try_wait(ctx.bar(B_KFULL + s), k_issued[s]) &&
-                 (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {}
-        }
-        if (v_issued[s] != 0xFFFFFFFFu) {
-          uint64_t t0 = lcptx::globaltimer_ns();
-          while (!lcptx::mbar_try_wait(ctx.bar(B_VFULL + s), v_issued[s]) &&
-                 (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {}
-        }
+        drain(ctx.bar(B_KFULL + s), k_valid, k_par, s);
+        drain(ctx.bar(B_VFULL + s), v_valid, v_par, s);
       }
     }
   } else if (warp == kWarpMma) {
     // ======================= MMA issuer (one thread) =========================
-    uint32_t item_it = 0, kv_it = 0;
-    uint32_t sfree_ph[2] = {0, 0}, pfull_ph[2] = {0, 0};
-    if (lane == 0) for (;;) {
-      const int slot = item_it & 1;
-      if (!wait_bar(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
-      const int item = (int)misc[1 + slot];
-      lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
-      if (item < 0) break;
-      const Item it = decode_item(p, item);
-      const int ntiles = (it.len + 1) >> 1;
-      bool ok = wait_bar(ctx, ctx.bar(B_QREADY + 0), item_it & 1) &&
-                wait_bar(ctx, ctx.bar(B_QREADY + 1), item_it & 1);
-      if (!ok) break;
-      const uint32_t q_addr[2] = {lcptx::smem_addr(sQ), lcptx::smem_addr(sQ + kTileBytes)};
-      auto issue_s = [&](int i, int s) -> bool {
-        if (!wait_bar(ctx, ctx.bar(B_SFREE + i), sfree_ph[i] ^ 1)) return false;
-        sfree_ph[i] ^= 1;
-        lcptx::tc_fence_after();
-        const uint32_t kb = lcptx::smem_addr(sK + s * kTileBytes);
-        const uint32_t d = tmem + (i ? kColS1 : kColS0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          uint64_t a = lcptx::smem_desc_sw128(q_addr[i] + 32 * kk, 16, 1024);
-          uint64_t b = lcptx::smem_desc_sw128(kb + 32 * kk, 16, 1024);
-          lcptx::mma_ss(d, a, b, kIdescQK, kk > 0);
-        }
-        lcptx::mma_commit(ctx.bar(B_SFULL + i));
-        return true;
-      };
-      auto issue_pv = [&](int i, int s, bool accumulate) -> bool {
-        if (!wait_bar(ctx, ctx.bar(B_PFULL + i), pfull_ph[i])) return false;
-        pfull_ph[i] ^= 1;
-        lcptx::tc_fence_after();
-        const uint32_t vb = lcptx::smem_addr(sV + s * kTileBytes);
-        const uint32_t d = tmem + (i ? kColO1 : kColO0);
-        const uint32_t a = tmem + (i ? kColP1 : kColP0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          uint64_t b = lcptx::smem_desc_sw128(vb + 2048 * kk, 8192, 1024);
-          lcptx::mma_ts(d, a + 8 * kk, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
-        }
-        lcptx::mma_commit(ctx.bar(B_ODONE + i));
-        return true;
-      };
-      // Tile 0: both S tiles.
-      {
-        const int s = kv_it % kStages;
-        ok = wait_bar(ctx, ctx.bar(B_KREADY + s), (kv_it / kStages) & 1) && issue_s(0, s) &&
-             issue_s(1, s);
-        if (!ok) break;
-        lcptx::mma_commit(ctx.bar(B_KEMPTY + s));
-      }
-      for (int t = 0; t < ntiles && ok; ++t) {
-        const uint32_t cur = kv_it + t;
-        const int s = cur % kStages;
-        const bool more = t + 1 < ntiles;
-        const int s_next = (cur + 1) % kStages;
-        if (more) {
-          ok = wait_bar(ctx, ctx.bar(B_KREADY + s_next), ((cur + 1) / kStages) & 1) &&
-               issue_s(0, s_next);
-          if (!ok) break;
-        }
-        ok = wait_bar(ctx, ctx.bar(B_VFULL + s), (cur / kStages) & 1) && issue_pv(0, s, t > 0);
-        if (!ok) break;
-        if (more) {
-          ok = issue_s(1, s_next);
-          if (!ok) break;
-          lcptx::mma_commit(ctx.bar(B_KEMPTY + s_next));
-        }
-        ok = issue_pv(1, s, t > 0);
-        if (!ok) break;
-        lcptx::mma_commit(ctx.bar(B_VEMPTY + s));
-      }
-      if (!ok) break;
-      kv_it += ntiles;
-      ++item_it;
-    }
     if (lane == 0) {
+      uint32_t item_it = 0;
+      int cs = 0;        // K/V stage of the current tile
+      uint32_t cph = 0;  // and its phase parity
+      uint32_t sfree_bits = 0, pfull_bits = 0;  // bit i: phase parity for tile i
+      const int kbar = k_rot ? B_KFULL : B_KREADY;
+      // Operand descriptors, built once: the high word (stride byte offset
+      // 1024, version 1, 128-byte swizzle) is common; the low word holds the
+      // start address >> 4 and the leading byte offset, and steps by 32 bytes
+      // per 16-wide K slice of Q/K and by 2048 bytes (16 keys) for V.
+      constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      constexpr uint32_t kTileLo = kTileBytes >> 4;
+      const uint32_t q_lo0 = (lcptx::smem_addr(sQ) >> 4) | (1u << 16);
+      const uint32_t k_lo0 = (lcptx::smem_addr(sK) >> 4) | (1u << 16);
+      const uint32_t v_lo0 = (lcptx::smem_addr(sV) >> 4) | (512u << 16);
+      auto desc = [](uint32_t lo) -> uint64_t {
+        return (static_cast<uint64_t>(kDescHi) << 32) | lo;
+      };
+      for (;;) {
+        const int slot = item_it & 1;
+        if (!wait_bar(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
+        const int item = (int)misc[1 + slot];
+        lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
+        if (item < 0) break;
+        const Item it = decode_item(p, item);
+        const int ntiles = (it.len + 1) >> 1;
+        const int buf = item_it & 1;
+        const uint32_t qph = (item_it >> 1) & 1;
+        bool ok = wait_bar(ctx, ctx.bar(B_QREADY + 2 * buf), qph) &&
+                  wait_bar(ctx, ctx.bar(B_QREADY + 2 * buf + 1), qph);
+        if (!ok) break;
+        const uint32_t q_lo = q_lo0 + 2 * buf * kTileLo;
+        auto issue_s = [&](int i, int s) -> bool {
+          if (!wait_bar(ctx, ctx.bar(B_SFREE + i), ((sfree_bits >> i) & 1u) ^ 1u)) return false;
+          sfree_bits ^= 1u << i;
+          lcptx::tc_fence_after();
+          const uint32_t qa = q_lo + i * kTileLo, kb = k_lo0 + s * kTileLo;
+          const uint32_t d = tmem + (i ? kColS1 : kColS0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            lcptx::mma_ss(d, desc(qa + 2 * kk), desc(kb + 2 * kk), kIdescQK, kk > 0);
+          lcptx::mma_commit(ctx.bar(B_SFULL + i));
+          return true;
+        };
+        auto issue_pv = [&](int i, int s, bool accumulate) -> bool {
+          if (!wait_bar(ctx, ctx.bar(B_PFULL + i), (pfull_bits >> i) & 1u)) return false;
+          pfull_bits ^= 1u << i;
+          lcptx::tc_fence_after();
+          const uint32_t vb = v_lo0 + s * kTileLo;
+          const uint32_t d = tmem + (i ? kColO1 : kColO0);
+          const uint32_t a = tmem + (i ? kColP1 : kColP0);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            lcptx::mma_ts(d, a + 8 * kk, desc(vb + 128 * kk), kIdescPV,
+                          (accumulate || kk > 0) ? 1u : 0u);
+          lcptx::mma_commit(ctx.bar(B_ODONE + i));
+          return true;
+        };
+        // tile 0: both S tiles
+        ok = wait_bar(ctx, ctx.bar(kbar + cs), cph) && issue_s(0, cs) && issue_s(1, cs);
+        if (!ok) break;
+        lcptx::mma_commit(ctx.bar(B_KEMPTY + cs));
+        for (int t = 0; t < ntiles && ok; ++t) {
+          const bool more = t + 1 < ntiles;
+          const int ns = cs + 1 == kStages ? 0 : cs + 1;
+          const uint32_t nph = ns == 0 ? cph ^ 1u : cph;
+          if (more) {
+            ok = wait_bar(ctx, ctx.bar(kbar + ns), nph) && issue_s(0, ns);
+            if (!ok) break;
+          }
+          ok = wait_bar(ctx, ctx.bar(B_VFULL + cs), cph) && issue_pv(0, cs, t > 0);
+          if (!ok) break;
+          if (more) {
+            ok = issue_s(1, ns);
+            if (!ok) break;
+            lcptx::mma_commit(ctx.bar(B_KEMPTY + ns));
+          }
+          ok = issue_pv(1, cs, t > 0);
+          if (!ok) break;
+          lcptx::mma_commit(ctx.bar(B_VEMPTY + cs));
+          cs = ns;
+          cph = nph;
+        }
+        if (!ok) break;
+        ++item_it;
+      }
       // Drain: wait until every MMA this thread issued has completed.
       lcptx::mma_commit(ctx.bar(B_DRAIN));
-      uint64_t t0 = lcptx::globaltimer_ns();
+      const uint64_t t0 = lcptx::globaltimer_ns();
       while (!lcptx::mbar_try_wait(ctx.bar(B_DRAIN), 0) &&
-             (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {}
+             (long long)(lcptx::globaltimer_ns() - t0) < p.timeout_ns) {
+      }
     }
     __syncwarp();
-  } else if (warp >= kWarpRope) {
+  } else {
     // ======================= RoPE warps ======================================
     const int rt = tid - kWarpRope * 32;
     uint32_t item_it = 0, kv_it = 0;
+    EntryStream es;
     for (;;) {
       const int slot = item_it & 1;
       if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
@@ -480,38 +632,50 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       if (item < 0) break;
       const Item it = decode_item(p, item);
       const int seg_base = it.seg ? p.Nc : 0;  // sequence index of the segment's token 0
+      const int buf = item_it & 1;
+      const uint32_t qph = (item_it >> 1) & 1;
       bool ok = true;
       for (int i = 0; i < 2 && ok; ++i) {
-        ok = wait_warp(ctx, ctx.bar(B_QFULL + i), item_it & 1);
+        const int qi = 2 * buf + i;
+        ok = wait_warp(ctx, ctx.bar(B_QFULL + qi), qph);
         if (!ok) break;
-        int r0 = it.row0 + 128 * i;
-        int nrows = min(128, it.seg_len - r0);
-        if (nrows > 0) rope_tile(sQ + i * kTileBytes, 0, nrows, seg_base + r0, tab, p, rt);
+        const int r0 = it.row0 + 128 * i;
+        const int nrows = min(128, it.seg_len - r0);
+#pragma unroll 1
+        for (int r = rt; r < nrows; r += kRopeThreads)
+          rope_row(sQ + qi * kTileBytes, r, seg_base + r0 + r, tab, p);
         lcptx::fence_proxy_async_smem();
-        lcptx::mbar_arrive(ctx.bar(B_QREADY + i));
+        lcptx::mbar_arrive(ctx.bar(B_QREADY + qi));
       }
       if (!ok) break;
-      const int ntiles = (it.len + 1) >> 1;
-      for (int t = 0; t < ntiles; ++t, ++kv_it) {
-        const int s = kv_it % kStages;
-        ok = wait_warp(ctx, ctx.bar(B_KFULL + s), (kv_it / kStages) & 1);
-        if (!ok) break;
-        int sa, ra, na;
-        entry_block(p, it.ent[2 * t], sa, ra, na);
-        uint8_t *tile = sK + s * kTileBytes;
-        rope_tile(tile, 0, na, (sa ? p.Nc : 0) + ra, tab, p, rt);
-        if (2 * t + 1 < it.len) {
-          int sb, rb, nb;
-          entry_block(p, it.ent[2 * t + 1], sb, rb, nb);
-          rope_tile(tile, 64, 64 + nb, (sb ? p.Nc : 0) + rb - 64, tab, p, rt);
+      if (!k_rot) {
+        const int ntiles = (it.len + 1) >> 1;
+        es.start(it.ent, it.len, lane);
+        for (int t = 0; t < ntiles; ++t, ++kv_it) {
+          const int s = kv_it % kStages;
+          uint32_t ea, eb;
+          es.pair(t, lane, ea, eb);
+          ok = wait_warp(ctx, ctx.bar(B_KFULL + s), (kv_it / kStages) & 1);
+          if (!ok) break;
+          uint8_t *tile = sK + s * kTileBytes;
+          // Row rt of each of the tile's two key blocks (one code copy).
+#pragma unroll 1
+          for (int half = 0; half < 2; ++half) {
+            if (half == 1 && 2 * t + 1 >= it.len) break;
+            int sx, rx, nx;
+            entry_block(p, half ? eb : ea, sx, rx, nx);
+            if (rt < nx) rope_row(tile, 64 * half + rt, (sx ? p.Nc : 0) + rx + rt, tab, p);
+          }
+          lcptx::fence_proxy_async_smem();
+          lcptx::mbar_arrive(ctx.bar(B_KREADY + s));
         }
-        lcptx::fence_proxy_async_smem();
-        lcptx::mbar_arrive(ctx.bar(B_KREADY + s));
+        if (!ok) break;
       }
-      if (!ok) break;
       ++item_it;
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ======================= softmax warpgroups ==============================
     const int wg = warp >> 2;              // which Q tile
     const int row = tid & 127;             // TMEM lane == tile row
@@ -520,6 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
     const uint32_t tS = tmem + lane_base + (wg ? kColS1 : kColS0);
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
     const uint32_t tP = tmem + lane_base + (wg ? kColP1 : kColP0);
+    const float sl2 = p.scale_log2;
     uint32_t item_it = 0, sfull_ph = 0, odone_ph = 0;
     for (;;) {
       const int slot = item_it & 1;
@@ -530,38 +695,35 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       if (item < 0) break;
       const Item it = decode_item(p, item);
       const int ntiles = (it.len + 1) >> 1;
+      // Mask limits of this warp's rows, one tile per lane, 32 tiles at a time.
+      uint32_t lim_lane = 0;
       float m_ref = -INFINITY, l_sum = 0.f;
       bool ok = true;
       for (int t = 0; t < ntiles; ++t) {
-        // Mask limits for this warp's rows (uniform across the warp).
-        int sa, ra, na, nb = 0;
-        uint32_t ea = it.ent[2 * t];
-        entry_block(p, ea, sa, ra, na);
-        if (!((ea >> (24 + qsub)) & 1u)) na = 0;
-        if (2 * t + 1 < it.len) {
-          uint32_t eb = it.ent[2 * t + 1];
-          int sb, rb;
-          entry_block(p, eb, sb, rb, nb);
-          if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
-        }
+        if ((t & 31) == 0) lim_lane = tile_limits(p, it, t + lane, qsub);
+        const uint32_t lim = __shfl_sync(0xffffffffu, lim_lane, t & 31);
+        const int na = lim & 0xFF, nb = (lim >> 8) & 0xFF;
         ok = wait_warp(ctx, ctx.bar(B_SFULL + wg), sfull_ph);
         if (!ok) break;
         sfull_ph ^= 1;
         lcptx::tc_fence_after();
-        float s[128];
-        {
-          uint32_t r32[32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            lcptx::tmem_ld32(tS + 32 * c, r32);
-            lcptx::tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s[32 * c + j] = __uint_as_float(r32[j]);
-          }
-        }
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        lcptx::tmem_ld32(tS, r0);
+        lcptx::tmem_ld32(tS + 32, r1);
+        lcptx::tmem_ld32(tS + 64, r2);
+        lcptx::tmem_ld32(tS + 96, r3);
+        lcptx::tmem_wait_ld();
         lcptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SFREE + wg));
+        float s[128];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          s[j] = __uint_as_float(r0[j]);
+          s[32 + j] = __uint_as_float(r1[j]);
+          s[64 + j] = __uint_as_float(r2[j]);
+          s[96 + j] = __uint_as_float(r3[j]);
+        }
         if (na < 64) {
 #pragma unroll
           for (int j = 0; j < 64; ++j)
@@ -572,59 +734,100 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           for (int j = 0; j < 64; ++j)
             if (j >= nb) s[64 + j] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // The first tile sets the reference max exactly.  Later tiles reuse
+        // it: P = 2^(x) with x = s * scale_log2 - m_ref and no row max at all,
+        // which is valid as long as no element exceeds m_ref + 8 -- certain
+        // when the tile's sum is at most 2^8.  Otherwise the row max is taken,
+        // and if it is above m_ref + 8 the reference moves up, O and l are
+        // rescaled and P is redone from the logits kept in s.
+        if (t == 0) m_ref = row_max(s) * sl2;
+        float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        bool o_ready = (t == 0);  // P / O of this warpgroup free (previous P*V done)
+        float l_tile = 0.f;
+        // One pass: s <- s * mul + add in place, P = 2^s pipelined (the ex2 of
+        // pair j is issued after pair j-8 is packed and summed), P to TMEM in
+        // 32-key chunks; waits for the previous P*V just before the first store.
+        auto pass = [&](float mul, float add) -> bool {
+          const float2 mul2 = make_float2(mul, mul), add2 = make_float2(add, add);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
+          float e[16];
+          uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 128; ++j) mx = fmaxf(mx, s[j]);
-        const float mt = mx * p.scale_log2;
+          for (int j = 0; j < 72; ++j) {
+            if (j >= 8) {  // consume pair k = j - 8
+              const int k = j - 8;
+              const float2 v = make_float2(e[2 * (k & 7)], e[2 * (k & 7) + 1]);
+              acc[k & 3] = __fadd2_rn(acc[k & 3], v);
+              pk[k & 15] = pack_bf16(v.x, v.y);
+              if ((k & 15) == 15) {
+                if (!o_ready) {
+                  if (!wait_warp(ctx, ctx.bar(B_ODONE + wg), odone_ph)) return false;
+                  odone_ph ^= 1;
+                  lcptx::tc_fence_after();
+                  o_ready = true;
+                }
+                lcptx::tmem_st16(tP + 16 * (k >> 4), pk);
+              }
+            }
+            if (j < 64) {  // logits and ex2 of pair j
+              const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), mul2, add2);
+              s[2 * j] = x.x;
+              s[2 * j + 1] = x.y;
+              if (kPolyMask & (1u << (j & 7))) {
+                const float2 y = exp2_poly2(x);
+                e[2 * (j & 7)] = y.x;
+                e[2 * (j & 7) + 1] = y.y;
+              } else {
+                e[2 * (j & 7)] = ex2(x.x);
+                e[2 * (j & 7) + 1] = ex2(x.y);
+              }
+            }
+          }
+          const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+          l_tile = a.x + a.y;
+          return true;
+        };
+        ok = pass(sl2, -m_use);
+        if (!ok) break;
         float alpha = 1.f;
         bool rescale_o = false;
-        if (t == 0) {
-          m_ref = mt;
-        } else {
-          bool need = mt > m_ref + kRescaleThreshold;
-          if (__any_sync(0xffffffffu, need)) {
-            float m_new = fmaxf(m_ref, mt);
+        if (t > 0 && __any_sync(0xffffffffu, !(l_tile <= 256.f))) {
+          const float mt = row_max(s) + m_use;  // s now holds logits minus m_use
+          if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
+            const float m_new = fmaxf(m_ref, mt);
             alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);
             l_sum *= alpha;
             m_ref = m_new;
+            const float m_new_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+            ok = pass(1.f, m_use - m_new_use);
+            if (!ok) break;
+            m_use = m_new_use;
             rescale_o = true;
           }
         }
-        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        uint32_t pk[64];
-        float lsum_t = 0.f;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          float p0 = ex2(fmaf(s[2 * j], p.scale_log2, -m_use));
-          float p1 = ex2(fmaf(s[2 * j + 1], p.scale_log2, -m_use));
-          lsum_t += p0 + p1;
-          pk[j] = pack_bf16(p0, p1);
-        }
-        l_sum += lsum_t;
-        // P and O may be touched only after the previous P*V finished.
-        if (t > 0) {
+        if (!o_ready) {  // (a tile always stores P, so this is only a safeguard)
           ok = wait_warp(ctx, ctx.bar(B_ODONE + wg), odone_ph);
           if (!ok) break;
           odone_ph ^= 1;
           lcptx::tc_fence_after();
-          if (rescale_o) {
-            uint32_t o32[32];
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-              lcptx::tmem_ld32(tO + 32 * c, o32);
-              lcptx::tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o32[j] = __float_as_uint(__uint_as_float(o32[j]) * alpha);
-              lcptx::tmem_st32(tO + 32 * c, o32);
-            }
-          }
         }
-        {
-          uint32_t h0[32], h1[32];
+        l_sum += l_tile;
+        if (rescale_o) {
+          uint32_t o0[32], o1[32];
+          lcptx::tmem_ld32(tO, o0);
+          lcptx::tmem_ld32(tO + 32, o1);
+          lcptx::tmem_wait_ld();
+          const float2 al = make_float2(alpha, alpha);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) { h0[j] = pk[j]; h1[j] = pk[32 + j]; }
-          lcptx::tmem_st32(tP, h0);
-          lcptx::tmem_st32(tP + 32, h1);
+          for (int j = 0; j < 16; ++j) {
+            float2 u = __fmul2_rn(make_float2(__uint_as_float(o0[2 * j]), __uint_as_float(o0[2 * j + 1])), al);
+            float2 v = __fmul2_rn(make_float2(__uint_as_float(o1[2 * j]), __uint_as_float(o1[2 * j + 1])), al);
+            o0[2 * j] = __float_as_uint(u.x); o0[2 * j + 1] = __float_as_uint(u.y);
+            o1[2 * j] = __float_as_uint(v.x); o1[2 * j + 1] = __float_as_uint(v.y);
+          }
+          lcptx::tmem_st32(tO, o0);
+          lcptx::tmem_st32(tO + 32, o1);
         }
         lcptx::tmem_wait_st();
         lcptx::tc_fence_before();
@@ -638,20 +841,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       odone_ph ^= 1;
       lcptx::tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      uint8_t *stage = sQ + wg * kTileBytes;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o32[32];
-        lcptx::tmem_ld32(tO + 32 * c, o32);
+      const int buf = item_it & 1;
+      uint8_t *stage = sQ + (2 * buf + wg) * kTileBytes;
+      {
+        uint32_t o0[32], o1[32];
+        lcptx::tmem_ld32(tO, o0);
+        lcptx::tmem_ld32(tO + 32, o1);
         lcptx::tmem_wait_ld();
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t *o = ch < 4 ? o0 + 8 * ch : o1 + 8 * (ch - 4);
           uint4 v;
-          v.x = pack_bf16(__uint_as_float(o32[8 * ch + 0]) * inv_l, __uint_as_float(o32[8 * ch + 1]) * inv_l);
-          v.y = pack_bf16(__uint_as_float(o32[8 * ch + 2]) * inv_l, __uint_as_float(o32[8 * ch + 3]) * inv_l);
-          v.z = pack_bf16(__uint_as_float(o32[8 * ch + 4]) * inv_l, __uint_as_float(o32[8 * ch + 5]) * inv_l);
-          v.w = pack_bf16(__uint_as_float(o32[8 * ch + 6]) * inv_l, __uint_as_float(o32[8 * ch + 7]) * inv_l);
-          *reinterpret_cast<uint4 *>(stage + swz(row, 4 * c + ch)) = v;
+          v.x = pack_bf16(__uint_as_float(o[0]) * inv_l, __uint_as_float(o[1]) * inv_l);
+          v.y = pack_bf16(__uint_as_float(o[2]) * inv_l, __uint_as_float(o[3]) * inv_l);
+          v.z = pack_bf16(__uint_as_float(o[4]) * inv_l, __uint_as_float(o[5]) * inv_l);
+          v.w = pack_bf16(__uint_as_float(o[6]) * inv_l, __uint_as_float(o[7]) * inv_l);
+          *reinterpret_cast<uint4 *>(stage + swz(row, ch)) = v;
         }
       }
       lcptx::tc_fence_before();
@@ -668,13 +873,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         if (ok) {
           const uint32_t src = lcptx::smem_addr(stage);
           const int r0 = it.row0 + 128 * wg;
-          if (r0 < it.seg_len)
-            lcptx::tma_store_4d(&p.tmO[it.seg], src, 0, it.h, r0, it.b);
+          if (r0 < it.seg_len) lcptx::tma_store_4d(&p.tmO[it.seg], src, 0, it.h, r0, it.b);
           if (r0 + 64 < it.seg_len)
             lcptx::tma_store_4d(&p.tmO[it.seg], src + kBoxBytes, 0, it.h, r0 + 64, it.b);
           lcptx::bulk_commit_group();
           lcptx::bulk_wait_group_read0();
-          lcptx::mbar_arrive(ctx.bar(B_QEMPTY + wg));
+          lcptx::mbar_arrive(ctx.bar(B_QEMPTY + 2 * buf + wg));
         }
       }
       if ((warp & 3) == 0) ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
@@ -746,6 +950,57 @@ __global__ void watchdog_selftest_kernel(int *status, long long timeout_ns) {
     c.timeout_ns = timeout_ns;
     wait_bar(c, c.bar(0), 0);  // nothing ever arrives: the wait must give up
   }
+}
+
+// Standalone rotation of K (or any [B, ntok, heads, 64] bf16 tensor) into a
+// separate buffer, 16 bytes per thread step; used when the attention kernel
+// is given K already rotated.  Same arithmetic as rope_row.
+__global__ void rope_k_kernel(const uint4 *src, uint4 *dst, long long n_chunks, int heads,
+                              long long ntok, int tok_offset, const float *tab, int T, int H,
+                              int W, lc_divmod div_hw, lc_divmod div_w) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_chunks;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int ch = (int)(i & 7);
+    const long long tokhead = i >> 3;
+    const int n = (int)((tokhead / heads) % ntok) + tok_offset;
+    const int t = lc_div(n, div_hw);
+    const int rem = n - t * div_hw.d;
+    const int hh = lc_div(rem, div_w);
+    const int w = rem - hh * div_w.d;
+    const float *c, *s;
+    if (ch < 2) { c = tab + t * 8 + 4 * ch; s = c + T * 8; }
+    else if (ch < 5) { c = tab + T * 16 + hh * 12 + 4 * (ch - 2); s = c + H * 12; }
+    else { c = tab + T * 16 + H * 24 + w * 12 + 4 * (ch - 5); s = c + W * 12; }
+    const float4 cc = __ldg(reinterpret_cast<const float4 *>(c));
+    const float4 ss = __ldg(reinterpret_cast<const float4 *>(s));
+    const uint4 raw = __ldg(src + i);
+    uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+    const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float a = __uint_as_float(wds[q] << 16);
+      const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
+      __nv_bfloat162 o2 = __floats2bfloat162_rn(a * cs[q] - b * sn[q], a * sn[q] + b * cs[q]);
+      wds[q] = *reinterpret_cast<uint32_t *>(&o2);
+    }
+    dst[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  }
+}
+
+lc_status launch_rope_k(const void *src, void *dst, int batch, long long ntok, int heads,
+                        int tok_offset, const lc_rope3d_s *rope, cudaStream_t stream) {
+  const long long n_chunks = (long long)batch * ntok * heads * (LC_HEAD_DIM / 8);
+  int dev = 0, n_sm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (n_chunks + 255) / 256;
+  const int grid = (int)(want < 8LL * n_sm ? want : 8LL * n_sm);
+  rope_k_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint4 *>(src),
+                                          static_cast<uint4 *>(dst), n_chunks, heads, ntok,
+                                          tok_offset, rope->tab, rope->T, rope->H, rope->W,
+                                          lc_make_divmod(rope->H * rope->W),
+                                          lc_make_divmod(rope->W));
+  return lc_from_cuda(cudaGetLastError());
 }
 
 }  // namespace
@@ -840,6 +1095,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   prm.T = rope->T; prm.H = rope->H; prm.W = rope->W;
   prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.gc = plan->gc;
   prm.heads = heads;
+  prm.k_prerotated = 0;
   long long total = (long long)batch * heads * prm.n_groups_active;
   if (total == 0) return LC_OK;
   if (total >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
@@ -849,6 +1105,16 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
 
   const size_t smem = 1024 + SmemOffsets::tab + sizeof(float) * (size_t)rope->n_floats;
   if (smem > 227 * 1024) return LC_ERR_UNSUPPORTED;
+  // The kernel's setmaxnreg split needs at least kRegsAtLaunchMin registers
+  // per thread at launch; with fewer, raising the softmax warps' count could
+  // never complete, so such a build is refused instead of launched.
+  static int regs_at_launch = -1;
+  if (regs_at_launch < 0) {
+    cudaFuncAttributes fa;
+    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, bsa_sm100_kernel));
+    regs_at_launch = fa.numRegs;
+  }
+  if (regs_at_launch < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;
   LC_CUDA_TRY(cudaFuncSetAttribute(bsa_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)smem));
   int dev = 0, n_sm = 0;
@@ -866,17 +1132,54 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     }
     return lc_from_cuda(e);
   }
+  // K is rotated once per call into scratch (one pass over K) and the kernel
+  // loads it rotated; rotating every loaded K tile in the kernel instead (as
+  // the allocation-free entry point does) measured slower.  LC_BSA_K_PREPASS=0
+  // selects the in-kernel rotation here too, for comparison.
+  static const bool k_prepass = [] {
+    const char *e = getenv("LC_BSA_K_PREPASS");
+    return !(e && e[0] == '0');
+  }();
   int *counter = nullptr;
-  LC_CUDA_TRY(cudaMallocAsync(&counter, sizeof(int), stream));
-  prm.work_counter = counter;
-  cudaError_t e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
-  if (e == cudaSuccess) {
-    bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
-    e = cudaGetLastError();
+  void *k_rot = nullptr, *ck_rot = nullptr;
+  cudaError_t e = cudaSuccess;
+  if (k_prepass) {
+    const size_t kb = (size_t)batch * (cached ? Nn : N) * heads * LC_HEAD_DIM * 2;
+    e = cudaMallocAsync(&k_rot, kb, stream);
+    if (e == cudaSuccess)
+      s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
+                        stream);
+    if (e == cudaSuccess && s == LC_OK && cached && Nc > 0) {
+      e = cudaMallocAsync(&ck_rot, (size_t)batch * Nc * heads * LC_HEAD_DIM * 2, stream);
+      if (e == cudaSuccess) s = launch_rope_k(cond_k, ck_rot, batch, Nc, heads, 0, rope, stream);
+    }
+    if (e == cudaSuccess && s == LC_OK) {
+      if (cached) {
+        s = encode_segment(&prm.tmK[1], k_rot, batch, Nn, 0, Nn, heads);
+        if (s == LC_OK && Nc > 0) s = encode_segment(&prm.tmK[0], ck_rot, batch, Nc, 0, Nc, heads);
+        if (s == LC_OK && Nc == 0) prm.tmK[0] = prm.tmK[1];
+      } else {
+        s = encode_segment(&prm.tmK[1], k_rot, batch, N, Nc, Nn, heads);
+        if (s == LC_OK && Nc > 0) s = encode_segment(&prm.tmK[0], k_rot, batch, N, 0, Nc, heads);
+        if (s == LC_OK && Nc == 0) prm.tmK[0] = prm.tmK[1];
+      }
+      prm.k_prerotated = 1;
+    }
   }
-  cudaError_t e2 = cudaFreeAsync(counter, stream);
-  if (e == cudaSuccess) e = e2;
+  if (e == cudaSuccess && s == LC_OK) e = cudaMallocAsync(&counter, sizeof(int), stream);
+  if (e == cudaSuccess && s == LC_OK) {
+    prm.work_counter = counter;
+    e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
+    if (e == cudaSuccess) {
+      bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+      e = cudaGetLastError();
+    }
+  }
+  if (counter) cudaFreeAsync(counter, stream);
+  if (k_rot) cudaFreeAsync(k_rot, stream);
+  if (ck_rot) cudaFreeAsync(ck_rot, stream);
+  if (s != LC_OK) return s;
   return lc_from_cuda(e);
 }
 

@@ -57,6 +57,44 @@ lc_status run_forward(const void *q, const void *k, const void *v, const void *c
 
 }  // namespace
 
+namespace {
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[kMaxDevices] = {nullptr};
+}  // namespace
+
+// The library's own stream-ordered pool for per-call scratch.  It keeps what
+// it has allocated (release threshold = all), so steady-state calls reuse the
+// memory with no driver allocation, and the device's default pool is left
+// untouched.  The memory stays with the process until it exits.
+cudaMemPool_t lc_scratch_pool(lc_status *st) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = LC_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_pool_mu);
+  if (!g_pool[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    e = cudaMemPoolCreate(&pool, &props);
+    if (e == cudaSuccess) {
+      uint64_t keep = ~0ull;
+      e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    }
+    if (e != cudaSuccess) {
+      *st = lc_from_cuda(e);
+      return nullptr;
+    }
+    g_pool[dev] = pool;
+  }
+  *st = LC_OK;
+  return g_pool[dev];
+}
+
 int *lc_device_status_ptr(lc_status *st) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);

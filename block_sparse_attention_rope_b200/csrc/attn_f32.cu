@@ -159,6 +159,7 @@ lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
   int nrows = cached ? plan->Nb : plan->nq;
   if (nrows == 0) return LC_OK;
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));
   dim3 grid(nrows, heads, batch);
   attn_f32_kernel<<<grid, 64, 0, stream>>>(a);
   LC_CUDA_TRY(cudaGetLastError());

@@ -45,7 +45,10 @@
 
 namespace {
 
-constexpr int kStages = 3;
+#ifndef LC_KV_STAGES
+#define LC_KV_STAGES 3
+#endif
+constexpr int kStages = LC_KV_STAGES;
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
@@ -1126,6 +1129,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     prm.work_counter = counter_scratch;
     cudaError_t e = cudaMemsetAsync(counter_scratch, 0, sizeof(int), stream);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, rope->ready, 0);
     if (e == cudaSuccess) {
       bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
       e = cudaGetLastError();
@@ -1142,15 +1146,19 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   }();
   int *counter = nullptr;
   void *k_rot = nullptr, *ck_rot = nullptr;
-  cudaError_t e = cudaSuccess;
-  if (k_prepass) {
+  cudaMemPool_t pool = lc_scratch_pool(&s);
+  if (s != LC_OK) return s;
+  cudaError_t e = cudaStreamWaitEvent(stream, rope->ready, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
+  if (e == cudaSuccess && k_prepass) {
     const size_t kb = (size_t)batch * (cached ? Nn : N) * heads * LC_HEAD_DIM * 2;
-    e = cudaMallocAsync(&k_rot, kb, stream);
+    e = cudaMallocFromPoolAsync(&k_rot, kb, pool, stream);
     if (e == cudaSuccess)
       s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
                         stream);
     if (e == cudaSuccess && s == LC_OK && cached && Nc > 0) {
-      e = cudaMallocAsync(&ck_rot, (size_t)batch * Nc * heads * LC_HEAD_DIM * 2, stream);
+      e = cudaMallocFromPoolAsync(&ck_rot, (size_t)batch * Nc * heads * LC_HEAD_DIM * 2, pool,
+                                  stream);
       if (e == cudaSuccess) s = launch_rope_k(cond_k, ck_rot, batch, Nc, heads, 0, rope, stream);
     }
     if (e == cudaSuccess && s == LC_OK) {
@@ -1166,11 +1174,11 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
       prm.k_prerotated = 1;
     }
   }
-  if (e == cudaSuccess && s == LC_OK) e = cudaMallocAsync(&counter, sizeof(int), stream);
+  if (e == cudaSuccess && s == LC_OK)
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&counter), sizeof(int), pool, stream);
   if (e == cudaSuccess && s == LC_OK) {
     prm.work_counter = counter;
     e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
     if (e == cudaSuccess) {
       bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
       e = cudaGetLastError();

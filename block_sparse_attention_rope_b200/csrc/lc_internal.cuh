@@ -50,12 +50,15 @@ struct lc_rope3d_s {
   double theta;
   int dt, dh, dw;
   int device;
+  cudaEvent_t ready;        // recorded after the table kernel
   long long n_floats;
   float *tab;
 };
 
-// Per-device library state: the status word kernels report into.
+// Per-device library state: the status word kernels report into, and the
+// library's stream-ordered pool for per-call scratch (keeps its memory).
 int *lc_device_status_ptr(lc_status *st);
+cudaMemPool_t lc_scratch_pool(lc_status *st);
 
 // Map a CUDA error to a status (out-of-memory gets its own code).
 static inline lc_status lc_from_cuda(cudaError_t e) {

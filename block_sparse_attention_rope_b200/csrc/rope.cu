@@ -110,6 +110,8 @@ extern "C" lc_status lc_rope3d_tables(lc_rope3d *out, int T, int H, int W, doubl
   int nb = (int)((r->n_floats + tpb - 1) / tpb);
   rope_tables_kernel<<<nb, tpb, 0, st>>>(r->tab, T, H, W, theta, dim_t, dim_h, dim_w);
   e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->ready, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventRecord(r->ready, st);
   if (e != cudaSuccess) {
     cudaFreeAsync(r->tab, st);
     delete r;
@@ -122,6 +124,7 @@ extern "C" lc_status lc_rope3d_tables(lc_rope3d *out, int T, int H, int W, doubl
 extern "C" lc_status lc_rope3d_destroy(lc_rope3d rope, void *stream) {
   if (!rope) return LC_OK;
   cudaError_t e = cudaFreeAsync(rope->tab, static_cast<cudaStream_t>(stream));
+  cudaEventDestroy(rope->ready);
   delete rope;
   return lc_from_cuda(e);
 }
@@ -129,6 +132,7 @@ extern "C" lc_status lc_rope3d_destroy(lc_rope3d rope, void *stream) {
 extern "C" lc_status lc_rope3d_copy_tables(lc_rope3d rope, float *host, void *stream) {
   if (!rope || !host) return LC_ERR_INVALID_ARGUMENT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LC_CUDA_TRY(cudaStreamWaitEvent(st, rope->ready, 0));
   LC_CUDA_TRY(cudaMemcpyAsync(host, rope->tab, sizeof(float) * rope->n_floats,
                               cudaMemcpyDeviceToHost, st));
   LC_CUDA_TRY(cudaStreamSynchronize(st));
@@ -154,6 +158,7 @@ extern "C" lc_status lc_rope3d_apply(const void *x, void *out, int batch, long l
   long long want = (n_chunks + tpb - 1) / tpb;
   int nb = (int)(want < 148LL * 16 ? want : 148LL * 16);
   lc_divmod dhw = lc_make_divmod(rope->H * rope->W), dw = lc_make_divmod(rope->W);
+  LC_CUDA_TRY(cudaStreamWaitEvent(st, rope->ready, 0));
   if (dtype == LC_DTYPE_F32)
     rope_apply_kernel<float><<<nb, tpb, 0, st>>>(static_cast<const float *>(x),
                                                  static_cast<float *>(out), n_chunks, heads, ntok,

@@ -135,6 +135,22 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(value: float, dist, device: str = "cuda") -> float:
+    """Max of a per-rank time over all ranks (one all-reduce, outside the data
+    path); identity without a process group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch element (weak scaling: fixed work per GPU)."""
+    return rank
+
+
 # ----------------------------------------------------------------------------- ours
 def time_forward(api, torch, w, d, plan, rope, steps, warmup, dist, stream):
     """Device time of `steps` back-to-back forward calls, bracketed by a
@@ -164,10 +180,7 @@ def time_forward(api, torch, w, d, plan, rope, steps, warmup, dist, stream):
         dist.barrier()
     per = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
     total = evs[0].elapsed_time(evs[-1])
-    if dist is not None:
-        t = torch.tensor([total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(total, dist)
     st = api.last_device_status()
     if st != 0:
         raise RuntimeError("device status %d after the timed region" % st)
@@ -212,7 +225,7 @@ def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, str
     info = plan.info()
     pairs = info.attended_token_pairs_noisy if w.cached else info.attended_token_pairs
     flops = 4.0 * w.head_dim * w.heads * w.batch * pairs
-    host = synthetic.make_inputs(w, seed_offset=rank)
+    host = synthetic.make_inputs(w, seed_offset=rank_seed_offset(rank))
     host = {k: v.pin_memory() for k, v in host.items()}
     d = {k: v.cuda() for k, v in host.items()}
     total_ms, launch_ms, out = time_forward(api, torch, w, d, plan, rope, steps, warmup, dist,
@@ -305,10 +318,7 @@ def run_ours(a):
         res = measure_workload(api, synthetic, torch, a.workload, 1, 1, dist, rank, stream,
                                e2e_steps=a.e2e_steps)
         e2e_ms = res["e2e_ms"]
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, dist)
         e2e = {"value": round(world * res["flops"] / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": res["h2d"],
                "d2h_bytes_per_step": res["d2h"],

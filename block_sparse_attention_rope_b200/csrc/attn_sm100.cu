@@ -1138,12 +1138,8 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   }
   // K is rotated once per call into scratch (one pass over K) and the kernel
   // loads it rotated; rotating every loaded K tile in the kernel instead (as
-  // the allocation-free entry point does) measured slower.  LC_BSA_K_PREPASS=0
-  // selects the in-kernel rotation here too, for comparison.
-  static const bool k_prepass = [] {
-    const char *e = getenv("LC_BSA_K_PREPASS");
-    return !(e && e[0] == '0');
-  }();
+  // the allocation-free entry point does, having no scratch) measured slower.
+  const bool k_prepass = true;
   int *counter = nullptr;
   void *k_rot = nullptr, *ck_rot = nullptr;
   cudaMemPool_t pool = lc_scratch_pool(&s);

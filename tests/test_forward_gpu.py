@@ -121,6 +121,40 @@ def test_large_logits_exercise_rescaling(api, name, qscale):
     assert np.abs(lse.numpy() - ref_lse).max() <= parity.BF16_LSE_ABS * qscale
 
 
+@pytest.mark.parametrize("name", ["small_i2v", "ragged", "many_heads", "batch2"])
+def test_in_kernel_k_rotation_path(api, name):
+    """The allocation-free entry point rotates each loaded K tile in shared
+    memory (no pre-rotated copy of K); check that path against the oracle."""
+    w = SMALL[name]
+    inputs = synthetic.make_inputs(w)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    d = {k: v.cuda() for k, v in inputs.items()}
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(w.batch, w.heads, w.n_tokens, device="cuda")
+    api.forward_noalloc(d["q"], d["k"], d["v"], plan, rope, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    ref_out, ref_lse = full_oracle(w, inputs)
+    check_all_rows(w, out.cpu(), lse.cpu(), ref_out, ref_lse)
+
+
+def test_in_kernel_k_rotation_full_size_sampled(api):
+    w = synthetic.get("i2v_480p")
+    inputs = synthetic.make_inputs(w)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    d = {k: v.cuda() for k, v in inputs.items()}
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(w.batch, w.heads, w.n_tokens, device="cuda")
+    api.forward_noalloc(d["q"], d["k"], d["v"], plan, rope, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    rows = parity.sample_rows(w, n_random_blocks=16)
+    ref_out, ref_lse = parity.oracle_rows(w, inputs, rows)
+    parity.compare(w, out.cpu(), lse.cpu(), ref_out, ref_lse, rows)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_cached_equals_noisy_rows_of_forward(api, dtype):
     w = Workload("x", T=5, H=8, W=24, n_cond=2, heads=3, local=1, stride=3, dtype=dtype)

@@ -231,6 +231,7 @@ def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, str
     total_ms, launch_ms, out = time_forward(api, torch, w, d, plan, rope, steps, warmup, dist,
                                             stream)
     res = {"w": w, "flops": flops, "pairs": pairs, "total_ms": total_ms, "launch_ms": launch_ms,
+           "scores": kernel_scores_per_head(plan, w.cached) * w.heads * w.batch,
            "spread": [round(x, 4) for x in time_forward.last_spread],
            "nnz": info.nnz}
     if e2e_steps:
@@ -239,6 +240,26 @@ def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, str
         res["e2e_ms"], res["h2d"], res["d2h"] = time_e2e(api, torch, w, host, plan, rope,
                                                          e2e_steps, stream)
     return res
+
+
+def kernel_scores_per_head(plan, cached: bool) -> int:
+    """Score elements the bf16 kernel forms (one exp2 each) per head: work
+    items are groups of 4 consecutive query blocks of one segment (two
+    128-row tiles), walking the union of their key lists 128 keys at a time.
+    Counted on the host from the plan's block CSR."""
+    import numpy as np
+    rp, ci = (t.numpy() for t in plan.csr())
+    inf = plan.info()
+    Cb, Nb = inf.num_cond_blocks, inf.num_noisy_blocks
+    total = 0
+    for seg0, nb in ((0, Cb), (Cb, Nb)):
+        if cached and seg0 == 0:
+            continue
+        for g in range(0, nb, 4):
+            r0, r1 = seg0 + g, seg0 + min(g + 4, nb)
+            n = len(np.unique(ci[rp[r0]:rp[r1]]))
+            total += 256 * 128 * ((n + 1) // 2)
+    return total
 
 
 def oracle_sample(w, x, heads, row_stride):
@@ -283,12 +304,27 @@ def cpu_baseline(name: str):
     from block_sparse_attention_rope_b200 import synthetic
     w = synthetic.get(name)
     x = synthetic.make_inputs(w)
-    heads, stride = list(range(8)), 6
+    heads, stride = list(range(8)), 3
     tf, sec, threads, pairs = oracle_sample(w, x, heads, stride)
     sample = ("fp64 oracle (C, OpenMP) on heads 0-7 x every %dth query row of %s "
               "(%.3g attended token pairs, RoPE of those heads included), %.1f s" %
               (stride, name, pairs, sec))
     return tf, sec, threads, sample
+
+
+def exp_roofline(res, clocks):
+    """The softmax's exp2 runs on the MUFU unit: 16 results per clock per SM
+    on B200, 148 SMs.  At head dim 64 that unit, not the tensor pipe, sets the
+    ceiling (4*64 attended FLOP per exp2 against ~16 x 256 per clock)."""
+    mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    peak = 148 * 16 * mhz * 1e6 / 1e9
+    achieved = res["scores"] / (res["launch_ms"] * 1e-3) / 1e9
+    return {"bound": "alu", "unit": "Gexp2/s", "achieved": round(achieved, 1),
+            "peak": round(peak, 1), "frac": round(achieved / peak, 4),
+            "peak_derivation": "148 SM x 16 MUFU ex2/clk x median SM clock under load (%.0f MHz)"
+                               % mhz,
+            "work": "%d score elements per launch (kernel tiles, masked padding included)"
+                    % res["scores"]}
 
 
 def run_ours(a):
@@ -361,6 +397,7 @@ def run_ours(a):
                      "peak_source": peak_src, "traffic": traffic_for(w.name),
                      "kernel": "bsa_sm100_kernel",
                      "algorithmic": "4*64*32*%d FLOP per launch" % main["pairs"]},
+        "exp_roofline": exp_roofline(main, clocks),
         "gpu_launches": a.steps,
         "clocks": clocks,
         "e2e": e2e,

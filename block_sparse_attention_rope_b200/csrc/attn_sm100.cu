@@ -76,6 +76,17 @@ constexpr int kRegsAtLaunchMin = (256 * kRegsSoftmax + 128 * kRegsOther + kThrea
 #define LC_POLY_EXP2_MASK 0x00u
 #endif
 constexpr uint32_t kPolyMask = LC_POLY_EXP2_MASK;
+// exp pass shape: pairs in flight between ex2 and their use (kLag <= kRing),
+// and whether all logits are formed before the ex2 stream starts.
+#ifndef LC_PASS_LAG
+#define LC_PASS_LAG 4
+#endif
+#ifndef LC_LOGITS_FIRST
+#define LC_LOGITS_FIRST 1
+#endif
+constexpr int kLag = LC_PASS_LAG, kRing = 16;
+constexpr bool kLogitsFirst = LC_LOGITS_FIRST != 0;
+static_assert(kLag <= kRing, "exp pass ring");
 
 struct __align__(64) Sm100Params {
   CUtensorMap tmQ[2], tmK[2], tmV[2], tmO[2];  // [0] condition segment, [1] noisy segment
@@ -754,13 +765,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           const float2 mul2 = make_float2(mul, mul), add2 = make_float2(add, add);
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                            make_float2(0.f, 0.f)};
-          float e[16];
+          float e[2 * kRing];
           uint32_t pk[16];
+          if (kLogitsFirst) {  // all 64 FFMA2 up front, independent of the ex2 stream
 #pragma unroll
-          for (int j = 0; j < 72; ++j) {
-            if (j >= 8) {  // consume pair k = j - 8
-              const int k = j - 8;
-              const float2 v = make_float2(e[2 * (k & 7)], e[2 * (k & 7) + 1]);
+            for (int j = 0; j < 64; ++j) {
+              const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), mul2, add2);
+              s[2 * j] = x.x;
+              s[2 * j + 1] = x.y;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 64 + kLag; ++j) {
+            if (j >= kLag) {  // consume pair k = j - kLag
+              const int k = j - kLag;
+              const float2 v = make_float2(e[2 * (k & (kRing - 1))], e[2 * (k & (kRing - 1)) + 1]);
               acc[k & 3] = __fadd2_rn(acc[k & 3], v);
               pk[k & 15] = pack_bf16(v.x, v.y);
               if ((k & 15) == 15) {
@@ -774,16 +793,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
               }
             }
             if (j < 64) {  // logits and ex2 of pair j
-              const float2 x = __ffma2_rn(make_float2(s[2 * j], s[2 * j + 1]), mul2, add2);
-              s[2 * j] = x.x;
-              s[2 * j + 1] = x.y;
+              float2 x = make_float2(s[2 * j], s[2 * j + 1]);
+              if (!kLogitsFirst) {
+                x = __ffma2_rn(x, mul2, add2);
+                s[2 * j] = x.x;
+                s[2 * j + 1] = x.y;
+              }
               if (kPolyMask & (1u << (j & 7))) {
                 const float2 y = exp2_poly2(x);
-                e[2 * (j & 7)] = y.x;
-                e[2 * (j & 7) + 1] = y.y;
+                e[2 * (j & (kRing - 1))] = y.x;
+                e[2 * (j & (kRing - 1)) + 1] = y.y;
               } else {
-                e[2 * (j & 7)] = ex2(x.x);
-                e[2 * (j & 7) + 1] = ex2(x.y);
+                e[2 * (j & (kRing - 1))] = ex2(x.x);
+                e[2 * (j & (kRing - 1)) + 1] = ex2(x.y);
               }
             }
           }

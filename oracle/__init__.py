@@ -94,6 +94,9 @@ def segment_sizes(T: int, H: int, W: int, n_cond: int, block: int = 64):
     """(Nc, Nn, Cb, Nb): condition / noisy token counts and block counts.
     Condition frames come first on the time axis (myzaker / QbitAI page,
     section on the unified tasks)."""
+    if min(T, H, W, block) <= 0 or not 0 <= n_cond <= T:
+        raise ValueError(f"bad sizes T={T} H={H} W={W} block={block} n_cond={n_cond} "
+                         "(n_cond counts latent frames, 0 <= n_cond <= T)")
     Nc = n_cond * H * W
     Nn = (T - n_cond) * H * W
     return Nc, Nn, -(-Nc // block), -(-Nn // block)

@@ -54,6 +54,9 @@ def _load():
         "lc_rope3d_apply": (S, [vp, vp, I, LL, I, I, LL, I, vp, vp]),
         "lc_bsa_forward": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_bsa_forward_cached": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_bsa_forward_cached_ex": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, ctypes.c_uint,
+                                         vp, vp, vp]),
+        "lc_bsa_cond_cache": (S, [vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_bsa_forward_noalloc": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
@@ -67,6 +70,7 @@ def _load():
 
 
 lib = _load()
+COND_K_ROTATED = 1  # LC_FLAG_COND_K_ROTATED
 
 
 def status_string(s: int) -> str:
@@ -226,10 +230,12 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope:
 def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Optional[torch.Tensor],
                    cond_v: Optional[torch.Tensor], plan: Plan, rope: Rope3D, *,
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                   return_lse: bool = False, softmax_scale: float = 0.0, stream=None):
+                   return_lse: bool = False, softmax_scale: float = 0.0,
+                   cond_k_rotated: bool = False, stream=None):
     """Noisy-query attention with the condition tokens' K/V passed separately
-    (lc_bsa_forward_cached).  q, k, v: [B, Nn, heads, 64]; cond_k, cond_v:
-    [B, Nc, heads, 64], pre-RoPE."""
+    (lc_bsa_forward_cached / lc_bsa_forward_cached_ex).  q, k, v:
+    [B, Nn, heads, 64]; cond_k, cond_v: [B, Nc, heads, 64], pre-RoPE, or
+    already rotated (cond_k_rotated=True, e.g. from cond_cache)."""
     B, Nn, heads, hd = q.shape
     Nc = plan.n_cond_tokens
     _check_bmhk("q", q, (B, plan.n_tokens - Nc, heads, hd), q.dtype)
@@ -247,11 +253,53 @@ def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Op
         lse = torch.empty(B, heads, Nn, dtype=torch.float32, device=q.device)
     if lse is not None:
         _check_bmhk("lse", lse, (B, heads, Nn), torch.float32)
-    _check(lib.lc_bsa_forward_cached(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k),
-                                     _ptr(cond_v), out.data_ptr(), _ptr(lse), B, heads, hd,
-                                     _dtype_code(q), float(softmax_scale), plan.handle,
-                                     rope.handle, _stream(stream)), "lc_bsa_forward_cached")
+    if cond_k_rotated:
+        _check(lib.lc_bsa_forward_cached_ex(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k), _ptr(cond_v), out.data_ptr(),
+            _ptr(lse), B, heads, hd, _dtype_code(q), float(softmax_scale), COND_K_ROTATED,
+            plan.handle, rope.handle, _stream(stream)), "lc_bsa_forward_cached_ex")
+    else:
+        _check(lib.lc_bsa_forward_cached(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k),
+                                         _ptr(cond_v), out.data_ptr(), _ptr(lse), B, heads, hd,
+                                         _dtype_code(q), float(softmax_scale), plan.handle,
+                                         rope.handle, _stream(stream)), "lc_bsa_forward_cached")
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def cond_cache(cond_k: torch.Tensor, plan: Plan, rope: Rope3D, *,
+               cond_q: Optional[torch.Tensor] = None, cond_v: Optional[torch.Tensor] = None,
+               cond_k_rot: Optional[torch.Tensor] = None, cond_out: Optional[torch.Tensor] = None,
+               cond_lse: Optional[torch.Tensor] = None, return_lse: bool = False,
+               softmax_scale: float = 0.0, stream=None):
+    """Producer side of the condition-token KV cache (lc_bsa_cond_cache):
+    returns cond_k_rot = R(cond_k) and, when cond_q and cond_v are given, the
+    condition tokens' own attention output (and lse with return_lse)."""
+    B, Nc, heads, hd = cond_k.shape
+    _check_bmhk("cond_k", cond_k, (B, plan.n_cond_tokens, heads, hd), cond_k.dtype)
+    want_out = cond_q is not None or cond_v is not None
+    if want_out:
+        if cond_q is None or cond_v is None:
+            raise ValueError("cond_q and cond_v go together")
+        _check_bmhk("cond_q", cond_q, cond_k.shape, cond_k.dtype)
+        _check_bmhk("cond_v", cond_v, cond_k.shape, cond_k.dtype)
+    if cond_k_rot is None:
+        cond_k_rot = torch.empty_like(cond_k)
+    _check_bmhk("cond_k_rot", cond_k_rot, cond_k.shape, cond_k.dtype)
+    if want_out and cond_out is None:
+        cond_out = torch.empty_like(cond_k)
+    if want_out and return_lse and cond_lse is None:
+        cond_lse = torch.empty(B, heads, Nc, dtype=torch.float32, device=cond_k.device)
+    if cond_out is not None:
+        _check_bmhk("cond_out", cond_out, cond_k.shape, cond_k.dtype)
+    if cond_lse is not None:
+        _check_bmhk("cond_lse", cond_lse, (B, heads, Nc), torch.float32)
+    _check(lib.lc_bsa_cond_cache(_ptr(cond_q), cond_k.data_ptr(), _ptr(cond_v),
+                                 cond_k_rot.data_ptr(), _ptr(cond_out), _ptr(cond_lse), B, heads,
+                                 hd, _dtype_code(cond_k), float(softmax_scale), plan.handle,
+                                 rope.handle, _stream(stream)), "lc_bsa_cond_cache")
+    if not want_out:
+        return cond_k_rot
+    return (cond_k_rot, cond_out, cond_lse) if cond_lse is not None else (cond_k_rot, cond_out)
 
 
 def forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D,

@@ -32,13 +32,14 @@ lc_status check_common(const lc_bsa_plan_s *plan, const lc_rope3d_s *rope, int b
 lc_status run_forward(const void *q, const void *k, const void *v, const void *cond_k,
                       const void *cond_v, void *out, float *lse, int batch, int heads, int head_dim,
                       lc_dtype dtype, float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
-                      void *stream, bool cached) {
+                      void *stream, lc_fwd_mode mode, bool cond_k_rotated) {
   lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
   if (s != LC_OK) return s;
-  if (!q || !k || !v || !out) return LC_ERR_INVALID_ARGUMENT;
-  if (cached && plan->Nc > 0 && (!cond_k || !cond_v)) return LC_ERR_INVALID_ARGUMENT;
-  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
-      (cached && plan->Nc > 0 && (misaligned(cond_k) || misaligned(cond_v))) ||
+  const bool cond_only = mode == LC_FWD_COND, split = mode != LC_FWD_FULL;
+  if (!q || !out || (!cond_only && (!k || !v))) return LC_ERR_INVALID_ARGUMENT;
+  if (split && plan->Nc > 0 && (!cond_k || !cond_v)) return LC_ERR_INVALID_ARGUMENT;
+  if (misaligned(q) || misaligned(out) || (!cond_only && (misaligned(k) || misaligned(v))) ||
+      (split && plan->Nc > 0 && (misaligned(cond_k) || misaligned(cond_v))) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return LC_ERR_INVALID_ARGUMENT;
   if (!(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;  // NaN
@@ -50,9 +51,10 @@ lc_status run_forward(const void *q, const void *k, const void *v, const void *c
     return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
                                  static_cast<const float *>(v), static_cast<const float *>(cond_k),
                                  static_cast<const float *>(cond_v), static_cast<float *>(out),
-                                 lse, batch, heads, scale, cached, plan, rope, dev_status, st);
-  return lc_launch_forward_sm100(q, k, v, cond_k, cond_v, out, lse, batch, heads, scale, cached,
-                                 plan, rope, dev_status, st);
+                                 lse, batch, heads, scale, mode, cond_k_rotated, plan, rope,
+                                 dev_status, st);
+  return lc_launch_forward_sm100(q, k, v, cond_k, cond_v, out, lse, batch, heads, scale, mode,
+                                 cond_k_rotated, plan, rope, dev_status, st);
 }
 
 }  // namespace
@@ -122,7 +124,7 @@ extern "C" lc_status lc_bsa_forward(const void *q, const void *k, const void *v,
                                     float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
                                     void *stream) {
   return run_forward(q, k, v, nullptr, nullptr, out, lse, batch, heads, head_dim, dtype,
-                     softmax_scale, plan, rope, stream, false);
+                     softmax_scale, plan, rope, stream, LC_FWD_FULL, false);
 }
 
 extern "C" lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
@@ -131,7 +133,43 @@ extern "C" lc_status lc_bsa_forward_cached(const void *q, const void *k, const v
                                            lc_dtype dtype, float softmax_scale, lc_bsa_plan plan,
                                            lc_rope3d rope, void *stream) {
   return run_forward(q, k, v, cond_k, cond_v, out, lse, batch, heads, head_dim, dtype,
-                     softmax_scale, plan, rope, stream, true);
+                     softmax_scale, plan, rope, stream, LC_FWD_CACHED, false);
+}
+
+extern "C" lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
+                                              const void *cond_k, const void *cond_v, void *out,
+                                              float *lse, int batch, int heads, int head_dim,
+                                              lc_dtype dtype, float softmax_scale, unsigned flags,
+                                              lc_bsa_plan plan, lc_rope3d rope, void *stream) {
+  if (flags & ~LC_FLAG_COND_K_ROTATED) return LC_ERR_INVALID_ARGUMENT;
+  return run_forward(q, k, v, cond_k, cond_v, out, lse, batch, heads, head_dim, dtype,
+                     softmax_scale, plan, rope, stream, LC_FWD_CACHED,
+                     (flags & LC_FLAG_COND_K_ROTATED) != 0);
+}
+
+extern "C" lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *cond_v,
+                                       void *cond_k_rot, void *cond_out, float *cond_lse,
+                                       int batch, int heads, int head_dim, lc_dtype dtype,
+                                       float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
+                                       void *stream) {
+  lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
+  if (s != LC_OK) return s;
+  if (plan->Nc == 0) return LC_OK;
+  if (!cond_k || !cond_k_rot || misaligned(cond_k) || misaligned(cond_k_rot))
+    return LC_ERR_INVALID_ARGUMENT;
+  const size_t elem = dtype == LC_DTYPE_F32 ? 4 : 2;
+  const uintptr_t bytes = (uintptr_t)batch * plan->Nc * heads * LC_HEAD_DIM * elem;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(cond_k), b0 = reinterpret_cast<uintptr_t>(cond_k_rot);
+  if (a0 < b0 + bytes && b0 < a0 + bytes) return LC_ERR_INVALID_ARGUMENT;  // overlap
+  if (cond_out && (!cond_q || !cond_v)) return LC_ERR_INVALID_ARGUMENT;
+  if (!cond_out && cond_lse) return LC_ERR_INVALID_ARGUMENT;
+  if (cond_out && !(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;
+  // R(cond_k): the same per-pair arithmetic as every rotation in the library.
+  s = lc_rope3d_apply(cond_k, cond_k_rot, batch, plan->Nc, heads, head_dim, 0, dtype, rope,
+                      stream);
+  if (s != LC_OK || !cond_out) return s;
+  return run_forward(cond_q, nullptr, nullptr, cond_k_rot, cond_v, cond_out, cond_lse, batch,
+                     heads, head_dim, dtype, softmax_scale, plan, rope, stream, LC_FWD_COND, true);
 }
 
 extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const void *v,
@@ -155,10 +193,10 @@ extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const 
   if (dtype == LC_DTYPE_F32)  // the fp32 kernel needs no scratch
     return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
                                  static_cast<const float *>(v), nullptr, nullptr,
-                                 static_cast<float *>(out), lse, batch, heads, scale, false, plan,
-                                 rope, scratch + 1, st);
-  return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale, false,
-                                 plan, rope, scratch + 1, st, scratch);
+                                 static_cast<float *>(out), lse, batch, heads, scale, LC_FWD_FULL,
+                                 false, plan, rope, scratch + 1, st);
+  return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale,
+                                 LC_FWD_FULL, false, plan, rope, scratch + 1, st, scratch);
 }
 
 extern "C" lc_status lc_last_device_status(void *stream) {

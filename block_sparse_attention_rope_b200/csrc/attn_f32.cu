@@ -21,7 +21,9 @@ struct F32Args {
   lc_divmod div_hw, div_w;
   int Nc, Nn, Cb, heads;
   int q_block0;    // first CSR row processed (Cb when only noisy queries)
-  int cached;
+  int split_kv;    // condition K/V in cond_k / cond_v, noisy K/V in k / v
+  int q_mode;      // rows of q / out: 0 all tokens, 1 noisy tokens, 2 condition tokens
+  int cond_k_rot;  // cond_k already holds R(k)
   float scale;
 };
 
@@ -39,16 +41,14 @@ __device__ __forceinline__ void rope_row(float *x, int n, const F32Args &a) {
     if (p < 8) { c = cT[t * 8 + p]; s = sT[t * 8 + p]; }
     else if (p < 20) { c = cH[h * 12 + p - 8]; s = sH[h * 12 + p - 8]; }
     else { c = cW[w * 12 + p - 20]; s = sW[w * 12 + p - 20]; }
-    float x0 = x[2 * p], x1 = x[2 * p + 1];
-    x[2 * p] = x0 * c - x1 * s;
-    x[2 * p + 1] = x0 * s + x1 * c;
+    lc_rot_pair(x[2 * p], x[2 * p + 1], c, s, x[2 * p], x[2 * p + 1]);
   }
 }
 
 // Address of head `h` of sequence token m (full-sequence index) for K or V.
 __device__ __forceinline__ const float *kv_row(const float *full, const float *cond, int b, int m,
                                                int h, const F32Args &a) {
-  if (!a.cached) {
+  if (!a.split_kv) {
     long long N = (long long)a.Nc + a.Nn;
     return full + (((long long)b * N + m) * a.heads + h) * LC_HEAD_DIM;
   }
@@ -69,8 +69,8 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
   const int n = q_lo + tid;
   const bool valid = n < q_hi;
   // Row of the q / out tensors that holds token n.
-  const int q_row = a.cached ? n - a.Nc : n;
-  const long long Nq = a.cached ? a.Nn : (long long)a.Nc + a.Nn;
+  const int q_row = a.q_mode == 1 ? n - a.Nc : n;
+  const long long Nq = a.q_mode == 1 ? a.Nn : (a.q_mode == 2 ? a.Nc : (long long)a.Nc + a.Nn);
 
   float q[LC_HEAD_DIM], o[LC_HEAD_DIM];
   if (valid) {
@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
       const float *vs = kv_row(a.v, a.cond_v, b, m, h, a);
 #pragma unroll
       for (int d = 0; d < LC_HEAD_DIM; ++d) kr[d] = ks[d];
-      rope_row(kr, m, a);
+      if (!(a.cond_k_rot && m < a.Nc)) rope_row(kr, m, a);
 #pragma unroll
       for (int d = 0; d < LC_HEAD_DIM; ++d) {
         sK[tid][d] = kr[d];
@@ -141,9 +141,10 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
 
 lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 const float *cond_k, const float *cond_v, float *out, float *lse,
-                                int batch, int heads, float scale, bool cached,
-                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                int * /*dev_status*/, cudaStream_t stream) {
+                                int batch, int heads, float scale, lc_fwd_mode mode,
+                                bool cond_k_rotated, const lc_bsa_plan_s *plan,
+                                const lc_rope3d_s *rope, int * /*dev_status*/,
+                                cudaStream_t stream) {
   F32Args a;
   a.q = q; a.k = k; a.v = v; a.cond_k = cond_k; a.cond_v = cond_v;
   a.out = out; a.lse = lse;
@@ -153,10 +154,12 @@ lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
   a.div_hw = lc_make_divmod(rope->H * rope->W);
   a.div_w = lc_make_divmod(rope->W);
   a.Nc = plan->Nc; a.Nn = plan->Nn; a.Cb = plan->Cb; a.heads = heads;
-  a.cached = cached ? 1 : 0;
-  a.q_block0 = cached ? plan->Cb : 0;
+  a.split_kv = mode != LC_FWD_FULL;
+  a.q_mode = mode == LC_FWD_CACHED ? 1 : (mode == LC_FWD_COND ? 2 : 0);
+  a.cond_k_rot = (mode != LC_FWD_FULL && cond_k_rotated) ? 1 : 0;
+  a.q_block0 = mode == LC_FWD_CACHED ? plan->Cb : 0;
   a.scale = scale;
-  int nrows = cached ? plan->Nb : plan->nq;
+  int nrows = mode == LC_FWD_CACHED ? plan->Nb : (mode == LC_FWD_COND ? plan->Cb : plan->nq);
   if (nrows == 0) return LC_OK;
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));

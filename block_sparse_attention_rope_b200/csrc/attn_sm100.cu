@@ -102,6 +102,7 @@ struct __align__(64) Sm100Params {
   int T, H, W;
   int Nc, Nn, Cb, gc;
   int heads, n_groups_active, total_items;
+  int group_offset;        // first rank of grp_order this launch works on
   int lse_nq;              // rows of the lse tensor per (batch, head)
   int q_row_offset_noisy;  // row of the q/out/lse tensors holding noisy token 0
   int tab_floats;
@@ -190,7 +191,7 @@ __device__ __forceinline__ Item decode_item(const Sm100Params &p, int item) {
   Item it;
   int per = p.n_groups_active;
   int bh = item / per;
-  int g = p.grp_order[item - bh * per];
+  int g = p.grp_order[p.group_offset + item - bh * per];
   it.b = bh / p.heads;
   it.h = bh - it.b * p.heads;
   it.seg = g < p.gc ? 0 : 1;
@@ -274,7 +275,9 @@ __device__ __forceinline__ void rope_row(uint8_t *tile, int r, int n, const floa
     for (int q = 0; q < 4; ++q) {
       const float a = __uint_as_float(wds[q] << 16);
       const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
-      __nv_bfloat162 o2 = __floats2bfloat162_rn(a * cs[q] - b * sn[q], a * sn[q] + b * cs[q]);
+      float xr, yr;
+      lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
+      __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
       wds[q] = *reinterpret_cast<uint32_t *>(&o2);
     }
     *ptr = make_uint4(wds[0], wds[1], wds[2], wds[3]);
@@ -1005,7 +1008,9 @@ __global__ void rope_k_kernel(const uint4 *src, uint4 *dst, long long n_chunks, 
     for (int q = 0; q < 4; ++q) {
       const float a = __uint_as_float(wds[q] << 16);
       const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
-      __nv_bfloat162 o2 = __floats2bfloat162_rn(a * cs[q] - b * sn[q], a * sn[q] + b * cs[q]);
+      float xr, yr;
+      lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
+      __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
       wds[q] = *reinterpret_cast<uint32_t *>(&o2);
     }
     dst[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
@@ -1067,14 +1072,29 @@ int *lc_noalloc_scratch(lc_status *st) {
 
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, const void *cond_k,
                                   const void *cond_v, void *out, float *lse, int batch, int heads,
-                                  float scale, bool cached, const lc_bsa_plan_s *plan,
-                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
-                                  int *counter_scratch) {
+                                  float scale, lc_fwd_mode mode, bool cond_k_rotated,
+                                  const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                  int *dev_status, cudaStream_t stream, int *counter_scratch) {
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
   const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
+  const bool cached = mode == LC_FWD_CACHED, cond_only = mode == LC_FWD_COND;
+  if (counter_scratch && mode != LC_FWD_FULL) return LC_ERR_UNSUPPORTED;
+  if (cond_only && Nc == 0) return LC_OK;
   lc_status s = LC_OK;
-  if (cached) {
+  if (cond_only) {  // condition queries over condition keys only
+    s = encode_segment(&prm.tmQ[0], q, batch, Nc, 0, Nc, heads);
+    if (s == LC_OK) s = encode_segment(&prm.tmO[0], out, batch, Nc, 0, Nc, heads);
+    if (s == LC_OK) s = encode_segment(&prm.tmK[0], cond_k, batch, Nc, 0, Nc, heads);
+    if (s == LC_OK) s = encode_segment(&prm.tmV[0], cond_v, batch, Nc, 0, Nc, heads);
+    prm.q_row_offset_noisy = 0;
+    prm.lse_nq = (int)Nc;
+    // grp_order ranks noisy groups first (every noisy list holds all Cb
+    // condition blocks plus at least one noisy block, so it is longer than
+    // any condition list); the condition groups are the last gc ranks.
+    prm.group_offset = plan->gn;
+    prm.n_groups_active = plan->gc;
+  } else if (cached) {
     s = encode_segment(&prm.tmQ[1], q, batch, Nn, 0, Nn, heads);
     if (s == LC_OK) s = encode_segment(&prm.tmO[1], out, batch, Nn, 0, Nn, heads);
     if (s == LC_OK) s = encode_segment(&prm.tmK[1], k, batch, Nn, 0, Nn, heads);
@@ -1085,6 +1105,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     }
     prm.q_row_offset_noisy = 0;
     prm.lse_nq = (int)Nn;
+    prm.group_offset = 0;
     prm.n_groups_active = plan->gn;
   } else {
     s = encode_segment(&prm.tmQ[1], q, batch, N, Nc, Nn, heads);
@@ -1099,10 +1120,14 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     }
     prm.q_row_offset_noisy = (int)Nc;
     prm.lse_nq = (int)N;
+    prm.group_offset = 0;
     prm.n_groups_active = plan->G;
   }
   if (s != LC_OK) return s;
-  if (Nc == 0) {  // keep the unused condition maps valid descriptors
+  if (cond_only) {  // keep the unused noisy maps valid descriptors
+    prm.tmQ[1] = prm.tmQ[0]; prm.tmK[1] = prm.tmK[0];
+    prm.tmV[1] = prm.tmV[0]; prm.tmO[1] = prm.tmO[0];
+  } else if (Nc == 0) {  // keep the unused condition maps valid descriptors
     prm.tmQ[0] = prm.tmQ[1]; prm.tmK[0] = prm.tmK[1];
     prm.tmV[0] = prm.tmV[1]; prm.tmO[0] = prm.tmO[1];
   } else if (cached) {
@@ -1169,20 +1194,26 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   cudaError_t e = cudaStreamWaitEvent(stream, rope->ready, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
   if (e == cudaSuccess && k_prepass) {
-    const size_t kb = (size_t)batch * (cached ? Nn : N) * heads * LC_HEAD_DIM * 2;
-    e = cudaMallocFromPoolAsync(&k_rot, kb, pool, stream);
-    if (e == cudaSuccess)
-      s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
-                        stream);
-    if (e == cudaSuccess && s == LC_OK && cached && Nc > 0) {
+    // K of the query-side tensor (all tokens, or the noisy ones).
+    if (!cond_only) {
+      const size_t kb = (size_t)batch * (cached ? Nn : N) * heads * LC_HEAD_DIM * 2;
+      e = cudaMallocFromPoolAsync(&k_rot, kb, pool, stream);
+      if (e == cudaSuccess)
+        s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
+                          stream);
+    }
+    // Separately supplied condition K, unless the caller rotated it already.
+    if (e == cudaSuccess && s == LC_OK && (cached || cond_only) && Nc > 0 && !cond_k_rotated) {
       e = cudaMallocFromPoolAsync(&ck_rot, (size_t)batch * Nc * heads * LC_HEAD_DIM * 2, pool,
                                   stream);
       if (e == cudaSuccess) s = launch_rope_k(cond_k, ck_rot, batch, Nc, heads, 0, rope, stream);
     }
     if (e == cudaSuccess && s == LC_OK) {
-      if (cached) {
-        s = encode_segment(&prm.tmK[1], k_rot, batch, Nn, 0, Nn, heads);
-        if (s == LC_OK && Nc > 0) s = encode_segment(&prm.tmK[0], ck_rot, batch, Nc, 0, Nc, heads);
+      if (ck_rot) s = encode_segment(&prm.tmK[0], ck_rot, batch, Nc, 0, Nc, heads);
+      if (cond_only) {
+        prm.tmK[1] = prm.tmK[0];
+      } else if (cached) {
+        if (s == LC_OK) s = encode_segment(&prm.tmK[1], k_rot, batch, Nn, 0, Nn, heads);
         if (s == LC_OK && Nc == 0) prm.tmK[0] = prm.tmK[1];
       } else {
         s = encode_segment(&prm.tmK[1], k_rot, batch, N, Nc, Nn, heads);

@@ -90,19 +90,40 @@ __device__ __forceinline__ int lc_div(int n, lc_divmod dm) {
   return (int)(((unsigned long long)(unsigned)n * dm.m) >> 40);
 }
 
+// One RoPE channel pair (a, b) rotated by the angle with cosine c and sine s:
+// (a c - b s, a s + b c), each as one rounded product and one fused
+// multiply-add, spelled out so that every kernel that rotates (Q and K tiles,
+// the K pass, the public rotation, the fp32 path) produces the same bits for
+// the same input whatever the compiler would contract.
+__device__ __forceinline__ void lc_rot_pair(float a, float b, float c, float s, float &x,
+                                            float &y) {
+  x = __fmaf_rn(a, c, -__fmul_rn(b, s));
+  y = __fmaf_rn(a, s, __fmul_rn(b, c));
+}
+
 // Launch helpers implemented by the kernel translation units.
+// Which queries an attention launch computes and where its tensors live.
+//   LC_FWD_FULL    q, k, v, out hold all N tokens (cond_k / cond_v unused).
+//   LC_FWD_CACHED  q, k, v, out hold the Nn noisy tokens; the condition
+//                  tokens' K/V come from cond_k / cond_v ([B, Nc, heads, 64]).
+//   LC_FWD_COND    only the condition queries: q and out hold the Nc condition
+//                  tokens, K/V come from cond_k / cond_v (k and v unused).
+// cond_k_rotated: cond_k already holds R(k) (CACHED and COND only).
+enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2 };
+
 lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 const float *cond_k, const float *cond_v, float *out,
-                                float *lse, int batch, int heads, float scale, bool cached,
-                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                int *dev_status, cudaStream_t stream);
+                                float *lse, int batch, int heads, float scale, lc_fwd_mode mode,
+                                bool cond_k_rotated, const lc_bsa_plan_s *plan,
+                                const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream);
 // counter_scratch: NULL = allocate the scheduler counter stream-ordered for
-// this launch; else a device int the caller provides (lc_bsa_forward_noalloc).
+// this launch; else a device int the caller provides (lc_bsa_forward_noalloc,
+// LC_FWD_FULL only).
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
                                   const void *cond_k, const void *cond_v, void *out,
-                                  float *lse, int batch, int heads, float scale, bool cached,
-                                  const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                  int *dev_status, cudaStream_t stream,
+                                  float *lse, int batch, int heads, float scale, lc_fwd_mode mode,
+                                  bool cond_k_rotated, const lc_bsa_plan_s *plan,
+                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
                                   int *counter_scratch = nullptr);
 
 // Fixed scratch of lc_bsa_forward_noalloc (attn_sm100.cu): device address of

@@ -54,10 +54,8 @@ __device__ __forceinline__ void rotate_chunk(float (&x)[8], int ch, int t, int h
   }
 #pragma unroll
   for (int p = 0; p < 4; ++p) {
-    float a = x[2 * p], b = x[2 * p + 1];
-    float cc = c[p], ss = s[p];
-    x[2 * p] = a * cc - b * ss;
-    x[2 * p + 1] = a * ss + b * cc;
+    const float a = x[2 * p], b = x[2 * p + 1];
+    lc_rot_pair(a, b, c[p], s[p], x[2 * p], x[2 * p + 1]);
   }
 }
 

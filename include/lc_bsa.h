@@ -176,6 +176,47 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
                                 lc_dtype dtype, float softmax_scale, lc_bsa_plan plan,
                                 lc_rope3d rope, void *stream);
 
+/* Flags of lc_bsa_forward_cached_ex. */
+#define LC_FLAG_COND_K_ROTATED 1u  /* cond_k already holds R(k) (lc_bsa_cond_cache) */
+
+/*
+ * lc_bsa_forward_cached_ex -- lc_bsa_forward_cached with flags.  With
+ * LC_FLAG_COND_K_ROTATED, cond_k is taken as already rotated (the cond_k_rot
+ * output of lc_bsa_cond_cache) and is not rotated again, so a cache built once
+ * serves every later call.  The results equal lc_bsa_forward_cached's on the
+ * pre-RoPE cond_k bit for bit.  Unknown flag bits: LC_ERR_INVALID_ARGUMENT;
+ * other errors as lc_bsa_forward.
+ */
+lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
+                                   const void *cond_k, const void *cond_v, void *out,
+                                   float *lse, int batch, int heads, int head_dim,
+                                   lc_dtype dtype, float softmax_scale, unsigned flags,
+                                   lc_bsa_plan plan, lc_rope3d rope, void *stream);
+
+/*
+ * lc_bsa_cond_cache -- the producer side of the condition-token KV cache
+ * (myzaker / QbitAI "背后技术原理", on the block attention with a KV cache:
+ * condition tokens never attend noise tokens, so their K/V features, and
+ * their own attention outputs, are computed once and reused at every later
+ * denoising step).  From the condition tokens' pre-RoPE cond_k it writes
+ * cond_k_rot = R(cond_k) with t in [0, n_cond_frames), the exact values the
+ * attention entry points rotate internally, for lc_bsa_forward_cached_ex with
+ * LC_FLAG_COND_K_ROTATED.  If cond_out is not NULL it also computes the
+ * condition tokens' attention (condition queries over condition keys, the
+ * condition rows of lc_bsa_forward on the whole sequence) into cond_out and,
+ * if cond_lse is not NULL, their lse.
+ *   cond_q, cond_k, cond_v, cond_k_rot, cond_out: [batch, Nc, heads, head_dim]
+ *   of dtype, 16-byte aligned; cond_lse: [batch, heads, Nc] fp32.  cond_q and
+ *   cond_v are read only when cond_out is given (else they may be NULL).
+ *   cond_k_rot must not overlap cond_k; the caller owns every buffer.
+ * With n_cond_frames == 0 there is nothing to do (LC_OK).  Errors as
+ * lc_bsa_forward.
+ */
+lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *cond_v,
+                            void *cond_k_rot, void *cond_out, float *cond_lse, int batch,
+                            int heads, int head_dim, lc_dtype dtype, float softmax_scale,
+                            lc_bsa_plan plan, lc_rope3d rope, void *stream);
+
 /*
  * lc_bsa_forward_noalloc -- lc_bsa_forward for callers that cannot allocate
  * device memory during the call: an application whose allocator owns all of

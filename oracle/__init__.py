@@ -131,6 +131,23 @@ def rope3d_apply(x, H: int, W: int, tok_offset: int = 0,
 
 
 # --------------------------------------------------------------------------
+# RMSNorm of q and k ahead of RoPE
+# --------------------------------------------------------------------------
+def rms_norm(x, weight, eps: float) -> np.ndarray:
+    """RMSNorm over the head dimension of x [..., hd]: x / sqrt(mean(x^2) +
+    eps) * weight, in fp64.  myzaker / QbitAI, section "背后技术原理": the
+    self- and cross-attention modules use RMSNorm for training stability.
+    Reading taken (the page gives no formula): the norm is applied to q and k
+    per token and per head over the 64 channels, with one learned weight per
+    channel shared by the heads, before the 3D-RoPE rotation."""
+    xf = _f64(x)
+    w = np.asarray(weight, dtype=np.float64).reshape(-1)
+    assert w.shape[0] == xf.shape[-1]
+    ms = np.mean(xf * xf, axis=-1, keepdims=True)
+    return xf / np.sqrt(ms + eps) * w
+
+
+# --------------------------------------------------------------------------
 # Mask
 # --------------------------------------------------------------------------
 def noisy_block_rule(i: int, j: int, local: int, stride: int) -> bool:
@@ -167,14 +184,21 @@ def attention_rows(q, k, v, *, H: int, W: int, Nc: int, block: int, local: int,
                    stride: int, rows, q_offset: int = 0, scale: Optional[float] = None,
                    theta: float = ROPE_THETA, dims: Sequence[int] = ROPE_DIMS,
                    nthreads: int = 0, q_rotated: Optional[np.ndarray] = None,
-                   k_rotated: Optional[np.ndarray] = None):
+                   k_rotated: Optional[np.ndarray] = None, q_norm=None, k_norm=None,
+                   norm_eps: float = 1e-6):
     """Masked softmax attention on RoPE-rotated q/k for selected rows.
 
     q: [B, Nq, heads, hd] (query r is token r + q_offset of the sequence);
     k, v: [B, N, heads, hd] (the full condition + noisy sequence);
-    rows: int array [R, 3] of (b, head, r).  Returns (out [R, hd], lse [R]).
+    rows: int array [R, 3] of (b, head, r).  q_norm / k_norm: optional
+    per-channel RMSNorm weights applied to q / k before the rotation.
+    Returns (out [R, hd], lse [R]).
     """
     qf = _f64(q)
+    if q_norm is not None and q_rotated is None:
+        qf = rms_norm(qf, q_norm, norm_eps)
+    if k_norm is not None and k_rotated is None:
+        k = rms_norm(k, k_norm, norm_eps)
     B, Nq, heads, hd = qf.shape
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
     qrot = q_rotated if q_rotated is not None else rope3d_apply(qf, H, W, q_offset, theta, dims)
@@ -200,7 +224,8 @@ def all_rows(B: int, Nq: int, heads: int) -> np.ndarray:
 
 
 def forward(q, k, v, *, T: int, H: int, W: int, n_cond: int, block: int = 64,
-            local: int, stride: int, scale: Optional[float] = None, nthreads: int = 0):
+            local: int, stride: int, scale: Optional[float] = None, nthreads: int = 0,
+            q_norm=None, k_norm=None, norm_eps: float = 1e-6):
     """Whole-layer oracle over the full sequence (q, k, v: [B, N, heads, hd]).
     Returns out [B, N, heads, hd] and lse [B, heads, N] (fp64)."""
     qf = _f64(q)
@@ -209,7 +234,8 @@ def forward(q, k, v, *, T: int, H: int, W: int, n_cond: int, block: int = 64,
     Nc = n_cond * H * W
     rows = all_rows(B, N, heads)
     o, l = attention_rows(qf, k, v, H=H, W=W, Nc=Nc, block=block, local=local,
-                          stride=stride, rows=rows, scale=scale, nthreads=nthreads)
+                          stride=stride, rows=rows, scale=scale, nthreads=nthreads,
+                          q_norm=q_norm, k_norm=k_norm, norm_eps=norm_eps)
     out = np.zeros((B, N, heads, hd))
     lse = np.zeros((B, heads, N))
     out[rows[:, 0], rows[:, 2], rows[:, 1]] = o
@@ -219,7 +245,8 @@ def forward(q, k, v, *, T: int, H: int, W: int, n_cond: int, block: int = 64,
 
 def forward_cached(q, k, v, cond_k, cond_v, *, T: int, H: int, W: int, n_cond: int,
                    block: int = 64, local: int, stride: int,
-                   scale: Optional[float] = None, nthreads: int = 0):
+                   scale: Optional[float] = None, nthreads: int = 0,
+                   q_norm=None, k_norm=None, norm_eps: float = 1e-6):
     """Oracle of the cached form: q/k/v hold the noisy tokens only, cond_k /
     cond_v the condition tokens (pre-RoPE).  The keys are the condition tokens
     followed by the noisy tokens; noisy query r is token Nc + r.
@@ -233,7 +260,8 @@ def forward_cached(q, k, v, cond_k, cond_v, *, T: int, H: int, W: int, n_cond: i
     rows = all_rows(B, Nn, heads)
     o, l = attention_rows(qf, kf, vf, H=H, W=W, Nc=Nc, block=block, local=local,
                           stride=stride, rows=rows, q_offset=Nc, scale=scale,
-                          nthreads=nthreads)
+                          nthreads=nthreads, q_norm=q_norm, k_norm=k_norm,
+                          norm_eps=norm_eps)
     out = np.zeros((B, Nn, heads, hd))
     lse = np.zeros((B, heads, Nn))
     out[rows[:, 0], rows[:, 2], rows[:, 1]] = o

@@ -37,6 +37,12 @@ class PlanInfo(ctypes.Structure):
                 ("attended_token_pairs_noisy", ctypes.c_longlong)]
 
 
+class Opts(ctypes.Structure):
+    """lc_bsa_opts."""
+    _fields_ = [("flags", ctypes.c_uint), ("q_norm_weight", ctypes.c_void_p),
+                ("k_norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError("liblcbsa.so is not built (python -m block_sparse_attention_rope_b200.build)")
@@ -54,9 +60,10 @@ def _load():
         "lc_rope3d_apply": (S, [vp, vp, I, LL, I, I, LL, I, vp, vp]),
         "lc_bsa_forward": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_bsa_forward_cached": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
-        "lc_bsa_forward_cached_ex": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, ctypes.c_uint,
-                                         vp, vp, vp]),
-        "lc_bsa_cond_cache": (S, [vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_bsa_forward_ex": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp, vp]),
+        "lc_bsa_forward_cached_ex": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp,
+                                         vp]),
+        "lc_bsa_cond_cache": (S, [vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp, vp]),
         "lc_bsa_forward_noalloc": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
@@ -203,10 +210,26 @@ class Rope3D:
             pass
 
 
+def _opts(flags: int = 0, q_norm: Optional[torch.Tensor] = None,
+          k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, hd: int = 64):
+    """lc_bsa_opts for the _ex entry points, or None when nothing is set.
+    q_norm / k_norm: fp32 [head_dim] device tensors (RMSNorm weights)."""
+    for name, t in (("q_norm", q_norm), ("k_norm", k_norm)):
+        if t is not None and (not t.is_cuda or t.dtype != torch.float32 or
+                              tuple(t.shape) != (hd,) or not t.is_contiguous()):
+            raise ValueError("%s must be a contiguous fp32 CUDA tensor of shape (%d,)" % (name, hd))
+    if not flags and q_norm is None and k_norm is None:
+        return None
+    return Opts(flags, _ptr(q_norm), _ptr(k_norm), float(norm_eps))
+
+
 def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D, *,
             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-            return_lse: bool = False, softmax_scale: float = 0.0, stream=None):
-    """Block-sparse 3D-RoPE attention over the full sequence (lc_bsa_forward).
+            return_lse: bool = False, softmax_scale: float = 0.0,
+            q_norm: Optional[torch.Tensor] = None, k_norm: Optional[torch.Tensor] = None,
+            norm_eps: float = 1e-6, stream=None):
+    """Block-sparse 3D-RoPE attention over the full sequence (lc_bsa_forward,
+    or lc_bsa_forward_ex with RMSNorm weights q_norm / k_norm).
 
     q, k, v: [B, T*H*W, heads, 64], bf16 or fp32, on the plan's device.
     Returns out (and lse [B, heads, N] fp32 when asked)."""
@@ -221,9 +244,16 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope:
         lse = torch.empty(B, heads, N, dtype=torch.float32, device=q.device)
     if lse is not None:
         _check_bmhk("lse", lse, (B, heads, N), torch.float32)
-    _check(lib.lc_bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse),
-                              B, heads, hd, _dtype_code(q), float(softmax_scale), plan.handle,
-                              rope.handle, _stream(stream)), "lc_bsa_forward")
+    opts = _opts(0, q_norm, k_norm, norm_eps, hd)
+    if opts is not None:
+        _check(lib.lc_bsa_forward_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     _ptr(lse), B, heads, hd, _dtype_code(q), float(softmax_scale),
+                                     ctypes.byref(opts), plan.handle, rope.handle,
+                                     _stream(stream)), "lc_bsa_forward_ex")
+    else:
+        _check(lib.lc_bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  _ptr(lse), B, heads, hd, _dtype_code(q), float(softmax_scale),
+                                  plan.handle, rope.handle, _stream(stream)), "lc_bsa_forward")
     return (out, lse) if (return_lse or lse is not None) else out
 
 
@@ -231,7 +261,8 @@ def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Op
                    cond_v: Optional[torch.Tensor], plan: Plan, rope: Rope3D, *,
                    out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                    return_lse: bool = False, softmax_scale: float = 0.0,
-                   cond_k_rotated: bool = False, stream=None):
+                   cond_k_rotated: bool = False, q_norm: Optional[torch.Tensor] = None,
+                   k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None):
     """Noisy-query attention with the condition tokens' K/V passed separately
     (lc_bsa_forward_cached / lc_bsa_forward_cached_ex).  q, k, v:
     [B, Nn, heads, 64]; cond_k, cond_v: [B, Nc, heads, 64], pre-RoPE, or
@@ -253,10 +284,11 @@ def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Op
         lse = torch.empty(B, heads, Nn, dtype=torch.float32, device=q.device)
     if lse is not None:
         _check_bmhk("lse", lse, (B, heads, Nn), torch.float32)
-    if cond_k_rotated:
+    opts = _opts(COND_K_ROTATED if cond_k_rotated else 0, q_norm, k_norm, norm_eps, hd)
+    if opts is not None:
         _check(lib.lc_bsa_forward_cached_ex(
             q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k), _ptr(cond_v), out.data_ptr(),
-            _ptr(lse), B, heads, hd, _dtype_code(q), float(softmax_scale), COND_K_ROTATED,
+            _ptr(lse), B, heads, hd, _dtype_code(q), float(softmax_scale), ctypes.byref(opts),
             plan.handle, rope.handle, _stream(stream)), "lc_bsa_forward_cached_ex")
     else:
         _check(lib.lc_bsa_forward_cached(q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(cond_k),
@@ -270,7 +302,8 @@ def cond_cache(cond_k: torch.Tensor, plan: Plan, rope: Rope3D, *,
                cond_q: Optional[torch.Tensor] = None, cond_v: Optional[torch.Tensor] = None,
                cond_k_rot: Optional[torch.Tensor] = None, cond_out: Optional[torch.Tensor] = None,
                cond_lse: Optional[torch.Tensor] = None, return_lse: bool = False,
-               softmax_scale: float = 0.0, stream=None):
+               softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
+               k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None):
     """Producer side of the condition-token KV cache (lc_bsa_cond_cache):
     returns cond_k_rot = R(cond_k) and, when cond_q and cond_v are given, the
     condition tokens' own attention output (and lse with return_lse)."""
@@ -293,9 +326,11 @@ def cond_cache(cond_k: torch.Tensor, plan: Plan, rope: Rope3D, *,
         _check_bmhk("cond_out", cond_out, cond_k.shape, cond_k.dtype)
     if cond_lse is not None:
         _check_bmhk("cond_lse", cond_lse, (B, heads, Nc), torch.float32)
+    opts = _opts(0, q_norm, k_norm, norm_eps, hd)
     _check(lib.lc_bsa_cond_cache(_ptr(cond_q), cond_k.data_ptr(), _ptr(cond_v),
                                  cond_k_rot.data_ptr(), _ptr(cond_out), _ptr(cond_lse), B, heads,
-                                 hd, _dtype_code(cond_k), float(softmax_scale), plan.handle,
+                                 hd, _dtype_code(cond_k), float(softmax_scale),
+                                 None if opts is None else ctypes.byref(opts), plan.handle,
                                  rope.handle, _stream(stream)), "lc_bsa_cond_cache")
     if not want_out:
         return cond_k_rot

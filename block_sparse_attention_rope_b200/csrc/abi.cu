@@ -32,7 +32,8 @@ lc_status check_common(const lc_bsa_plan_s *plan, const lc_rope3d_s *rope, int b
 lc_status run_forward(const void *q, const void *k, const void *v, const void *cond_k,
                       const void *cond_v, void *out, float *lse, int batch, int heads, int head_dim,
                       lc_dtype dtype, float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
-                      void *stream, lc_fwd_mode mode, bool cond_k_rotated) {
+                      void *stream, lc_fwd_mode mode, bool cond_k_rotated,
+                      const lc_qk_norm &norm = lc_qk_norm()) {
   lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
   if (s != LC_OK) return s;
   const bool cond_only = mode == LC_FWD_COND, split = mode != LC_FWD_FULL;
@@ -51,10 +52,29 @@ lc_status run_forward(const void *q, const void *k, const void *v, const void *c
     return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
                                  static_cast<const float *>(v), static_cast<const float *>(cond_k),
                                  static_cast<const float *>(cond_v), static_cast<float *>(out),
-                                 lse, batch, heads, scale, mode, cond_k_rotated, plan, rope,
-                                 dev_status, st);
+                                 lse, batch, heads, scale, mode, cond_k_rotated, norm, plan,
+                                 rope, dev_status, st);
   return lc_launch_forward_sm100(q, k, v, cond_k, cond_v, out, lse, batch, heads, scale, mode,
-                                 cond_k_rotated, plan, rope, dev_status, st);
+                                 cond_k_rotated, norm, plan, rope, dev_status, st);
+}
+
+// Options -> flags and norm; false on a bad option.
+bool parse_opts(const lc_bsa_opts *opts, unsigned allowed_flags, unsigned *flags,
+                lc_qk_norm *norm) {
+  *flags = 0;
+  *norm = lc_qk_norm();
+  if (!opts) return true;
+  if (opts->flags & ~allowed_flags) return false;
+  *flags = opts->flags;
+  const bool any = opts->q_norm_weight || opts->k_norm_weight;
+  if (any && !(opts->norm_eps >= 0.f && opts->norm_eps <= 3.0e38f)) return false;  // NaN, inf
+  if ((reinterpret_cast<uintptr_t>(opts->q_norm_weight) |
+       reinterpret_cast<uintptr_t>(opts->k_norm_weight)) & 3u)
+    return false;
+  norm->q_w = opts->q_norm_weight;
+  norm->k_w = opts->k_norm_weight;
+  norm->eps = opts->norm_eps;
+  return true;
 }
 
 }  // namespace
@@ -136,24 +156,42 @@ extern "C" lc_status lc_bsa_forward_cached(const void *q, const void *k, const v
                      softmax_scale, plan, rope, stream, LC_FWD_CACHED, false);
 }
 
+extern "C" lc_status lc_bsa_forward_ex(const void *q, const void *k, const void *v, void *out,
+                                       float *lse, int batch, int heads, int head_dim,
+                                       lc_dtype dtype, float softmax_scale,
+                                       const lc_bsa_opts *opts, lc_bsa_plan plan, lc_rope3d rope,
+                                       void *stream) {
+  unsigned flags;
+  lc_qk_norm norm;
+  if (!parse_opts(opts, 0u, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
+  return run_forward(q, k, v, nullptr, nullptr, out, lse, batch, heads, head_dim, dtype,
+                     softmax_scale, plan, rope, stream, LC_FWD_FULL, false, norm);
+}
+
 extern "C" lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
                                               const void *cond_k, const void *cond_v, void *out,
                                               float *lse, int batch, int heads, int head_dim,
-                                              lc_dtype dtype, float softmax_scale, unsigned flags,
-                                              lc_bsa_plan plan, lc_rope3d rope, void *stream) {
-  if (flags & ~LC_FLAG_COND_K_ROTATED) return LC_ERR_INVALID_ARGUMENT;
+                                              lc_dtype dtype, float softmax_scale,
+                                              const lc_bsa_opts *opts, lc_bsa_plan plan,
+                                              lc_rope3d rope, void *stream) {
+  unsigned flags;
+  lc_qk_norm norm;
+  if (!parse_opts(opts, LC_FLAG_COND_K_ROTATED, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
   return run_forward(q, k, v, cond_k, cond_v, out, lse, batch, heads, head_dim, dtype,
                      softmax_scale, plan, rope, stream, LC_FWD_CACHED,
-                     (flags & LC_FLAG_COND_K_ROTATED) != 0);
+                     (flags & LC_FLAG_COND_K_ROTATED) != 0, norm);
 }
 
 extern "C" lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *cond_v,
                                        void *cond_k_rot, void *cond_out, float *cond_lse,
                                        int batch, int heads, int head_dim, lc_dtype dtype,
-                                       float softmax_scale, lc_bsa_plan plan, lc_rope3d rope,
-                                       void *stream) {
+                                       float softmax_scale, const lc_bsa_opts *opts,
+                                       lc_bsa_plan plan, lc_rope3d rope, void *stream) {
   lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
   if (s != LC_OK) return s;
+  unsigned flags;
+  lc_qk_norm norm;
+  if (!parse_opts(opts, 0u, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
   if (plan->Nc == 0) return LC_OK;
   if (!cond_k || !cond_k_rot || misaligned(cond_k) || misaligned(cond_k_rot))
     return LC_ERR_INVALID_ARGUMENT;
@@ -164,12 +202,14 @@ extern "C" lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, c
   if (cond_out && (!cond_q || !cond_v)) return LC_ERR_INVALID_ARGUMENT;
   if (!cond_out && cond_lse) return LC_ERR_INVALID_ARGUMENT;
   if (cond_out && !(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;
-  // R(cond_k): the same per-pair arithmetic as every rotation in the library.
-  s = lc_rope3d_apply(cond_k, cond_k_rot, batch, plan->Nc, heads, head_dim, 0, dtype, rope,
-                      stream);
+  // R(norm_k(cond_k)): the same per-row arithmetic as every rotation in the
+  // library.
+  s = lc_rotate_rows(cond_k, cond_k_rot, batch, plan->Nc, heads, 0, dtype, rope, norm.k_w,
+                     norm.eps, static_cast<cudaStream_t>(stream));
   if (s != LC_OK || !cond_out) return s;
   return run_forward(cond_q, nullptr, nullptr, cond_k_rot, cond_v, cond_out, cond_lse, batch,
-                     heads, head_dim, dtype, softmax_scale, plan, rope, stream, LC_FWD_COND, true);
+                     heads, head_dim, dtype, softmax_scale, plan, rope, stream, LC_FWD_COND, true,
+                     norm);
 }
 
 extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const void *v,
@@ -194,9 +234,10 @@ extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const 
     return lc_launch_forward_f32(static_cast<const float *>(q), static_cast<const float *>(k),
                                  static_cast<const float *>(v), nullptr, nullptr,
                                  static_cast<float *>(out), lse, batch, heads, scale, LC_FWD_FULL,
-                                 false, plan, rope, scratch + 1, st);
+                                 false, lc_qk_norm(), plan, rope, scratch + 1, st);
   return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale,
-                                 LC_FWD_FULL, false, plan, rope, scratch + 1, st, scratch);
+                                 LC_FWD_FULL, false, lc_qk_norm(), plan, rope, scratch + 1, st,
+                                 scratch);
 }
 
 extern "C" lc_status lc_last_device_status(void *stream) {

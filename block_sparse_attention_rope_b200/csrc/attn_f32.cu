@@ -24,10 +24,20 @@ struct F32Args {
   int split_kv;    // condition K/V in cond_k / cond_v, noisy K/V in k / v
   int q_mode;      // rows of q / out: 0 all tokens, 1 noisy tokens, 2 condition tokens
   int cond_k_rot;  // cond_k already holds R(k)
+  const float *q_nw, *k_nw;  // RMSNorm weights [64] ahead of the rotation, or NULL
+  float norm_eps;
   float scale;
 };
 
-__device__ __forceinline__ void rope_row(float *x, int n, const F32Args &a) {
+__device__ __forceinline__ void rope_row(float *x, int n, const F32Args &a, const float *nw) {
+  if (nw) {  // RMSNorm first, summed in the library's fixed order
+    float c8[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) c8[ch] = lc_sumsq8(x + 8 * ch);
+    const float inv = lc_rms_inv(lc_sumsq_tree8(c8), a.norm_eps);
+#pragma unroll
+    for (int d = 0; d < LC_HEAD_DIM; ++d) x[d] = lc_rms_apply(x[d], inv, __ldg(nw + d));
+  }
   int t = lc_div(n, a.div_hw);
   int rem = n - t * a.div_hw.d;
   int h = lc_div(rem, a.div_w);
@@ -77,7 +87,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
     const float *src = a.q + (((long long)b * Nq + q_row) * a.heads + h) * LC_HEAD_DIM;
 #pragma unroll
     for (int d = 0; d < LC_HEAD_DIM; ++d) q[d] = src[d];
-    rope_row(q, n, a);
+    rope_row(q, n, a, a.q_nw);
   } else {
 #pragma unroll
     for (int d = 0; d < LC_HEAD_DIM; ++d) q[d] = 0.f;
@@ -103,7 +113,7 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
       const float *vs = kv_row(a.v, a.cond_v, b, m, h, a);
 #pragma unroll
       for (int d = 0; d < LC_HEAD_DIM; ++d) kr[d] = ks[d];
-      if (!(a.cond_k_rot && m < a.Nc)) rope_row(kr, m, a);
+      if (!(a.cond_k_rot && m < a.Nc)) rope_row(kr, m, a, a.k_nw);
 #pragma unroll
       for (int d = 0; d < LC_HEAD_DIM; ++d) {
         sK[tid][d] = kr[d];
@@ -142,9 +152,9 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
 lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 const float *cond_k, const float *cond_v, float *out, float *lse,
                                 int batch, int heads, float scale, lc_fwd_mode mode,
-                                bool cond_k_rotated, const lc_bsa_plan_s *plan,
-                                const lc_rope3d_s *rope, int * /*dev_status*/,
-                                cudaStream_t stream) {
+                                bool cond_k_rotated, const lc_qk_norm &norm,
+                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                int * /*dev_status*/, cudaStream_t stream) {
   F32Args a;
   a.q = q; a.k = k; a.v = v; a.cond_k = cond_k; a.cond_v = cond_v;
   a.out = out; a.lse = lse;
@@ -159,6 +169,9 @@ lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
   a.cond_k_rot = (mode != LC_FWD_FULL && cond_k_rotated) ? 1 : 0;
   a.q_block0 = mode == LC_FWD_CACHED ? plan->Cb : 0;
   a.scale = scale;
+  a.q_nw = norm.q_w;
+  a.k_nw = norm.k_w;
+  a.norm_eps = norm.eps;
   int nrows = mode == LC_FWD_CACHED ? plan->Nb : (mode == LC_FWD_COND ? plan->Cb : plan->nq);
   if (nrows == 0) return LC_OK;
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));

@@ -108,6 +108,9 @@ struct __align__(64) Sm100Params {
   int tab_floats;
   int k_prerotated;        // K tensors already hold R(k): skip the K rotation
   float scale_log2;
+  const float *q_norm_w;   // RMSNorm weights [64] applied ahead of the rotation, or NULL
+  const float *k_norm_w;
+  float norm_eps;
 };
 
 // Shared memory carve-up (offsets from a 1024-aligned base).
@@ -118,7 +121,8 @@ struct SmemOffsets {
   static constexpr int bars = v + kStages * kTileBytes;        // mbarriers
   static constexpr int n_bars = 64;
   static constexpr int misc = bars + n_bars * 8;               // tmem base, items, abort
-  static constexpr int tab = misc + 64;                        // rope tables (fp32)
+  static constexpr int normw = misc + 64;                      // q, k RMSNorm weights (fp32)
+  static constexpr int tab = normw + 2 * 64 * 4;               // rope tables (fp32)
 };
 
 // Barrier indices.
@@ -249,9 +253,43 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// Rotate one token row (64 bf16 channels, 128-byte swizzled) in place.
+// One 16-byte chunk (8 bf16 channels, packed pairs in wds) of a token row:
+// optional RMSNorm (inv = 1/rms of the row, w8 = the chunk's 8 weights), then
+// the rotation of its 4 channel pairs, rounded back to bf16.
+__device__ __forceinline__ void rot_chunk_bf16(uint32_t (&wds)[4], const float4 cc,
+                                               const float4 ss, bool norm, float inv,
+                                               const float (&w8)[8]) {
+  const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float a = __uint_as_float(wds[q] << 16);
+    float b = __uint_as_float(wds[q] & 0xFFFF0000u);
+    if (norm) {
+      a = lc_rms_apply(a, inv, w8[2 * q]);
+      b = lc_rms_apply(b, inv, w8[2 * q + 1]);
+    }
+    float xr, yr;
+    lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
+    __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
+    wds[q] = *reinterpret_cast<uint32_t *>(&o2);
+  }
+}
+
+// Sum of squares of the 8 bf16 channels of a chunk.
+__device__ __forceinline__ float sumsq_chunk_bf16(const uint32_t (&wds)[4]) {
+  float v[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[2 * q] = __uint_as_float(wds[q] << 16);
+    v[2 * q + 1] = __uint_as_float(wds[q] & 0xFFFF0000u);
+  }
+  return lc_sumsq8(v);
+}
+
+// Rotate one token row (64 bf16 channels, 128-byte swizzled) in place, after
+// an RMSNorm with the 64 weights nw when nw is not NULL.
 __device__ __forceinline__ void rope_row(uint8_t *tile, int r, int n, const float *tab,
-                                         const Sm100Params &p) {
+                                         const Sm100Params &p, const float *nw) {
   const int t = lc_div(n, p.div_hw);
   const int rem = n - t * p.div_hw.d;
   const int hh = lc_div(rem, p.div_w);
@@ -261,25 +299,29 @@ __device__ __forceinline__ void rope_row(uint8_t *tile, int r, int n, const floa
   const float *cW = tab + p.T * 16 + p.H * 24 + w * 12, *sW = cW + p.W * 12;
   uint8_t *rowp = tile + r * 128;
   const int x = r & 7;
+  float inv = 1.f;
+  if (nw) {
+    float c8[8];
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ x) << 4));
+      const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
+      c8[ch] = sumsq_chunk_bf16(wds);
+    }
+    inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
+  }
 #pragma unroll
   for (int ch = 0; ch < 8; ++ch) {
     const float *c = ch < 2 ? cT + 4 * ch : (ch < 5 ? cH + 4 * (ch - 2) : cW + 4 * (ch - 5));
     const float *s = ch < 2 ? sT + 4 * ch : (ch < 5 ? sH + 4 * (ch - 2) : sW + 4 * (ch - 5));
-    const float4 cc = *reinterpret_cast<const float4 *>(c);
-    const float4 ss = *reinterpret_cast<const float4 *>(s);
     uint4 *ptr = reinterpret_cast<uint4 *>(rowp + ((ch ^ x) << 4));
-    uint4 raw = *ptr;
+    const uint4 raw = *ptr;
     uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-    const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
+    float w8[8];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = __uint_as_float(wds[q] << 16);
-      const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
-      float xr, yr;
-      lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
-      __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
-      wds[q] = *reinterpret_cast<uint32_t *>(&o2);
-    }
+    for (int e = 0; e < 8; ++e) w8[e] = nw ? nw[8 * ch + e] : 1.f;
+    rot_chunk_bf16(wds, *reinterpret_cast<const float4 *>(c), *reinterpret_cast<const float4 *>(s),
+                   nw != nullptr, inv, w8);
     *ptr = make_uint4(wds[0], wds[1], wds[2], wds[3]);
   }
 }
@@ -385,6 +427,9 @@ __device__ __forceinline__ uint32_t tile_limits(const Sm100Params &p, const Item
   return (uint32_t)na | ((uint32_t)nb << 8);
 }
 
+// kQKNorm: the RoPE warps apply the RMSNorm weights of p (instantiated
+// separately so that the plain path carries no trace of it).
+template <bool kQKNorm>
 __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_constant__ Sm100Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -397,6 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SmemOffsets::misc);
   // misc[0] tmem base, misc[1..2] scheduled items, misc[3] abort flag
   float *tab = reinterpret_cast<float *>(smem + SmemOffsets::tab);
+  float *s_normw = reinterpret_cast<float *>(smem + SmemOffsets::normw);  // [q 64 | k 64]
   Ctx ctx;
   ctx.bar0 = lcptx::smem_addr(smem + SmemOffsets::bars);
   ctx.abort_flag = reinterpret_cast<volatile int *>(&misc[3]);
@@ -405,6 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
 
   // ---- set-up: tables, barriers, TMEM
   for (int i = tid; i < p.tab_floats; i += kThreads) tab[i] = p.rope_tab[i];
+  if (tid < 64 && p.q_norm_w) s_normw[tid] = p.q_norm_w[tid];
+  if (tid < 64 && p.k_norm_w) s_normw[64 + tid] = p.k_norm_w[tid];
   if (tid == 0) {
     misc[3] = 0;
     for (int i = 0; i < 4; ++i) {
@@ -638,6 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   } else {
     // ======================= RoPE warps ======================================
     const int rt = tid - kWarpRope * 32;
+    const float *q_nw = (kQKNorm && p.q_norm_w) ? s_normw : nullptr;
+    const float *k_nw = (kQKNorm && p.k_norm_w) ? s_normw + 64 : nullptr;
     uint32_t item_it = 0, kv_it = 0;
     EntryStream es;
     for (;;) {
@@ -660,7 +710,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         const int nrows = min(128, it.seg_len - r0);
 #pragma unroll 1
         for (int r = rt; r < nrows; r += kRopeThreads)
-          rope_row(sQ + qi * kTileBytes, r, seg_base + r0 + r, tab, p);
+          rope_row(sQ + qi * kTileBytes, r, seg_base + r0 + r, tab, p, q_nw);
         lcptx::fence_proxy_async_smem();
         lcptx::mbar_arrive(ctx.bar(B_QREADY + qi));
       }
@@ -681,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
             if (half == 1 && 2 * t + 1 >= it.len) break;
             int sx, rx, nx;
             entry_block(p, half ? eb : ea, sx, rx, nx);
-            if (rt < nx) rope_row(tile, 64 * half + rt, (sx ? p.Nc : 0) + rx + rt, tab, p);
+            if (rt < nx) rope_row(tile, 64 * half + rt, (sx ? p.Nc : 0) + rx + rt, tab, p, k_nw);
           }
           lcptx::fence_proxy_async_smem();
           lcptx::mbar_arrive(ctx.bar(B_KREADY + s));
@@ -982,10 +1032,13 @@ __global__ void watchdog_selftest_kernel(int *status, long long timeout_ns) {
 
 // Standalone rotation of K (or any [B, ntok, heads, 64] bf16 tensor) into a
 // separate buffer, 16 bytes per thread step; used when the attention kernel
-// is given K already rotated.  Same arithmetic as rope_row.
+// is given K already rotated.  Same arithmetic as rope_row: with nw, the
+// eight lanes that hold a row's chunks combine their sums of squares.
 __global__ void rope_k_kernel(const uint4 *src, uint4 *dst, long long n_chunks, int heads,
                               long long ntok, int tok_offset, const float *tab, int T, int H,
-                              int W, lc_divmod div_hw, lc_divmod div_w) {
+                              int W, lc_divmod div_hw, lc_divmod div_w, const float *nw,
+                              float eps) {
+  const unsigned group = 0xFFu << (threadIdx.x & 24);  // this lane's 8-lane group
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_chunks;
        i += (long long)gridDim.x * blockDim.x) {
     const int ch = (int)(i & 7);
@@ -999,26 +1052,23 @@ __global__ void rope_k_kernel(const uint4 *src, uint4 *dst, long long n_chunks, 
     if (ch < 2) { c = tab + t * 8 + 4 * ch; s = c + T * 8; }
     else if (ch < 5) { c = tab + T * 16 + hh * 12 + 4 * (ch - 2); s = c + H * 12; }
     else { c = tab + T * 16 + H * 24 + w * 12 + 4 * (ch - 5); s = c + W * 12; }
-    const float4 cc = __ldg(reinterpret_cast<const float4 *>(c));
-    const float4 ss = __ldg(reinterpret_cast<const float4 *>(s));
     const uint4 raw = __ldg(src + i);
     uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-    const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
+    float inv = 1.f, w8[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+    if (nw) {  // uniform: every lane of a group is in the loop together
+      inv = lc_rms_inv(lc_sumsq_lanes8(sumsq_chunk_bf16(wds), group), eps);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float a = __uint_as_float(wds[q] << 16);
-      const float b = __uint_as_float(wds[q] & 0xFFFF0000u);
-      float xr, yr;
-      lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
-      __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
-      wds[q] = *reinterpret_cast<uint32_t *>(&o2);
+      for (int e = 0; e < 8; ++e) w8[e] = __ldg(nw + 8 * ch + e);
     }
+    rot_chunk_bf16(wds, __ldg(reinterpret_cast<const float4 *>(c)),
+                   __ldg(reinterpret_cast<const float4 *>(s)), nw != nullptr, inv, w8);
     dst[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
   }
 }
 
 lc_status launch_rope_k(const void *src, void *dst, int batch, long long ntok, int heads,
-                        int tok_offset, const lc_rope3d_s *rope, cudaStream_t stream) {
+                        int tok_offset, const lc_rope3d_s *rope, cudaStream_t stream,
+                        const float *nw, float eps) {
   const long long n_chunks = (long long)batch * ntok * heads * (LC_HEAD_DIM / 8);
   int dev = 0, n_sm = 148;
   cudaGetDevice(&dev);
@@ -1029,7 +1079,7 @@ lc_status launch_rope_k(const void *src, void *dst, int batch, long long ntok, i
                                           static_cast<uint4 *>(dst), n_chunks, heads, ntok,
                                           tok_offset, rope->tab, rope->T, rope->H, rope->W,
                                           lc_make_divmod(rope->H * rope->W),
-                                          lc_make_divmod(rope->W));
+                                          lc_make_divmod(rope->W), nw, eps);
   return lc_from_cuda(cudaGetLastError());
 }
 
@@ -1073,8 +1123,9 @@ int *lc_noalloc_scratch(lc_status *st) {
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, const void *cond_k,
                                   const void *cond_v, void *out, float *lse, int batch, int heads,
                                   float scale, lc_fwd_mode mode, bool cond_k_rotated,
-                                  const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                  int *dev_status, cudaStream_t stream, int *counter_scratch) {
+                                  const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
+                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
+                                  int *counter_scratch) {
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
   const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
@@ -1146,6 +1197,9 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.gc = plan->gc;
   prm.heads = heads;
   prm.k_prerotated = 0;
+  prm.q_norm_w = norm.q_w;
+  prm.k_norm_w = norm.k_w;
+  prm.norm_eps = norm.eps;
   long long total = (long long)batch * heads * prm.n_groups_active;
   if (total == 0) return LC_OK;
   if (total >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
@@ -1158,15 +1212,18 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   // The kernel's setmaxnreg split needs at least kRegsAtLaunchMin registers
   // per thread at launch; with fewer, raising the softmax warps' count could
   // never complete, so such a build is refused instead of launched.
-  static int regs_at_launch = -1;
-  if (regs_at_launch < 0) {
+  const bool with_norm = prm.q_norm_w || prm.k_norm_w;
+  void (*const kern)(const Sm100Params) = with_norm ? bsa_sm100_kernel<true>
+                                                    : bsa_sm100_kernel<false>;
+  static int regs_at_launch[2] = {-1, -1};
+  int &regs = regs_at_launch[with_norm ? 1 : 0];
+  if (regs < 0) {
     cudaFuncAttributes fa;
-    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, bsa_sm100_kernel));
-    regs_at_launch = fa.numRegs;
+    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+    regs = fa.numRegs;
   }
-  if (regs_at_launch < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;
-  LC_CUDA_TRY(cudaFuncSetAttribute(bsa_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)smem));
+  if (regs < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;
+  LC_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   int dev = 0, n_sm = 0;
   LC_CUDA_TRY(cudaGetDevice(&dev));
   LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
@@ -1178,7 +1235,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, rope->ready, 0);
     if (e == cudaSuccess) {
-      bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+      kern<<<grid, kThreads, smem, stream>>>(prm);
       e = cudaGetLastError();
     }
     return lc_from_cuda(e);
@@ -1200,13 +1257,14 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
       e = cudaMallocFromPoolAsync(&k_rot, kb, pool, stream);
       if (e == cudaSuccess)
         s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
-                          stream);
+                          stream, norm.k_w, norm.eps);
     }
     // Separately supplied condition K, unless the caller rotated it already.
     if (e == cudaSuccess && s == LC_OK && (cached || cond_only) && Nc > 0 && !cond_k_rotated) {
       e = cudaMallocFromPoolAsync(&ck_rot, (size_t)batch * Nc * heads * LC_HEAD_DIM * 2, pool,
                                   stream);
-      if (e == cudaSuccess) s = launch_rope_k(cond_k, ck_rot, batch, Nc, heads, 0, rope, stream);
+      if (e == cudaSuccess)
+        s = launch_rope_k(cond_k, ck_rot, batch, Nc, heads, 0, rope, stream, norm.k_w, norm.eps);
     }
     if (e == cudaSuccess && s == LC_OK) {
       if (ck_rot) s = encode_segment(&prm.tmK[0], ck_rot, batch, Nc, 0, Nc, heads);
@@ -1229,7 +1287,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     prm.work_counter = counter;
     e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
     if (e == cudaSuccess) {
-      bsa_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+      kern<<<grid, kThreads, smem, stream>>>(prm);
       e = cudaGetLastError();
     }
   }

@@ -101,6 +101,36 @@ __device__ __forceinline__ void lc_rot_pair(float a, float b, float c, float s, 
   y = __fmaf_rn(a, s, __fmul_rn(b, c));
 }
 
+// RMSNorm of one 64-channel row (one token, one head) ahead of the rotation
+// (myzaker / QbitAI "背后技术原理": RMSNorm in the attention modules):
+// y = x / sqrt(mean(x^2) + eps) * w.  The mean square is summed in a fixed
+// order -- each 8-channel chunk sequentially, then the eight chunk sums as
+// ((c0+c1)+(c2+c3))+((c4+c5)+(c6+c7)) -- so that a thread holding the whole
+// row and eight lanes holding one chunk each (combined by xor-shuffles over
+// 1, 2, 4, which form the same sums) get the same bits.
+__device__ __forceinline__ float lc_sumsq8(const float *x) {
+  float a = __fmul_rn(x[0], x[0]);
+#pragma unroll
+  for (int i = 1; i < 8; ++i) a = __fmaf_rn(x[i], x[i], a);
+  return a;
+}
+__device__ __forceinline__ float lc_sumsq_tree8(const float *c) {
+  return __fadd_rn(__fadd_rn(__fadd_rn(c[0], c[1]), __fadd_rn(c[2], c[3])),
+                   __fadd_rn(__fadd_rn(c[4], c[5]), __fadd_rn(c[6], c[7])));
+}
+// Eight consecutive lanes (mask: their bits) each hold one chunk sum.
+__device__ __forceinline__ float lc_sumsq_lanes8(float c, unsigned mask) {
+  c = __fadd_rn(c, __shfl_xor_sync(mask, c, 1));
+  c = __fadd_rn(c, __shfl_xor_sync(mask, c, 2));
+  return __fadd_rn(c, __shfl_xor_sync(mask, c, 4));
+}
+__device__ __forceinline__ float lc_rms_inv(float sumsq, float eps) {
+  return rsqrtf(__fmaf_rn(sumsq, 0.015625f, eps));  // mean = sum / 64
+}
+__device__ __forceinline__ float lc_rms_apply(float x, float inv, float w) {
+  return __fmul_rn(__fmul_rn(x, inv), w);
+}
+
 // Launch helpers implemented by the kernel translation units.
 // Which queries an attention launch computes and where its tensors live.
 //   LC_FWD_FULL    q, k, v, out hold all N tokens (cond_k / cond_v unused).
@@ -111,20 +141,36 @@ __device__ __forceinline__ void lc_rot_pair(float a, float b, float c, float s, 
 // cond_k_rotated: cond_k already holds R(k) (CACHED and COND only).
 enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2 };
 
+// RMSNorm of q and k ahead of the rotation: device fp32 weights [64] or NULL.
+struct lc_qk_norm {
+  const float *q_w = nullptr;
+  const float *k_w = nullptr;
+  float eps = 0.f;
+};
+
 lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 const float *cond_k, const float *cond_v, float *out,
                                 float *lse, int batch, int heads, float scale, lc_fwd_mode mode,
-                                bool cond_k_rotated, const lc_bsa_plan_s *plan,
-                                const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream);
+                                bool cond_k_rotated, const lc_qk_norm &norm,
+                                const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                int *dev_status, cudaStream_t stream);
 // counter_scratch: NULL = allocate the scheduler counter stream-ordered for
 // this launch; else a device int the caller provides (lc_bsa_forward_noalloc,
 // LC_FWD_FULL only).
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
                                   const void *cond_k, const void *cond_v, void *out,
                                   float *lse, int batch, int heads, float scale, lc_fwd_mode mode,
-                                  bool cond_k_rotated, const lc_bsa_plan_s *plan,
-                                  const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
+                                  bool cond_k_rotated, const lc_qk_norm &norm,
+                                  const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
+                                  int *dev_status, cudaStream_t stream,
                                   int *counter_scratch = nullptr);
+// Rotate x [batch, ntok, heads, 64] of dtype (token n of x = sequence token
+// n + tok_offset) into out, after an RMSNorm with norm_w when not NULL
+// (rope.cu; the public lc_rope3d_apply is this without the norm).  Arguments
+// are checked by the caller.
+lc_status lc_rotate_rows(const void *x, void *out, int batch, long long ntok, int heads,
+                         long long tok_offset, lc_dtype dtype, const lc_rope3d_s *rope,
+                         const float *norm_w, float eps, cudaStream_t stream);
 
 // Fixed scratch of lc_bsa_forward_noalloc (attn_sm100.cu): device address of
 // g_lc_noalloc_scratch on the current device, looked up once per device.

@@ -62,7 +62,9 @@ __device__ __forceinline__ void rotate_chunk(float (&x)[8], int ch, int t, int h
 template <typename Tin>
 __global__ void rope_apply_kernel(const Tin *x, Tin *out, long long n_chunks, int heads,
                                   long long ntok, long long tok_offset, const float *tab, int T,
-                                  int H, int W, lc_divmod div_hw, lc_divmod div_w) {
+                                  int H, int W, lc_divmod div_hw, lc_divmod div_w,
+                                  const float *nw, float eps) {
+  const unsigned group = 0xFFu << (threadIdx.x & 24);  // the 8 lanes holding one row
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n_chunks;
        i += (long long)gridDim.x * blockDim.x) {
     int ch = (int)(i & 7);
@@ -77,6 +79,11 @@ __global__ void rope_apply_kernel(const Tin *x, Tin *out, long long n_chunks, in
     const Tin *src = x + i * 8;
 #pragma unroll
     for (int e = 0; e < 8; ++e) v[e] = (float)src[e];
+    if (nw) {  // uniform: every lane of a group is in the loop together
+      const float inv = lc_rms_inv(lc_sumsq_lanes8(lc_sumsq8(v), group), eps);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = lc_rms_apply(v[e], inv, __ldg(nw + 8 * ch + e));
+    }
     rotate_chunk(v, ch, t, h, w, tab, T, H, W);
     Tin *dst = out + i * 8;
 #pragma unroll
@@ -137,6 +144,29 @@ extern "C" lc_status lc_rope3d_copy_tables(lc_rope3d rope, float *host, void *st
   return LC_OK;
 }
 
+lc_status lc_rotate_rows(const void *x, void *out, int batch, long long ntok, int heads,
+                         long long tok_offset, lc_dtype dtype, const lc_rope3d_s *rope,
+                         const float *norm_w, float eps, cudaStream_t st) {
+  long long n_chunks = (long long)batch * ntok * heads * (LC_HEAD_DIM / 8);
+  if (n_chunks == 0) return LC_OK;
+  int tpb = 256;
+  long long want = (n_chunks + tpb - 1) / tpb;
+  int nb = (int)(want < 148LL * 16 ? want : 148LL * 16);
+  lc_divmod dhw = lc_make_divmod(rope->H * rope->W), dw = lc_make_divmod(rope->W);
+  LC_CUDA_TRY(cudaStreamWaitEvent(st, rope->ready, 0));
+  if (dtype == LC_DTYPE_F32)
+    rope_apply_kernel<float><<<nb, tpb, 0, st>>>(static_cast<const float *>(x),
+                                                 static_cast<float *>(out), n_chunks, heads, ntok,
+                                                 tok_offset, rope->tab, rope->T, rope->H, rope->W,
+                                                 dhw, dw, norm_w, eps);
+  else
+    rope_apply_kernel<__nv_bfloat16><<<nb, tpb, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(out), n_chunks,
+        heads, ntok, tok_offset, rope->tab, rope->T, rope->H, rope->W, dhw, dw, norm_w, eps);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}
+
 extern "C" lc_status lc_rope3d_apply(const void *x, void *out, int batch, long long ntok, int heads,
                                      int head_dim, long long tok_offset, lc_dtype dtype,
                                      lc_rope3d rope, void *stream) {
@@ -150,22 +180,6 @@ extern "C" lc_status lc_rope3d_apply(const void *x, void *out, int batch, long l
   int dev = -1;
   LC_CUDA_TRY(cudaGetDevice(&dev));
   if (dev != rope->device) return LC_ERR_INVALID_ARGUMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  long long n_chunks = (long long)batch * ntok * heads * (LC_HEAD_DIM / 8);
-  int tpb = 256;
-  long long want = (n_chunks + tpb - 1) / tpb;
-  int nb = (int)(want < 148LL * 16 ? want : 148LL * 16);
-  lc_divmod dhw = lc_make_divmod(rope->H * rope->W), dw = lc_make_divmod(rope->W);
-  LC_CUDA_TRY(cudaStreamWaitEvent(st, rope->ready, 0));
-  if (dtype == LC_DTYPE_F32)
-    rope_apply_kernel<float><<<nb, tpb, 0, st>>>(static_cast<const float *>(x),
-                                                 static_cast<float *>(out), n_chunks, heads, ntok,
-                                                 tok_offset, rope->tab, rope->T, rope->H, rope->W,
-                                                 dhw, dw);
-  else
-    rope_apply_kernel<__nv_bfloat16><<<nb, tpb, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(out), n_chunks,
-        heads, ntok, tok_offset, rope->tab, rope->T, rope->H, rope->W, dhw, dw);
-  LC_CUDA_TRY(cudaGetLastError());
-  return LC_OK;
+  return lc_rotate_rows(x, out, batch, ntok, heads, tok_offset, dtype, rope, nullptr, 0.f,
+                        static_cast<cudaStream_t>(stream));
 }

@@ -176,21 +176,49 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
                                 lc_dtype dtype, float softmax_scale, lc_bsa_plan plan,
                                 lc_rope3d rope, void *stream);
 
-/* Flags of lc_bsa_forward_cached_ex. */
+/* Flags of lc_bsa_opts. */
 #define LC_FLAG_COND_K_ROTATED 1u  /* cond_k already holds R(k) (lc_bsa_cond_cache) */
 
 /*
- * lc_bsa_forward_cached_ex -- lc_bsa_forward_cached with flags.  With
- * LC_FLAG_COND_K_ROTATED, cond_k is taken as already rotated (the cond_k_rot
- * output of lc_bsa_cond_cache) and is not rotated again, so a cache built once
- * serves every later call.  The results equal lc_bsa_forward_cached's on the
- * pre-RoPE cond_k bit for bit.  Unknown flag bits: LC_ERR_INVALID_ARGUMENT;
- * other errors as lc_bsa_forward.
+ * Options of the _ex entry points and of lc_bsa_cond_cache.  A NULL options
+ * pointer, or a zero-initialised struct, means none.
+ *   flags:          LC_FLAG_COND_K_ROTATED (lc_bsa_forward_cached_ex only).
+ *   q_norm_weight,  device fp32 [head_dim]: RMSNorm of q (resp. k and cond_k)
+ *   k_norm_weight:  ahead of the 3D-RoPE, x / sqrt(mean(x^2) + norm_eps) * w
+ *                   per token and head over the head's channels (myzaker /
+ *                   QbitAI "背后技术原理": RMSNorm in the attention modules).
+ *                   NULL: no norm.  4-byte aligned.
+ *   norm_eps:       >= 0 and finite; used only with a weight.
+ * The norm is fused into the same per-row rotation every entry point applies
+ * (in the tile loads, the one-pass K rotation and the fp32 kernel).
+ */
+typedef struct {
+    unsigned flags;
+    const float *q_norm_weight;
+    const float *k_norm_weight;
+    float norm_eps;
+} lc_bsa_opts;
+
+/* lc_bsa_forward with options (RMSNorm of q and k).  Flags must be 0.
+ * Errors as lc_bsa_forward, plus LC_ERR_INVALID_ARGUMENT for bad options. */
+lc_status lc_bsa_forward_ex(const void *q, const void *k, const void *v, void *out, float *lse,
+                            int batch, int heads, int head_dim, lc_dtype dtype,
+                            float softmax_scale, const lc_bsa_opts *opts, lc_bsa_plan plan,
+                            lc_rope3d rope, void *stream);
+
+/*
+ * lc_bsa_forward_cached_ex -- lc_bsa_forward_cached with options.  With
+ * LC_FLAG_COND_K_ROTATED, cond_k is taken as already normalised and rotated
+ * (the cond_k_rot output of lc_bsa_cond_cache with the same k_norm_weight) and
+ * is used as is, so a cache built once serves every later call; the results
+ * equal those of the same call on the raw cond_k bit for bit.  Unknown flag
+ * bits or bad options: LC_ERR_INVALID_ARGUMENT; other errors as
+ * lc_bsa_forward.
  */
 lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
                                    const void *cond_k, const void *cond_v, void *out,
                                    float *lse, int batch, int heads, int head_dim,
-                                   lc_dtype dtype, float softmax_scale, unsigned flags,
+                                   lc_dtype dtype, float softmax_scale, const lc_bsa_opts *opts,
                                    lc_bsa_plan plan, lc_rope3d rope, void *stream);
 
 /*
@@ -204,7 +232,9 @@ lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
  * LC_FLAG_COND_K_ROTATED.  If cond_out is not NULL it also computes the
  * condition tokens' attention (condition queries over condition keys, the
  * condition rows of lc_bsa_forward on the whole sequence) into cond_out and,
- * if cond_lse is not NULL, their lse.
+ * if cond_lse is not NULL, their lse.  opts (nullable, flags 0) carries the
+ * RMSNorm weights: cond_k_rot then holds R(norm_k(cond_k)) and cond_q is
+ * normalised with q_norm_weight, as in lc_bsa_forward_ex.
  *   cond_q, cond_k, cond_v, cond_k_rot, cond_out: [batch, Nc, heads, head_dim]
  *   of dtype, 16-byte aligned; cond_lse: [batch, heads, Nc] fp32.  cond_q and
  *   cond_v are read only when cond_out is given (else they may be NULL).
@@ -215,7 +245,8 @@ lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, const void *v,
 lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *cond_v,
                             void *cond_k_rot, void *cond_out, float *cond_lse, int batch,
                             int heads, int head_dim, lc_dtype dtype, float softmax_scale,
-                            lc_bsa_plan plan, lc_rope3d rope, void *stream);
+                            const lc_bsa_opts *opts, lc_bsa_plan plan, lc_rope3d rope,
+                            void *stream);
 
 /*
  * lc_bsa_forward_noalloc -- lc_bsa_forward for callers that cannot allocate

@@ -122,22 +122,27 @@ def test_cond_cache_errors(api):
     lib, INV = api.lib, 1
     # cond_k_rot overlapping cond_k
     assert lib.lc_bsa_cond_cache(None, big.data_ptr(), None, big[:, 1:].data_ptr(), None, None,
-                                 1, w.heads, 64, 0, 0.0, plan.handle, rope.handle, None) == INV
+                                 1, w.heads, 64, 0, 0.0, None, plan.handle, rope.handle,
+                                 None) == INV
     # lse without an output, output without q/v
     lse = torch.zeros(1, w.heads, Nc, device="cuda")
     k_rot = torch.empty_like(t)
     assert lib.lc_bsa_cond_cache(None, t.data_ptr(), None, k_rot.data_ptr(), None,
-                                 lse.data_ptr(), 1, w.heads, 64, 0, 0.0, plan.handle,
+                                 lse.data_ptr(), 1, w.heads, 64, 0, 0.0, None, plan.handle,
                                  rope.handle, None) == INV
     assert lib.lc_bsa_cond_cache(None, t.data_ptr(), t.data_ptr(), k_rot.data_ptr(),
                                  torch.empty_like(t).data_ptr(), None, 1, w.heads, 64, 0, 0.0,
-                                 plan.handle, rope.handle, None) == INV
+                                 None, plan.handle, rope.handle, None) == INV
     # unknown flag bits
     n = torch.zeros(1, w.n_noisy_tokens, w.heads, 64, dtype=torch.bfloat16, device="cuda")
     assert lib.lc_bsa_forward_cached_ex(n.data_ptr(), n.data_ptr(), n.data_ptr(), t.data_ptr(),
                                         t.data_ptr(), torch.empty_like(n).data_ptr(), None, 1,
-                                        w.heads, 64, 0, 0.0, ctypes.c_uint(6), plan.handle,
-                                        rope.handle, None) == INV
+                                        w.heads, 64, 0, 0.0, ctypes.byref(api.Opts(6)),
+                                        plan.handle, rope.handle, None) == INV
+    # cond_cache takes no flags
+    assert lib.lc_bsa_cond_cache(None, t.data_ptr(), None, k_rot.data_ptr(), None, None, 1,
+                                 w.heads, 64, 0, 0.0, ctypes.byref(api.Opts(1)), plan.handle,
+                                 rope.handle, None) == INV
     with pytest.raises(ValueError):
         api.cond_cache(t, plan, rope, cond_q=t)  # cond_v missing
 

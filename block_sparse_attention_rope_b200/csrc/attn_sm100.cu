@@ -49,6 +49,13 @@ namespace {
 #define LC_KV_STAGES 3
 #endif
 constexpr int kStages = LC_KV_STAGES;
+// 1: a K/V ring stage has one "full" barrier (K and V bytes together) and one
+// "empty" barrier (released after the stage's last P*V), which saves the MMA
+// issuer a wait and a commit per tile; 0: separate K and V barriers.
+#ifndef LC_KV_MERGED
+#define LC_KV_MERGED 1
+#endif
+constexpr bool kKVMerged = LC_KV_MERGED != 0;
 constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
 constexpr int kWarpMma = 9;
@@ -551,21 +558,23 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           ok = wait_bar(ctx, ctx.bar(B_KEMPTY + s), ph ^ 1);
           if (!ok) break;
           const uint32_t bk = ctx.bar(B_KFULL + s);
-          lcptx::mbar_arrive_expect_tx(bk, kTileBytes);
+          lcptx::mbar_arrive_expect_tx(bk, kKVMerged ? 2 * kTileBytes : kTileBytes);
           const uint32_t dk = lcptx::smem_addr(sK + s * kTileBytes);
           lcptx::tma_load_4d(dk, &p.tmK[sa], bk, 0, it.h, ra, it.b);
           lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[sb], bk, 0, it.h, rb, it.b);
           k_valid |= 1u << s;
           k_par = (k_par & ~(1u << s)) | (ph << s);
-          ok = wait_bar(ctx, ctx.bar(B_VEMPTY + s), ph ^ 1);
+          if (!kKVMerged) ok = wait_bar(ctx, ctx.bar(B_VEMPTY + s), ph ^ 1);
           if (!ok) break;
-          const uint32_t bv = ctx.bar(B_VFULL + s);
-          lcptx::mbar_arrive_expect_tx(bv, kTileBytes);
+          const uint32_t bv = ctx.bar(kKVMerged ? B_KFULL + s : B_VFULL + s);
+          if (!kKVMerged) lcptx::mbar_arrive_expect_tx(bv, kTileBytes);
           const uint32_t dv = lcptx::smem_addr(sV + s * kTileBytes);
           lcptx::tma_load_4d(dv, &p.tmV[sa], bv, 0, it.h, ra, it.b);
           lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[sb], bv, 0, it.h, rb, it.b);
-          v_valid |= 1u << s;
-          v_par = (v_par & ~(1u << s)) | (ph << s);
+          if (!kKVMerged) {
+            v_valid |= 1u << s;
+            v_par = (v_par & ~(1u << s)) | (ph << s);
+          }
         }
         if (!ok) break;
         ++item_it;
@@ -650,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         // tile 0: both S tiles
         ok = wait_bar(ctx, ctx.bar(kbar + cs), cph) && issue_s(0, cs) && issue_s(1, cs);
         if (!ok) break;
-        lcptx::mma_commit(ctx.bar(B_KEMPTY + cs));
+        if (!kKVMerged) lcptx::mma_commit(ctx.bar(B_KEMPTY + cs));
         for (int t = 0; t < ntiles && ok; ++t) {
           const bool more = t + 1 < ntiles;
           const int ns = cs + 1 == kStages ? 0 : cs + 1;
@@ -659,16 +668,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
             ok = wait_bar(ctx, ctx.bar(kbar + ns), nph) && issue_s(0, ns);
             if (!ok) break;
           }
-          ok = wait_bar(ctx, ctx.bar(B_VFULL + cs), cph) && issue_pv(0, cs, t > 0);
+          ok = (kKVMerged || wait_bar(ctx, ctx.bar(B_VFULL + cs), cph)) && issue_pv(0, cs, t > 0);
           if (!ok) break;
           if (more) {
             ok = issue_s(1, ns);
             if (!ok) break;
-            lcptx::mma_commit(ctx.bar(B_KEMPTY + ns));
+            if (!kKVMerged) lcptx::mma_commit(ctx.bar(B_KEMPTY + ns));
           }
           ok = issue_pv(1, cs, t > 0);
           if (!ok) break;
-          lcptx::mma_commit(ctx.bar(B_VEMPTY + cs));
+          lcptx::mma_commit(ctx.bar(kKVMerged ? B_KEMPTY + cs : B_VEMPTY + cs));
           cs = ns;
           cph = nph;
         }

@@ -188,6 +188,39 @@ def time_forward(api, torch, w, d, plan, rope, steps, warmup, dist, stream):
     return total, sum(per) / len(per), out
 
 
+def time_backward(api, synthetic, torch, name, steps, warmup, stream):
+    """Device time of the backward pass (lc_bsa_backward) on one workload:
+    the forward's out and lse are produced first, outside the timed region.
+    Algorithmic work 10 * 64 FLOP per attended pair and head (recomputed S,
+    dP, dQ, dK, dV)."""
+    w = synthetic.get(name)
+    x = synthetic.make_inputs(w, device="cuda")
+    g = synthetic.make_dout(w, device="cuda")
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    with torch.cuda.stream(stream):
+        out, lse = api.forward(x["q"], x["k"], x["v"], plan, rope, return_lse=True, stream=stream)
+        for _ in range(warmup):
+            api.backward(x["q"], x["k"], x["v"], out, lse, g, plan, rope, stream=stream)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    with torch.cuda.stream(stream):
+        ev[0].record(stream)
+        for _ in range(steps):
+            api.backward(x["q"], x["k"], x["v"], out, lse, g, plan, rope, stream=stream)
+        ev[1].record(stream)
+    torch.cuda.synchronize()
+    if api.last_device_status() != 0:
+        raise RuntimeError("device status set by the backward pass")
+    ms = ev[0].elapsed_time(ev[1]) / steps
+    pairs = plan.info().attended_token_pairs
+    flops = 10.0 * w.head_dim * w.heads * w.batch * pairs
+    return {"workload": name, "ms_per_layer": round(ms, 3),
+            "attended_tflops": round(flops / (ms * 1e-3) / 1e12, 3),
+            "work": "10*64 FLOP per attended pair and head",
+            "kernels": "bwd_delta, bwd_dq, bwd_dkdv (fp32 SIMT)"}
+
+
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):
     """End to end through the public API: pinned host inputs -> device ->
     forward -> result back to pinned host memory, every step."""
@@ -375,6 +408,9 @@ def run_ours(a):
                     "pct_bf16_peak": round(100.0 * r["flops"] / (r["launch_ms"] * 1e-3) / 1e12 / peak, 2),
                     "attended_pairs_per_head": r["pairs"],
                     "launch_ms_min_median_max": r["spread"]}
+    if not a.no_extra and a.workload == "i2v_480p":
+        extra["backward_i2v_480p"] = time_backward(api, synthetic, torch, "i2v_480p", 2, 1,
+                                                   stream)
     w = main["w"]
     ms = main["total_ms"] / a.steps
     value = world * main["flops"] * a.steps / (main["total_ms"] * 1e-3) / 1e12

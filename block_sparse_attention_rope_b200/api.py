@@ -64,6 +64,9 @@ def _load():
         "lc_bsa_forward_cached_ex": (S, [vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp,
                                          vp]),
         "lc_bsa_cond_cache": (S, [vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp, vp]),
+        "lc_bsa_backward": (S, [vp, vp, vp, vp, vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp,
+                                vp]),
+        "lc_bsa_plan_copy_csc": (S, [vp, vp, vp, vp]),
         "lc_bsa_forward_noalloc": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
@@ -146,6 +149,15 @@ class Plan:
         _check(lib.lc_bsa_plan_copy_csr(self.handle, rp.data_ptr(), ci.data_ptr(), _stream(stream)),
                "lc_bsa_plan_copy_csr")
         return rp, ci[:inf.nnz]
+
+    def csc(self, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        """Transpose of the block CSR: (col_ptr, row_idx), host int32."""
+        inf = self.info()
+        cp = torch.empty(inf.num_q_blocks + 1, dtype=torch.int32)
+        ri = torch.empty(max(inf.nnz, 1), dtype=torch.int32)
+        _check(lib.lc_bsa_plan_copy_csc(self.handle, cp.data_ptr(), ri.data_ptr(), _stream(stream)),
+               "lc_bsa_plan_copy_csc")
+        return cp, ri[:inf.nnz]
 
     @property
     def n_tokens(self) -> int:
@@ -296,6 +308,27 @@ def forward_cached(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cond_k: Op
                                          _dtype_code(q), float(softmax_scale), plan.handle,
                                          rope.handle, _stream(stream)), "lc_bsa_forward_cached")
     return (out, lse) if (return_lse or lse is not None) else out
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, plan: Plan, rope: Rope3D, *,
+             softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
+             k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None):
+    """Gradients (dq, dk, dv) of forward() for dout (lc_bsa_backward); out and
+    lse are the forward's results for the same q, k, v."""
+    B, N, heads, hd = q.shape
+    _check_bmhk("q", q, (B, plan.n_tokens, heads, hd), q.dtype)
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _check_bmhk(name, t, q.shape, q.dtype)
+    _check_bmhk("lse", lse, (B, heads, N), torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    opts = _opts(0, q_norm, k_norm, norm_eps, hd)
+    _check(lib.lc_bsa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                               dv.data_ptr(), B, heads, hd, _dtype_code(q), float(softmax_scale),
+                               None if opts is None else ctypes.byref(opts), plan.handle,
+                               rope.handle, _stream(stream)), "lc_bsa_backward")
+    return dq, dk, dv
 
 
 def cond_cache(cond_k: torch.Tensor, plan: Plan, rope: Rope3D, *,

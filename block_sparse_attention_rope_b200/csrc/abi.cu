@@ -182,6 +182,29 @@ extern "C" lc_status lc_bsa_forward_cached_ex(const void *q, const void *k, cons
                      (flags & LC_FLAG_COND_K_ROTATED) != 0, norm);
 }
 
+extern "C" lc_status lc_bsa_backward(const void *q, const void *k, const void *v, const void *out,
+                                     const float *lse, const void *dout, void *dq, void *dk,
+                                     void *dv, int batch, int heads, int head_dim, lc_dtype dtype,
+                                     float softmax_scale, const lc_bsa_opts *opts,
+                                     lc_bsa_plan plan, lc_rope3d rope, void *stream) {
+  lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype);
+  if (s != LC_OK) return s;
+  unsigned flags;
+  lc_qk_norm norm;
+  if (!parse_opts(opts, 0u, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
+  const void *ins[6] = {q, k, v, out, dout, lse};
+  for (const void *p : ins)
+    if (!p || misaligned(p)) return LC_ERR_INVALID_ARGUMENT;
+  void *outs[3] = {dq, dk, dv};
+  for (void *p : outs)
+    if (!p || misaligned(p)) return LC_ERR_INVALID_ARGUMENT;
+  if (batch > 65535 || heads > 65535) return LC_ERR_UNSUPPORTED;  // grid y / z
+  if (!(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;
+  float scale = softmax_scale > 0.f ? softmax_scale : 0.125f;
+  return lc_launch_backward(q, k, v, out, lse, dout, dq, dk, dv, batch, heads, scale, dtype, norm,
+                            plan, rope, static_cast<cudaStream_t>(stream));
+}
+
 extern "C" lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *cond_v,
                                        void *cond_k_rot, void *cond_out, float *cond_lse,
                                        int batch, int heads, int head_dim, lc_dtype dtype,

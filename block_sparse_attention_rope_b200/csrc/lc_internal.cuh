@@ -38,6 +38,9 @@ struct lc_bsa_plan_s {
   int *grp_cnt;             // [G]       planner work array
   uint32_t *grp_ent;        // [nnz]     (upper bound of the union lists)
   int *grp_order;           // [G]       groups by entry count, longest first
+  int *col_ptr;             // [nq + 1]  transpose (CSC): query blocks attending key block c
+  int *row_idx;             // [nnz]     ascending
+  int *col_cnt;             // [nq]      planner work array
   unsigned long long *pairs;  // [2] attended token pairs: all rows, noisy rows
   int *err;                 // [1] planner consistency flag
   long long pairs_host[2];
@@ -164,6 +167,12 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
                                   const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
                                   int *dev_status, cudaStream_t stream,
                                   int *counter_scratch = nullptr);
+// Gradients dq, dk, dv of the whole-sequence attention (attn_bwd.cu).
+lc_status lc_launch_backward(const void *q, const void *k, const void *v, const void *out,
+                             const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                             int batch, int heads, float scale, lc_dtype dtype,
+                             const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
+                             const lc_rope3d_s *rope, cudaStream_t stream);
 // Rotate x [batch, ntok, heads, 64] of dtype (token n of x = sequence token
 // n + tok_offset) into out, after an RMSNorm with norm_w when not NULL
 // (rope.cu; the public lc_rope3d_apply is this without the norm).  Arguments

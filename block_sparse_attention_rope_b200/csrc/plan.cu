@@ -15,7 +15,9 @@
 //   scan        one CTA: exclusive scans -> row_ptr, grp_ptr; checks nnz;
 //   row_fill    one warp per query block: ascending key ids -> col_idx;
 //   group_fill  one warp per group: union entries (key id | member mask << 24);
-//   order       one thread per group: rank by entry count, longest first.
+//   order       one thread per group: rank by entry count, longest first;
+//   col_scan,   one warp per key block: the transpose (CSC), ascending query
+//   col_fill    block ids attending it (walked by the backward pass).
 #include <algorithm>
 #include <new>
 
@@ -131,7 +133,8 @@ __device__ void block_exclusive_scan(const int *in, int *out, int n, long long *
 }
 
 __global__ void scan_kernel(PlanGeom g, const int *row_cnt, int *row_ptr, const int *grp_cnt,
-                            int *grp_ptr, long long nnz_expect, int *err) {
+                            int *grp_ptr, const int *col_cnt, int *col_ptr, long long nnz_expect,
+                            int *err) {
   __shared__ long long tot;
   block_exclusive_scan(row_cnt, row_ptr, g.nq, &tot);
   __syncthreads();
@@ -140,6 +143,47 @@ __global__ void scan_kernel(PlanGeom g, const int *row_cnt, int *row_ptr, const 
   block_exclusive_scan(grp_cnt, grp_ptr, g.G, &tot);
   __syncthreads();
   if (threadIdx.x == 0 && tot > nnz_expect) atomicOr(err, 2);
+  __syncthreads();
+  block_exclusive_scan(col_cnt, col_ptr, g.nq, &tot);
+  __syncthreads();
+  if (threadIdx.x == 0 && tot != nnz_expect) atomicOr(err, 16);
+}
+
+// Transpose of the pattern, one warp per key block c: how many query blocks
+// attend it, then their ids in ascending order.
+__global__ void col_scan_kernel(PlanGeom g, int *col_cnt) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= g.nq) return;
+  int c = warp, cnt = 0;
+  for (int r0 = 0; r0 < g.nq; r0 += 32) {
+    int r = r0 + lane;
+    cnt += __popc(__ballot_sync(0xffffffffu, r < g.nq && attends(r, c, g)));
+  }
+  if (lane == 0) col_cnt[c] = cnt;
+}
+
+__global__ void col_fill_kernel(PlanGeom g, const int *col_ptr, int *row_idx, long long nnz,
+                                int *err) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= g.nq) return;
+  int c = warp;
+  long long pos = col_ptr[c];
+  long long end = col_ptr[c + 1];
+  for (int r0 = 0; r0 < g.nq; r0 += 32) {
+    int r = r0 + lane;
+    bool a = r < g.nq && attends(r, c, g);
+    unsigned bal = __ballot_sync(0xffffffffu, a);
+    if (a) {
+      long long at = pos + __popc(bal & ((1u << lane) - 1u));
+      if (at < end && at < nnz)
+        row_idx[at] = r;
+      else
+        atomicOr(err, 32);
+    }
+    pos += __popc(bal);
+  }
 }
 
 __global__ void row_fill_kernel(PlanGeom g, const int *row_ptr, int *col_idx, long long nnz,
@@ -261,6 +305,7 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   carve<int>(probe, p->nq + 1); carve<int>(probe, nnz); carve<int>(probe, p->nq);
   carve<int>(probe, p->G + 1); carve<int>(probe, p->G); carve<uint32_t>(probe, nnz);
   carve<int>(probe, p->G); carve<unsigned long long>(probe, 2); carve<int>(probe, 1);
+  carve<int>(probe, p->nq + 1); carve<int>(probe, nnz); carve<int>(probe, p->nq);
   size_t bytes = reinterpret_cast<size_t>(probe);
   cudaError_t e = cudaMallocAsync(&p->mem, bytes, st);
   if (e != cudaSuccess) { delete p; return lc_from_cuda(e); }
@@ -274,6 +319,9 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->grp_order = carve<int>(q, p->G);
   p->pairs = carve<unsigned long long>(q, 2);
   p->err = carve<int>(q, 1);
+  p->col_ptr = carve<int>(q, p->nq + 1);
+  p->row_idx = carve<int>(q, nnz);
+  p->col_cnt = carve<int>(q, p->nq);
 
   PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride};
   e = cudaMemsetAsync(p->pairs, 0, 2 * sizeof(unsigned long long), st);
@@ -284,8 +332,10 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   if (e == cudaSuccess) {
     row_scan_kernel<<<row_blocks, tpb, 0, st>>>(g, p->row_cnt, p->pairs);
     group_count_kernel<<<grp_blocks, tpb, 0, st>>>(g, p->grp_cnt);
-    scan_kernel<<<1, 1024, 0, st>>>(g, p->row_cnt, p->row_ptr, p->grp_cnt, p->grp_ptr, nnz,
-                                    p->err);
+    col_scan_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_cnt);
+    scan_kernel<<<1, 1024, 0, st>>>(g, p->row_cnt, p->row_ptr, p->grp_cnt, p->grp_ptr,
+                                    p->col_cnt, p->col_ptr, nnz, p->err);
+    col_fill_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_ptr, p->row_idx, nnz, p->err);
     row_fill_kernel<<<row_blocks, tpb, 0, st>>>(g, p->row_ptr, p->col_idx, nnz, p->err);
     group_fill_kernel<<<grp_blocks, tpb, 0, st>>>(g, p->grp_ptr, p->grp_ent, nnz, p->err);
     order_kernel<<<(p->G + 127) / 128, 128, 0, st>>>(g, p->grp_cnt, p->grp_order);
@@ -333,6 +383,21 @@ extern "C" lc_status lc_bsa_plan_info(lc_bsa_plan plan, lc_bsa_plan_info_t *info
   info->attended_token_pairs = plan->pairs_host[0];
   info->attended_token_pairs_noisy = plan->pairs_host[1];
   return LC_OK;
+}
+
+extern "C" lc_status lc_bsa_plan_copy_csc(lc_bsa_plan plan, int *col_ptr_host, int *row_idx_host,
+                                          void *stream) {
+  if (!plan || !col_ptr_host || !row_idx_host) return LC_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  LC_CUDA_TRY(cudaStreamWaitEvent(st, plan->ready, 0));
+  LC_CUDA_TRY(cudaMemcpyAsync(col_ptr_host, plan->col_ptr, sizeof(int) * (plan->nq + 1),
+                              cudaMemcpyDeviceToHost, st));
+  LC_CUDA_TRY(cudaMemcpyAsync(row_idx_host, plan->row_idx, sizeof(int) * plan->nnz,
+                              cudaMemcpyDeviceToHost, st));
+  int err = 0;
+  LC_CUDA_TRY(cudaMemcpyAsync(&err, plan->err, sizeof(int), cudaMemcpyDeviceToHost, st));
+  LC_CUDA_TRY(cudaStreamSynchronize(st));
+  return err ? LC_ERR_DEVICE_CHECK : LC_OK;
 }
 
 extern "C" lc_status lc_bsa_plan_copy_csr(lc_bsa_plan plan, int *row_ptr_host, int *col_idx_host,

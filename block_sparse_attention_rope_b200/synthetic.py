@@ -19,6 +19,7 @@ from typing import Dict, Optional
 import torch
 
 SEED_Q, SEED_K, SEED_V, SEED_COND_K, SEED_COND_V = 1001, 1002, 1003, 1004, 1005
+SEED_DOUT = 1006  # output gradient of the backward pass
 
 
 @dataclass(frozen=True)
@@ -109,3 +110,12 @@ def make_inputs(w: Workload, device: Optional[str] = None, seed_offset: int = 0)
     if device is not None:
         out = {k: v.to(device) for k, v in out.items()}
     return out
+
+
+def make_dout(w: Workload, device: Optional[str] = None, seed_offset: int = 0) -> torch.Tensor:
+    """Seeded output gradient dO [B, Nq, heads, hd] for the backward pass
+    (Nq = all tokens, or the noisy ones for cached workloads), N(0,1) in the
+    workload's dtype."""
+    nq = w.n_noisy_tokens if w.cached else w.n_tokens
+    g = _randn((w.batch, nq, w.heads, w.head_dim), SEED_DOUT + seed_offset, w.torch_dtype())
+    return g.to(device) if device is not None else g

@@ -37,7 +37,7 @@
  *     [B, heads, Nq] fp32, natural log.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Every call is stream ordered and returns without waiting for the GPU,
- *     except lc_bsa_plan_info, lc_bsa_plan_copy_csr, lc_rope3d_copy_tables and
+ *     except lc_bsa_plan_info, lc_bsa_plan_copy_csr / _csc, lc_rope3d_copy_tables and
  *     lc_last_device_status, which synchronise the stream.
  *   - Errors are returned as lc_status; argument errors are detected before any
  *     GPU work is queued.  No C++ exception crosses this boundary.
@@ -108,6 +108,13 @@ lc_status lc_bsa_plan_destroy(lc_bsa_plan plan, void *stream);
 
 /* Sizes of a plan.  Waits for the plan's construction to finish. */
 lc_status lc_bsa_plan_info(lc_bsa_plan plan, lc_bsa_plan_info_t *info);
+
+/* Copy the transpose of the block CSR (CSC) to host memory:
+ * col_ptr_host[num_q_blocks + 1], row_idx_host[nnz] (int32): for key block c,
+ * the ascending query blocks that attend it (the backward pass walks these).
+ * Synchronises `stream`.  For checking the plan. */
+lc_status lc_bsa_plan_copy_csc(lc_bsa_plan plan, int *col_ptr_host, int *row_idx_host,
+                               void *stream);
 
 /* Copy the block CSR to host memory: row_ptr_host[num_q_blocks + 1],
  * col_idx_host[nnz] (int32).  Synchronises `stream`.  For checking the plan. */
@@ -247,6 +254,31 @@ lc_status lc_bsa_cond_cache(const void *cond_q, const void *cond_k, const void *
                             int heads, int head_dim, lc_dtype dtype, float softmax_scale,
                             const lc_bsa_opts *opts, lc_bsa_plan plan, lc_rope3d rope,
                             void *stream);
+
+/*
+ * lc_bsa_backward -- gradients of lc_bsa_forward (whole sequence) for the
+ * training path: the SimpleTuner page ("Guia de Início Rápido do LongCat-Video
+ * Edit", section "2) Mudanças no config") fine-tunes the model with LoRA and
+ * gradient checkpointing.  Given the forward's inputs q, k, v, its output
+ * `out` and lse (natural log, [batch, heads, N] fp32, as lc_bsa_forward wrote
+ * them) and the output gradient dout, writes
+ *   dv = P^T dout,  dS = P * (dout v^T - rowsum(dout * out)),
+ *   dq = norm_q^T(R^T(scale dS k')),  dk = norm_k^T(R^T(scale dS^T q'))
+ * over the attended pairs of `plan`, with P = exp(scale q' k'^T - lse) and
+ * q' = R(norm_q(q)), k' = R(norm_k(k)) as in the forward (opts: the same
+ * RMSNorm weights as the forward, flags 0; weight gradients are not
+ * produced).  All tensors [batch, N, heads, head_dim] of dtype, 16-byte
+ * aligned, caller owned; dq / dk / dv must not overlap the inputs.  fp32
+ * arithmetic for both dtypes (bf16 tensors are converted on load and the
+ * gradients rounded on store).  Scratch: batch * heads * N floats from the
+ * library's pool.  Errors as lc_bsa_forward; batch or heads above 65535:
+ * LC_ERR_UNSUPPORTED.
+ */
+lc_status lc_bsa_backward(const void *q, const void *k, const void *v, const void *out,
+                          const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                          int batch, int heads, int head_dim, lc_dtype dtype,
+                          float softmax_scale, const lc_bsa_opts *opts, lc_bsa_plan plan,
+                          lc_rope3d rope, void *stream);
 
 /*
  * lc_bsa_forward_noalloc -- lc_bsa_forward for callers that cannot allocate

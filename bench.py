@@ -218,7 +218,7 @@ def time_backward(api, synthetic, torch, name, steps, warmup, stream):
     return {"workload": name, "ms_per_layer": round(ms, 3),
             "attended_tflops": round(flops / (ms * 1e-3) / 1e12, 3),
             "work": "10*64 FLOP per attended pair and head",
-            "kernels": "bwd_delta, bwd_dq, bwd_dkdv (fp32 SIMT)"}
+            "kernels": "bwd_delta, bsa_bwd_sm100_kernel (tcgen05), bwd_dq_finalize"}
 
 
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):

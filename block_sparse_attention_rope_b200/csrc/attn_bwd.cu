@@ -15,13 +15,16 @@
 // CSR row, dk/dv walk a key block's CSC column ("longcat-video-rs", section
 // 03-03).
 //
-// Kernels: bwd_delta (D per row), bwd_dq (one CTA per query block x head x
-// batch, one thread per query row, key blocks staged rotated in shared
-// memory), bwd_dkdv (one CTA per key block, one thread per key row, query
-// blocks staged).  Every rotation uses the library's shared pair routine and
+// This file holds the fp32 path (bf16 goes to the tensor-core kernel in
+// attn_bwd_sm100.cu) and the pieces both paths share.  Kernels: bwd_delta (D
+// per row), bwd_dq (one CTA per query block x head x batch, one thread per
+// query row, key blocks staged rotated in shared memory), bwd_dkdv (one CTA
+// per key block, one thread per key row, query blocks staged),
+// bwd_dq_finalize (dq from the tensor-core path's fp32 sums).  Every rotation uses the library's shared pair routine and
 // RMSNorm order, so q' and k' are the forward's values before rounding.
 #include <cuda_bf16.h>
 #include <math.h>
+#include <string.h>
 
 #include "lc_internal.cuh"
 
@@ -312,6 +315,28 @@ __global__ void __launch_bounds__(64) bwd_dkdv_kernel(BwdArgs a) {
   }
 }
 
+// dq = norm_q^T(R^T dq_acc) for one (batch, token, head) row per thread.
+template <typename Tin>
+__global__ void bwd_dq_finalize_kernel(BwdArgs a, const float *acc, long long rows) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= rows) return;
+  const long long N = (long long)a.Nc + a.Nn;
+  const int n = (int)((i / a.heads) % N);
+  float g[LC_HEAD_DIM], x[LC_HEAD_DIM];
+  const float4 *src = reinterpret_cast<const float4 *>(acc + i * LC_HEAD_DIM);
+#pragma unroll
+  for (int c = 0; c < LC_HEAD_DIM / 4; ++c) {
+    const float4 v = src[c];
+    g[4 * c] = v.x; g[4 * c + 1] = v.y; g[4 * c + 2] = v.z; g[4 * c + 3] = v.w;
+  }
+  const Tin *Q = static_cast<const Tin *>(a.q) + i * LC_HEAD_DIM;
+#pragma unroll
+  for (int d = 0; d < LC_HEAD_DIM; ++d) x[d] = a.q_nw ? ld(Q, d) : 0.f;
+  rotate_norm_transpose(a, g, x, n, a.q_nw);
+#pragma unroll
+  for (int d = 0; d < LC_HEAD_DIM; ++d) st<Tin>(a.dq, i * LC_HEAD_DIM + d, g[d]);
+}
+
 template <typename Tin>
 lc_status launch_all(const BwdArgs &a, int batch, int nq, cudaStream_t st) {
   const long long rows = (long long)batch * (a.Nc + a.Nn) * a.heads;
@@ -328,11 +353,50 @@ lc_status launch_all(const BwdArgs &a, int batch, int nq, cudaStream_t st) {
 
 }  // namespace
 
+lc_status lc_bwd_delta(const void *out, const void *dout, float *delta, int batch, long long N,
+                       int heads, lc_dtype dtype, cudaStream_t stream) {
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.o = out; a.dout = dout; a.delta = delta; a.heads = heads;
+  a.Nc = 0; a.Nn = (int)N;
+  const long long rows = (long long)batch * N * heads;
+  if (rows == 0) return LC_OK;
+  if (dtype == LC_DTYPE_F32)
+    bwd_delta_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a, rows);
+  else
+    bwd_delta_kernel<__nv_bfloat16><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a, rows);
+  return lc_from_cuda(cudaGetLastError());
+}
+
+lc_status lc_bwd_dq_finalize(const float *dq_acc, const void *q, void *dq, int batch, long long N,
+                             int heads, lc_dtype dtype, const lc_qk_norm &norm,
+                             const lc_rope3d_s *rope, cudaStream_t stream) {
+  BwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.dq = dq; a.heads = heads; a.Nc = 0; a.Nn = (int)N;
+  a.tab = rope->tab;
+  a.q_nw = norm.q_w; a.norm_eps = norm.eps;
+  a.T = rope->T; a.H = rope->H; a.W = rope->W;
+  a.div_hw = lc_make_divmod(rope->H * rope->W);
+  a.div_w = lc_make_divmod(rope->W);
+  const long long rows = (long long)batch * N * heads;
+  if (rows == 0) return LC_OK;
+  const unsigned grid = (unsigned)((rows + 127) / 128);
+  if (dtype == LC_DTYPE_F32)
+    bwd_dq_finalize_kernel<float><<<grid, 128, 0, stream>>>(a, dq_acc, rows);
+  else
+    bwd_dq_finalize_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a, dq_acc, rows);
+  return lc_from_cuda(cudaGetLastError());
+}
+
 lc_status lc_launch_backward(const void *q, const void *k, const void *v, const void *out,
                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
                              int batch, int heads, float scale, lc_dtype dtype,
                              const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
                              const lc_rope3d_s *rope, cudaStream_t stream) {
+  if (dtype == LC_DTYPE_BF16)  // the tensor-core path
+    return lc_launch_backward_sm100(q, k, v, out, lse, dout, dq, dk, dv, batch, heads, scale,
+                                    norm, plan, rope, stream);
   BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.o = out; a.dout = dout; a.lse = lse;
   a.dq = dq; a.dk = dk; a.dv = dv;
@@ -356,8 +420,7 @@ lc_status lc_launch_backward(const void *q, const void *k, const void *v, const 
   cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&delta), dbytes, pool, stream);
   if (e != cudaSuccess) return lc_from_cuda(e);
   a.delta = delta;
-  s = dtype == LC_DTYPE_F32 ? launch_all<float>(a, batch, plan->nq, stream)
-                            : launch_all<__nv_bfloat16>(a, batch, plan->nq, stream);
+  s = launch_all<float>(a, batch, plan->nq, stream);
   cudaFreeAsync(delta, stream);
   return s;
 }

@@ -1,0 +1,778 @@
+// attn_bwd_sm100.cu -- tcgen05 backward of the block-sparse 3D-RoPE attention
+// (bf16 inputs, fp32 accumulation): dk and dv written directly, dq summed in
+// an fp32 buffer that attn_bwd.cu turns into dq.
+//
+// The gradients are the chain rule through the forward's definition (see
+// attn_bwd.cu for the formulas and the pages that motivate them).  Layout of
+// the work, one persistent CTA per SM:
+//   work item = (batch, head, key group of 2 key blocks = 128 keys), handed
+//               out longest query list first; the group walks the sorted
+//               union of the query blocks attending either key block (the
+//               plan's key-group lists), two query blocks (128 queries) per
+//               step.
+//   per step, with keys as TMEM lanes (M = 128):
+//     S^T  = K' Q'^T        dP^T = V dO^T          (tcgen05, into TMEM)
+//     P^T  = exp(scale S^T - lse),  dS^T = P^T (dP^T - D) scale
+//                           (warps 0-3, one key row per thread; P^T and dS^T
+//                            written back as bf16 over the consumed columns,
+//                            dS^T also to shared memory for dQ)
+//     dV  += P^T dO         dK' += dS^T Q'         (A from TMEM)
+//     dQ'  = dS K'          (A = dS from shared memory, MN-major; queries as
+//                            TMEM lanes), added to the fp32 buffer by warps
+//                            8-11 with vector atomics
+//   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
+//   warp 4: TMA producer (K, V per item, double-buffered; Q, dO per step,
+//   2 stages); warp 5: MMA issuer; warps 6-7: rotate K and Q tiles in shared
+//   memory and stage lse / D per step.
+//   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448).
+// Every mbarrier wait is bounded; on expiry the CTA stops, drains and frees
+// TMEM, and LC_DEVSTAT_TIMEOUT is set.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math.h>
+#include <string.h>
+
+#include "lc_internal.cuh"
+#include "sm100_ptx.cuh"
+#include "sm100_rope.cuh"
+#include "sm100_sync.cuh"
+
+namespace {
+
+using lcsm100::Ctx;
+using lcsm100::drain_wait;
+using lcsm100::rope_row;
+using lcsm100::wait_bar;
+using lcsm100::wait_warp;
+
+constexpr int kThreads = 384;
+constexpr int kWarpProducer = 4;
+constexpr int kWarpMma = 5;
+constexpr int kWarpRope = 6;  // and 7
+constexpr int kRopeThreads = 64;
+constexpr int kWarpDq = 8;    // 8-11
+constexpr int kQStages = 2;
+constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kBoxBytes = 64 * 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr uint32_t kIdescKQ = lcptx::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A in TMEM)
+constexpr uint32_t kIdescDQ = lcptx::idesc_bf16_f32(128, 64, 1, 1);   // dQ (A = dS, MN-major)
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct __align__(64) BwdParams {
+  CUtensorMap tmQ[2], tmK[2], tmV[2], tmG[2];  // [0] condition segment, [1] noisy; G = dO
+  const float *rope_tab;
+  const int *kg_ptr;
+  const uint32_t *kg_ent;
+  const int *kg_order;
+  int *work_counter;
+  int *status;
+  const float *lse;    // [B, heads, N] natural log (the forward's)
+  const float *delta;  // [B, heads, N] rowsum(dO * O)
+  float *dq_acc;       // [B, N, heads, 64] fp32, zero on entry
+  __nv_bfloat16 *dk, *dv;
+  const __nv_bfloat16 *k_raw;  // k as given (for the RMSNorm transpose)
+  const float *q_norm_w, *k_norm_w;
+  float norm_eps;
+  long long timeout_ns;
+  lc_divmod div_hw, div_w;
+  int T, H, W;
+  int Nc, Nn, Cb, kgc, heads, KG, total_items, tab_floats;
+  float scale;
+};
+
+struct SmemOffsets {
+  static constexpr int k = 0;                                  // [2] key tiles (rotated)
+  static constexpr int v = k + 2 * kTileBytes;                 // [2]
+  static constexpr int q = v + 2 * kTileBytes;                 // [kQStages] query tiles (rotated)
+  static constexpr int g = q + kQStages * kTileBytes;          // [kQStages] dO tiles
+  static constexpr int ds = g + kQStages * kTileBytes;         // dS^T, two MN-major 64-query tiles
+  static constexpr int lse = ds + 2 * kTileBytes;              // [kQStages][128] lse * log2e
+  static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] D
+  static constexpr int bars = del + kQStages * 128 * 4;
+  static constexpr int n_bars = 48;
+  static constexpr int misc = bars + n_bars * 8;
+  static constexpr int normw = misc + 64;
+  static constexpr int tab = normw + 2 * 64 * 4;
+};
+
+enum {
+  B_SCHED_FULL = 0,                 // [2]
+  B_SCHED_EMPTY = 2,                // [2]
+  B_KV_FULL = 4,                    // [2] K, V landed
+  B_KV_READY = 6,                   // [2] K rotated
+  B_KV_EMPTY = 8,                   // [2] item's MMAs done with K, V
+  B_QG_FULL = 10,                   // [kQStages] Q, dO landed
+  B_QG_READY = B_QG_FULL + kQStages,   // Q rotated, lse / D staged
+  B_QG_EMPTY = B_QG_READY + kQStages,  // step's MMAs done with Q, dO
+  B_SDP = B_QG_EMPTY + kQStages,    // S^T and dP^T in TMEM
+  B_PDS = B_SDP + 1,                // P^T, dS^T written (4 warps)
+  B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete
+  B_DQ_FULL = B_STEP + 1,           // dQ of a step in TMEM
+  B_DQ_EMPTY = B_DQ_FULL + 1,       // dQ read out (4 warps)
+  B_ACC = B_DQ_EMPTY + 1,           // item's dK, dV complete
+  B_EPI_FREE = B_ACC + 1,           // dK, dV read out (4 warps)
+  B_DRAIN = B_EPI_FREE + 1,
+  B_COUNT = B_DRAIN + 1
+};
+static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
+constexpr int kSchedConsumers = 4 + 1 + 2 + 4;  // elementwise, MMA, RoPE, dQ warps
+
+struct KItem {
+  int b, h, seg, kb0, cnt, krow0, seg_len, len;
+  const uint32_t *ent;
+};
+
+__device__ __forceinline__ KItem decode_kitem(const BwdParams &p, int item) {
+  KItem it;
+  const int per = p.KG;
+  const int bh = item / per;
+  const int g = p.kg_order[item - bh * per];
+  it.b = bh / p.heads;
+  it.h = bh - it.b * p.heads;
+  it.seg = g < p.kgc ? 0 : 1;
+  const int j = it.seg ? g - p.kgc : g;  // group index within the segment
+  const int nblk = it.seg ? (p.Nn + 63) / 64 : p.Cb;
+  it.kb0 = (it.seg ? p.Cb : 0) + 2 * j;
+  it.cnt = min(2, nblk - 2 * j);
+  it.krow0 = 128 * j;
+  it.seg_len = it.seg ? p.Nn : p.Nc;
+  const int lo = p.kg_ptr[g];
+  it.len = p.kg_ptr[g + 1] - lo;
+  it.ent = p.kg_ent + lo;
+  return it;
+}
+
+// Query block of a list entry -> segment, first row in the segment, tokens.
+__device__ __forceinline__ void qblock(const BwdParams &p, uint32_t e, int &seg, int &row,
+                                       int &cnt) {
+  const int r = (int)(e & 0xFFFFFFu);
+  if (r < p.Cb) {
+    seg = 0;
+    row = 64 * r;
+    cnt = min(64, p.Nc - row);
+  } else {
+    seg = 1;
+    row = 64 * (r - p.Cb);
+    cnt = min(64, p.Nn - row);
+  }
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// cos / sin of pair p (0..31) at token n.
+__device__ __forceinline__ void pair_angle(const BwdParams &a, const float *tab, int n, int p,
+                                           float &c, float &s) {
+  const int t = lc_div(n, a.div_hw);
+  const int rem = n - t * a.div_hw.d;
+  const int hh = lc_div(rem, a.div_w);
+  const int w = rem - hh * a.div_w.d;
+  if (p < 8) {
+    c = tab[t * 8 + p];
+    s = tab[a.T * 8 + t * 8 + p];
+  } else if (p < 20) {
+    c = tab[a.T * 16 + hh * 12 + p - 8];
+    s = tab[a.T * 16 + a.H * 12 + hh * 12 + p - 8];
+  } else {
+    c = tab[a.T * 16 + a.H * 24 + w * 12 + p - 20];
+    s = tab[a.T * 16 + a.H * 24 + a.W * 12 + w * 12 + p - 20];
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  uint8_t *sK = smem + SmemOffsets::k;
+  uint8_t *sV = smem + SmemOffsets::v;
+  uint8_t *sQ = smem + SmemOffsets::q;
+  uint8_t *sG = smem + SmemOffsets::g;
+  uint8_t *sDS = smem + SmemOffsets::ds;
+  float *sLse = reinterpret_cast<float *>(smem + SmemOffsets::lse);
+  float *sDel = reinterpret_cast<float *>(smem + SmemOffsets::del);
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SmemOffsets::misc);
+  // misc[0] tmem base, misc[1..2] scheduled items, misc[3] abort flag
+  float *s_normw = reinterpret_cast<float *>(smem + SmemOffsets::normw);  // [q 64 | k 64]
+  float *tab = reinterpret_cast<float *>(smem + SmemOffsets::tab);
+  Ctx ctx;
+  ctx.bar0 = lcptx::smem_addr(smem + SmemOffsets::bars);
+  ctx.abort_flag = reinterpret_cast<volatile int *>(&misc[3]);
+  ctx.status = p.status;
+  ctx.timeout_ns = p.timeout_ns;
+  const long long N = (long long)p.Nc + p.Nn;
+
+  for (int i = tid; i < p.tab_floats; i += kThreads) tab[i] = p.rope_tab[i];
+  if (tid < 64 && p.q_norm_w) s_normw[tid] = p.q_norm_w[tid];
+  if (tid < 64 && p.k_norm_w) s_normw[64 + tid] = p.k_norm_w[tid];
+  if (tid == 0) {
+    misc[3] = 0;
+    for (int i = 0; i < 2; ++i) {
+      lcptx::mbar_init(ctx.bar(B_SCHED_FULL + i), 1);
+      lcptx::mbar_init(ctx.bar(B_SCHED_EMPTY + i), kSchedConsumers);
+      lcptx::mbar_init(ctx.bar(B_KV_FULL + i), 1);
+      lcptx::mbar_init(ctx.bar(B_KV_READY + i), kRopeThreads);
+      lcptx::mbar_init(ctx.bar(B_KV_EMPTY + i), 1);
+    }
+    for (int s = 0; s < kQStages; ++s) {
+      lcptx::mbar_init(ctx.bar(B_QG_FULL + s), 1);
+      lcptx::mbar_init(ctx.bar(B_QG_READY + s), kRopeThreads);
+      lcptx::mbar_init(ctx.bar(B_QG_EMPTY + s), 1);
+    }
+    lcptx::mbar_init(ctx.bar(B_SDP), 1);
+    lcptx::mbar_init(ctx.bar(B_PDS), 4);
+    lcptx::mbar_init(ctx.bar(B_STEP), 1);
+    lcptx::mbar_init(ctx.bar(B_DQ_FULL), 1);
+    lcptx::mbar_init(ctx.bar(B_DQ_EMPTY), 4);
+    lcptx::mbar_init(ctx.bar(B_ACC), 1);
+    lcptx::mbar_init(ctx.bar(B_EPI_FREE), 4);
+    lcptx::mbar_init(ctx.bar(B_DRAIN), 1);
+    lcptx::fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    lcptx::tmem_alloc(lcptx::smem_addr(&misc[0]), kTmemCols);
+    lcptx::tmem_relinquish();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    for (int i = 0; i < 2; ++i) {
+      lcptx::tma_prefetch_desc(&p.tmQ[i]);
+      lcptx::tma_prefetch_desc(&p.tmK[i]);
+      lcptx::tma_prefetch_desc(&p.tmV[i]);
+      lcptx::tma_prefetch_desc(&p.tmG[i]);
+    }
+  }
+  lcptx::tc_fence_before();
+  __syncthreads();
+  lcptx::tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == kWarpProducer) {
+    // ======================= TMA producer (one thread) =======================
+    if (lane == 0) {
+      uint32_t item_it = 0, q_it = 0;
+      uint32_t kv_valid = 0, kv_par = 0, q_valid = 0, q_par = 0;  // for the drain
+      for (;;) {
+        const int slot = item_it & 1;
+        int item = atomicAdd(p.work_counter, 1);
+        if (item >= p.total_items) item = -1;
+        if (!wait_bar(ctx, ctx.bar(B_SCHED_EMPTY + slot), ((item_it >> 1) & 1) ^ 1)) break;
+        misc[1 + slot] = (uint32_t)item;
+        lcptx::mbar_arrive(ctx.bar(B_SCHED_FULL + slot));
+        if (item < 0) break;
+        const KItem it = decode_kitem(p, item);
+        const int kb = item_it & 1;
+        const uint32_t kph = (item_it >> 1) & 1;
+        bool ok = wait_bar(ctx, ctx.bar(B_KV_EMPTY + kb), kph ^ 1);
+        if (!ok) break;
+        {
+          const uint32_t bar = ctx.bar(B_KV_FULL + kb);
+          lcptx::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+          const uint32_t dk = lcptx::smem_addr(sK + kb * kTileBytes);
+          const uint32_t dv = lcptx::smem_addr(sV + kb * kTileBytes);
+          // rows past the segment end (a missing second block) read as zeros
+          lcptx::tma_load_4d(dk, &p.tmK[it.seg], bar, 0, it.h, it.krow0, it.b);
+          lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[it.seg], bar, 0, it.h, it.krow0 + 64, it.b);
+          lcptx::tma_load_4d(dv, &p.tmV[it.seg], bar, 0, it.h, it.krow0, it.b);
+          lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[it.seg], bar, 0, it.h, it.krow0 + 64, it.b);
+          kv_valid |= 1u << kb;
+          kv_par = (kv_par & ~(1u << kb)) | (kph << kb);
+        }
+        const int nsteps = (it.len + 1) >> 1;
+        for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
+          const int s = q_it % kQStages;
+          const uint32_t ph = (q_it / kQStages) & 1;
+          ok = wait_bar(ctx, ctx.bar(B_QG_EMPTY + s), ph ^ 1);
+          if (!ok) break;
+          int sa, ra, na, sb, rb, nb;
+          qblock(p, __ldg(it.ent + 2 * t), sa, ra, na);
+          if (2 * t + 1 < it.len) {
+            qblock(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
+          } else {  // no second query block: a box past the noisy segment's end reads zeros
+            sb = 1;
+            rb = p.Nn;
+          }
+          const uint32_t bar = ctx.bar(B_QG_FULL + s);
+          lcptx::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
+          const uint32_t dq = lcptx::smem_addr(sQ + s * kTileBytes);
+          const uint32_t dg = lcptx::smem_addr(sG + s * kTileBytes);
+          lcptx::tma_load_4d(dq, &p.tmQ[sa], bar, 0, it.h, ra, it.b);
+          lcptx::tma_load_4d(dq + kBoxBytes, &p.tmQ[sb], bar, 0, it.h, rb, it.b);
+          lcptx::tma_load_4d(dg, &p.tmG[sa], bar, 0, it.h, ra, it.b);
+          lcptx::tma_load_4d(dg + kBoxBytes, &p.tmG[sb], bar, 0, it.h, rb, it.b);
+          q_valid |= 1u << s;
+          q_par = (q_par & ~(1u << s)) | (ph << s);
+        }
+        if (!ok) break;
+        ++item_it;
+      }
+      // Drain: every load this thread issued must land before the CTA exits.
+      for (int i = 0; i < 2; ++i)
+        if ((kv_valid >> i) & 1u) drain_wait(ctx.bar(B_KV_FULL + i), (kv_par >> i) & 1u, p.timeout_ns);
+      for (int s = 0; s < kQStages; ++s)
+        if ((q_valid >> s) & 1u) drain_wait(ctx.bar(B_QG_FULL + s), (q_par >> s) & 1u, p.timeout_ns);
+    }
+  } else if (warp == kWarpMma) {
+    // ======================= MMA issuer (one thread) =========================
+    if (lane == 0) {
+      uint32_t item_it = 0, q_it = 0, k_step = 0;
+      uint32_t pds_ph = 0, step_ph = 0;
+      bool step_pending = false;
+      constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+      constexpr uint32_t kTileLo = kTileBytes >> 4;
+      auto desc = [](uint32_t lo) -> uint64_t {
+        return (static_cast<uint64_t>(kDescHi) << 32) | lo;
+      };
+      // K-major operands (leading byte offset 16) and MN-major ones with one
+      // 64-element chunk (leading byte offset unused); dS^T as the MN-major A
+      // of dQ has two 64-query chunks 16 KB apart.
+      const uint32_t k_km = (lcptx::smem_addr(sK) >> 4) | (1u << 16);
+      const uint32_t v_km = (lcptx::smem_addr(sV) >> 4) | (1u << 16);
+      const uint32_t q_km = (lcptx::smem_addr(sQ) >> 4) | (1u << 16);
+      const uint32_t g_km = (lcptx::smem_addr(sG) >> 4) | (1u << 16);
+      const uint32_t k_mn = (lcptx::smem_addr(sK) >> 4) | (512u << 16);
+      const uint32_t q_mn = (lcptx::smem_addr(sQ) >> 4) | (512u << 16);
+      const uint32_t g_mn = (lcptx::smem_addr(sG) >> 4) | (512u << 16);
+      const uint32_t ds_mn = (lcptx::smem_addr(sDS) >> 4) | ((uint32_t)(kTileBytes >> 4) << 16);
+      for (;;) {
+        const int slot = item_it & 1;
+        if (!wait_bar(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
+        const int item = (int)misc[1 + slot];
+        lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
+        if (item < 0) break;
+        const KItem it = decode_kitem(p, item);
+        const int kb = item_it & 1;
+        const uint32_t kph = (item_it >> 1) & 1;
+        bool ok = wait_bar(ctx, ctx.bar(B_KV_READY + kb), kph);
+        const int nsteps = (it.len + 1) >> 1;
+        for (int t = 0; t < nsteps && ok; ++t, ++q_it, ++k_step) {
+          const int s = q_it % kQStages;
+          const uint32_t ph = (q_it / kQStages) & 1;
+          ok = wait_bar(ctx, ctx.bar(B_QG_READY + s), ph);
+          if (!ok) break;
+          // S^T of this step overwrites P^T of the previous one: its P*V must be done.
+          if (step_pending) {
+            ok = wait_bar(ctx, ctx.bar(B_STEP), step_ph);
+            if (!ok) break;
+            step_ph ^= 1;
+            step_pending = false;
+          }
+          lcptx::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            lcptx::mma_ss(tmem + kColST, desc(k_km + kb * kTileLo + 2 * kk),
+                          desc(q_km + s * kTileLo + 2 * kk), kIdescKQ, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            lcptx::mma_ss(tmem + kColDPT, desc(v_km + kb * kTileLo + 2 * kk),
+                          desc(g_km + s * kTileLo + 2 * kk), kIdescKQ, kk > 0);
+          lcptx::mma_commit(ctx.bar(B_SDP));
+          ok = wait_bar(ctx, ctx.bar(B_PDS), pds_ph);
+          if (!ok) break;
+          pds_ph ^= 1;
+          if (t == 0 && item_it > 0) {  // the previous item's dK, dV have been read out
+            ok = wait_bar(ctx, ctx.bar(B_EPI_FREE), (item_it - 1) & 1);
+            if (!ok) break;
+          }
+          lcptx::tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            lcptx::mma_ts(tmem + kColDV, tmem + kColST + 8 * kk, desc(g_mn + s * kTileLo + 128 * kk),
+                          kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            lcptx::mma_ts(tmem + kColDK, tmem + kColDPT + 8 * kk, desc(q_mn + s * kTileLo + 128 * kk),
+                          kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+          if (k_step > 0) {  // the dQ warps have read the previous step's dQ
+            ok = wait_bar(ctx, ctx.bar(B_DQ_EMPTY), (k_step - 1) & 1);
+            if (!ok) break;
+            lcptx::tc_fence_after();
+          }
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            lcptx::mma_ss(tmem + kColDQ, desc(ds_mn + 128 * kk), desc(k_mn + kb * kTileLo + 128 * kk),
+                          kIdescDQ, kk > 0);
+          lcptx::mma_commit(ctx.bar(B_DQ_FULL));
+          lcptx::mma_commit(ctx.bar(B_QG_EMPTY + s));
+          lcptx::mma_commit(ctx.bar(B_STEP));
+          step_pending = true;
+          if (t + 1 == nsteps) {
+            lcptx::mma_commit(ctx.bar(B_ACC));
+            lcptx::mma_commit(ctx.bar(B_KV_EMPTY + kb));
+          }
+        }
+        if (!ok) break;
+        ++item_it;
+      }
+      lcptx::mma_commit(ctx.bar(B_DRAIN));
+      drain_wait(ctx.bar(B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == kWarpRope || warp == kWarpRope + 1) {
+    // ======================= RoPE warps: K per item, Q + lse / D per step ====
+    const int rt = tid - kWarpRope * 32;
+    const float *q_nw = p.q_norm_w ? s_normw : nullptr;
+    const float *k_nw = p.k_norm_w ? s_normw + 64 : nullptr;
+    uint32_t item_it = 0, q_it = 0;
+    for (;;) {
+      const int slot = item_it & 1;
+      if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
+      const int item = (int)misc[1 + slot];
+      __syncwarp();
+      if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
+      if (item < 0) break;
+      const KItem it = decode_kitem(p, item);
+      const int kb = item_it & 1;
+      bool ok = wait_warp(ctx, ctx.bar(B_KV_FULL + kb), (item_it >> 1) & 1);
+      if (!ok) break;
+      const int seg_tok = it.seg ? p.Nc : 0;
+      for (int r = rt; r < 128; r += kRopeThreads)
+        if (it.krow0 + r < it.seg_len && (r >> 6) < it.cnt)
+          rope_row(sK + kb * kTileBytes, r, seg_tok + it.krow0 + r, tab, p, k_nw);
+      lcptx::fence_proxy_async_smem();
+      lcptx::mbar_arrive(ctx.bar(B_KV_READY + kb));
+      const int nsteps = (it.len + 1) >> 1;
+      const float *lse_bh = p.lse + ((long long)it.b * p.heads + it.h) * N;
+      const float *del_bh = p.delta + ((long long)it.b * p.heads + it.h) * N;
+      for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
+        const int s = q_it % kQStages;
+        ok = wait_warp(ctx, ctx.bar(B_QG_FULL + s), (q_it / kQStages) & 1);
+        if (!ok) break;
+        for (int r = rt; r < 128; r += kRopeThreads) {
+          const int e = 2 * t + (r >> 6);
+          float l2 = 0.f, dl = 0.f;
+          if (e < it.len) {
+            int qs, qr, qn;
+            qblock(p, __ldg(it.ent + e), qs, qr, qn);
+            if ((r & 63) < qn) {
+              const int tok = (qs ? p.Nc : 0) + qr + (r & 63);
+              rope_row(sQ + s * kTileBytes, r, tok, tab, p, q_nw);
+              l2 = __ldg(lse_bh + tok) * kLog2e;
+              dl = __ldg(del_bh + tok);
+            }
+          }
+          sLse[s * 128 + r] = l2;
+          sDel[s * 128 + r] = dl;
+        }
+        lcptx::fence_proxy_async_smem();
+        lcptx::mbar_arrive(ctx.bar(B_QG_READY + s));
+      }
+      if (!ok) break;
+      ++item_it;
+    }
+  } else if (warp >= kWarpDq) {
+    // ======================= dQ warps: TMEM dQ -> fp32 atomics ================
+    const int qrow = tid - kWarpDq * 32;  // TMEM lane == query row of the step
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    uint32_t item_it = 0, dq_ph = 0;
+    for (;;) {
+      const int slot = item_it & 1;
+      if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
+      const int item = (int)misc[1 + slot];
+      __syncwarp();
+      if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
+      if (item < 0) break;
+      const KItem it = decode_kitem(p, item);
+      const int nsteps = (it.len + 1) >> 1;
+      bool ok = true;
+      for (int t = 0; t < nsteps; ++t) {
+        ok = wait_warp(ctx, ctx.bar(B_DQ_FULL), dq_ph);
+        if (!ok) break;
+        dq_ph ^= 1;
+        lcptx::tc_fence_after();
+        uint32_t a0[32], a1[32];
+        lcptx::tmem_ld32(tmem + lane_base + kColDQ, a0);
+        lcptx::tmem_ld32(tmem + lane_base + kColDQ + 32, a1);
+        lcptx::tmem_wait_ld();
+        lcptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_DQ_EMPTY));
+        const int e = 2 * t + (qrow >> 6);
+        if (e < it.len) {
+          int qs, qr, qn;
+          qblock(p, __ldg(it.ent + e), qs, qr, qn);
+          if ((qrow & 63) < qn) {
+            const long long tok = (qs ? p.Nc : 0) + qr + (qrow & 63);
+            float4 *dst = reinterpret_cast<float4 *>(
+                p.dq_acc + (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              atomicAdd(dst + c, make_float4(__uint_as_float(a0[4 * c]), __uint_as_float(a0[4 * c + 1]),
+                                             __uint_as_float(a0[4 * c + 2]), __uint_as_float(a0[4 * c + 3])));
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              atomicAdd(dst + 8 + c, make_float4(__uint_as_float(a1[4 * c]), __uint_as_float(a1[4 * c + 1]),
+                                                 __uint_as_float(a1[4 * c + 2]), __uint_as_float(a1[4 * c + 3])));
+          }
+        }
+      }
+      if (!ok) break;
+      ++item_it;
+    }
+  } else {
+    // ======================= elementwise warps 0-3 (thread = key row) ========
+    const int kr = tid;  // TMEM lane == key row of the group
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tST = tmem + lane_base + kColST, tDPT = tmem + lane_base + kColDPT;
+    const float sl2 = p.scale * kLog2e;
+    uint32_t item_it = 0, q_it = 0, sdp_ph = 0;
+    for (;;) {
+      const int slot = item_it & 1;
+      if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
+      const int item = (int)misc[1 + slot];
+      __syncwarp();
+      if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
+      if (item < 0) break;
+      const KItem it = decode_kitem(p, item);
+      const bool key_valid = (kr >> 6) < it.cnt && it.krow0 + kr < it.seg_len;
+      const int nsteps = (it.len + 1) >> 1;
+      bool ok = true;
+      for (int t = 0; t < nsteps; ++t, ++q_it) {
+        const int s = q_it % kQStages;
+        // attended query tokens of the step's two query blocks, for this key row
+        int lim[2];
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          lim[hq] = 0;
+          const int e = 2 * t + hq;
+          if (key_valid && e < it.len) {
+            const uint32_t ent = __ldg(it.ent + e);
+            if ((ent >> (24 + (kr >> 6))) & 1u) {
+              int qs, qr, qn;
+              qblock(p, ent, qs, qr, qn);
+              lim[hq] = qn;
+            }
+          }
+        }
+        // the staged lse / D of this step (written by the RoPE warps), then S^T, dP^T
+        ok = wait_warp(ctx, ctx.bar(B_QG_READY + s), (q_it / kQStages) & 1) &&
+             wait_warp(ctx, ctx.bar(B_SDP), sdp_ph);
+        if (!ok) break;
+        sdp_ph ^= 1;
+        lcptx::tc_fence_after();
+        const float *l2 = sLse + s * 128, *dl = sDel + s * 128;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {  // 32 queries at a time
+          uint32_t sr[32], dr[32];
+          lcptx::tmem_ld32(tST + 32 * c, sr);
+          lcptx::tmem_ld32(tDPT + 32 * c, dr);
+          lcptx::tmem_wait_ld();
+          const int hq = c >> 1;
+          const int jb = (c & 1) * 32;  // first query of the chunk within its block
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float pv[2], dv2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int j = 32 * c + 2 * i + u;
+              const bool on = jb + 2 * i + u < lim[hq];
+              const float pe = on ? ex2(__uint_as_float(sr[2 * i + u]) * sl2 - l2[j]) : 0.f;
+              pv[u] = pe;
+              dv2[u] = pe * (__uint_as_float(dr[2 * i + u]) - dl[j]) * p.scale;
+            }
+            pp[i] = pack_bf16(pv[0], pv[1]);
+            dd[i] = pack_bf16(dv2[0], dv2[1]);
+          }
+          lcptx::tmem_st16(tST + 16 * c, pp);
+          lcptx::tmem_st16(tDPT + 16 * c, dd);
+          // dS^T row kr, queries 32c..32c+31, into the MN-major dQ operand:
+          // tile hq (queries 64 hq .. 64 hq + 63), 16-byte chunks (c & 1) * 4 + i.
+          uint8_t *tile = sDS + hq * kTileBytes;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<uint4 *>(tile + swz(kr, (c & 1) * 4 + i)) =
+                make_uint4(dd[4 * i], dd[4 * i + 1], dd[4 * i + 2], dd[4 * i + 3]);
+        }
+        lcptx::fence_proxy_async_smem();
+        lcptx::tmem_wait_st();
+        lcptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));
+      }
+      if (!ok) break;
+      // ---- epilogue: dK = R^T dK' (and the RMSNorm transpose), dV; stored bf16
+      ok = wait_warp(ctx, ctx.bar(B_ACC), item_it & 1);
+      if (!ok) break;
+      lcptx::tc_fence_after();
+      const int tok = (it.seg ? p.Nc : 0) + it.krow0 + kr;
+      const long long off = (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM;
+      float dkv[64];
+      {
+        uint32_t a[32], b2[32];
+        lcptx::tmem_ld32(tmem + lane_base + kColDV, a);
+        lcptx::tmem_ld32(tmem + lane_base + kColDV + 32, b2);
+        lcptx::tmem_wait_ld();
+        if (key_valid) {
+          uint4 *gv = reinterpret_cast<uint4 *>(p.dv + off);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            gv[c] = make_uint4(pack_bf16(__uint_as_float(a[8 * c]), __uint_as_float(a[8 * c + 1])),
+                               pack_bf16(__uint_as_float(a[8 * c + 2]), __uint_as_float(a[8 * c + 3])),
+                               pack_bf16(__uint_as_float(a[8 * c + 4]), __uint_as_float(a[8 * c + 5])),
+                               pack_bf16(__uint_as_float(a[8 * c + 6]), __uint_as_float(a[8 * c + 7])));
+            gv[4 + c] = make_uint4(pack_bf16(__uint_as_float(b2[8 * c]), __uint_as_float(b2[8 * c + 1])),
+                                   pack_bf16(__uint_as_float(b2[8 * c + 2]), __uint_as_float(b2[8 * c + 3])),
+                                   pack_bf16(__uint_as_float(b2[8 * c + 4]), __uint_as_float(b2[8 * c + 5])),
+                                   pack_bf16(__uint_as_float(b2[8 * c + 6]), __uint_as_float(b2[8 * c + 7])));
+          }
+        }
+        lcptx::tmem_ld32(tmem + lane_base + kColDK, a);
+        lcptx::tmem_ld32(tmem + lane_base + kColDK + 32, b2);
+        lcptx::tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < 32; ++d) {
+          dkv[d] = __uint_as_float(a[d]);
+          dkv[32 + d] = __uint_as_float(b2[d]);
+        }
+      }
+      lcptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_EPI_FREE));
+      if (key_valid) {
+#pragma unroll
+        for (int q2 = 0; q2 < 32; ++q2) {  // R^T: turn each pair back
+          float c, sn;
+          pair_angle(p, tab, tok, q2, c, sn);
+          const float u = dkv[2 * q2], w = dkv[2 * q2 + 1];
+          dkv[2 * q2] = fmaf(u, c, w * sn);
+          dkv[2 * q2 + 1] = fmaf(w, c, -u * sn);
+        }
+        if (p.k_norm_w) {  // y = x inv w:  dx = inv (w g) - x inv^3 / 64 * sum(g w x)
+          float c8[8];
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            float x8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x8[e] = __bfloat162float(p.k_raw[off + 8 * ch + e]);
+            c8[ch] = lc_sumsq8(x8);
+          }
+          const float inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
+          float dot = 0.f;
+#pragma unroll
+          for (int d = 0; d < 64; ++d)
+            dot = fmaf(dkv[d] * s_normw[64 + d], __bfloat162float(p.k_raw[off + d]), dot);
+          const float k3 = inv * inv * inv * (1.f / 64.f) * dot;
+#pragma unroll
+          for (int d = 0; d < 64; ++d)
+            dkv[d] = inv * s_normw[64 + d] * dkv[d] - __bfloat162float(p.k_raw[off + d]) * k3;
+        }
+        uint4 *gk = reinterpret_cast<uint4 *>(p.dk + off);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          gk[c] = make_uint4(pack_bf16(dkv[8 * c], dkv[8 * c + 1]), pack_bf16(dkv[8 * c + 2], dkv[8 * c + 3]),
+                             pack_bf16(dkv[8 * c + 4], dkv[8 * c + 5]), pack_bf16(dkv[8 * c + 6], dkv[8 * c + 7]));
+      }
+      ++item_it;
+    }
+  }
+
+  // ---- teardown
+  lcptx::tc_fence_before();
+  __syncthreads();
+  lcptx::tc_fence_after();
+  if (warp == kWarpMma) lcptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, const void *out,
+                                   const float *lse, const void *dout, void *dq, void *dk,
+                                   void *dv, int batch, int heads, float scale,
+                                   const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
+                                   const lc_rope3d_s *rope, cudaStream_t stream) {
+  BwdParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
+  const void *src[4] = {q, k, v, dout};
+  CUtensorMap *maps[4] = {prm.tmQ, prm.tmK, prm.tmV, prm.tmG};
+  for (int i = 0; i < 4; ++i) {
+    lc_status s = lc_encode_segment(&maps[i][1], src[i], batch, N, Nc, Nn, heads);
+    if (s == LC_OK && Nc > 0) s = lc_encode_segment(&maps[i][0], src[i], batch, N, 0, Nc, heads);
+    if (s != LC_OK) return s;
+    if (Nc == 0) maps[i][0] = maps[i][1];  // unused, kept a valid descriptor
+  }
+  prm.rope_tab = rope->tab;
+  prm.kg_ptr = plan->kgrp_ptr;
+  prm.kg_ent = plan->kgrp_ent;
+  prm.kg_order = plan->kgrp_order;
+  prm.lse = lse;
+  prm.dk = static_cast<__nv_bfloat16 *>(dk);
+  prm.dv = static_cast<__nv_bfloat16 *>(dv);
+  prm.k_raw = static_cast<const __nv_bfloat16 *>(k);
+  prm.q_norm_w = norm.q_w;
+  prm.k_norm_w = norm.k_w;
+  prm.norm_eps = norm.eps;
+  prm.timeout_ns = 2000000000LL;
+  prm.div_hw = lc_make_divmod(rope->H * rope->W);
+  prm.div_w = lc_make_divmod(rope->W);
+  prm.T = rope->T; prm.H = rope->H; prm.W = rope->W;
+  prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.kgc = plan->kgc;
+  prm.heads = heads;
+  prm.KG = plan->KG;
+  prm.tab_floats = (int)rope->n_floats;
+  prm.scale = scale;
+  const long long total = (long long)batch * heads * plan->KG;
+  if (total == 0) return LC_OK;
+  if (total >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
+  prm.total_items = (int)total;
+  const size_t smem = 1024 + SmemOffsets::tab + sizeof(float) * (size_t)rope->n_floats;
+  if (smem > 227 * 1024) return LC_ERR_UNSUPPORTED;
+  lc_status s = LC_OK;
+  prm.status = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
+  cudaMemPool_t pool = lc_scratch_pool(&s);
+  if (s != LC_OK) return s;
+  int dev = 0, n_sm = 0;
+  LC_CUDA_TRY(cudaGetDevice(&dev));
+  LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  LC_CUDA_TRY(cudaFuncSetAttribute(bsa_bwd_sm100_kernel,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));
+  const size_t rows = (size_t)batch * N * heads;
+  float *delta = nullptr, *dq_acc = nullptr;
+  int *counter = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&delta), rows * sizeof(float),
+                                          pool, stream);
+  if (e == cudaSuccess)
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&dq_acc),
+                                rows * LC_HEAD_DIM * sizeof(float), pool, stream);
+  if (e == cudaSuccess)
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&counter), sizeof(int), pool, stream);
+  if (e == cudaSuccess)
+    e = cudaMemsetAsync(dq_acc, 0, rows * LC_HEAD_DIM * sizeof(float), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+  if (e == cudaSuccess)
+    s = lc_bwd_delta(out, dout, delta, batch, N, heads, LC_DTYPE_BF16, stream);
+  if (e == cudaSuccess && s == LC_OK) {
+    prm.delta = delta;
+    prm.dq_acc = dq_acc;
+    prm.work_counter = counter;
+    const int grid = (int)(total < n_sm ? total : n_sm);
+    bsa_bwd_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess && s == LC_OK)
+    s = lc_bwd_dq_finalize(dq_acc, q, dq, batch, N, heads, LC_DTYPE_BF16, norm, rope, stream);
+  if (counter) cudaFreeAsync(counter, stream);
+  if (dq_acc) cudaFreeAsync(dq_acc, stream);
+  if (delta) cudaFreeAsync(delta, stream);
+  if (s != LC_OK) return s;
+  return lc_from_cuda(e);
+}

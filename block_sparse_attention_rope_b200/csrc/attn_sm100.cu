@@ -42,6 +42,8 @@
 
 #include "lc_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "sm100_sync.cuh"
+#include "sm100_rope.cuh"
 
 namespace {
 
@@ -155,43 +157,9 @@ enum {
 static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
 constexpr int kSchedConsumers = 8 + 1 + 2;  // softmax warps, MMA warp, RoPE warps
 
-struct Ctx {
-  uint32_t bar0;                 // smem address of barrier 0
-  volatile int *abort_flag;      // smem
-  int *status;
-  long long timeout_ns;
-  __device__ uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
-};
-
-// Bounded wait: true when the phase of `parity` completed; false when the CTA
-// aborted or this wait timed out (which sets the abort flag and the status).
-// (Everything is inlined: register-split regions must not contain calls.)
-__device__ __forceinline__ bool wait_bar_slow(const Ctx &c, uint32_t bar, uint32_t parity) {
-  uint64_t t0 = lcptx::globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (lcptx::mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0) {
-      if (*c.abort_flag) return false;
-      if ((long long)(lcptx::globaltimer_ns() - t0) > c.timeout_ns) {
-        atomicOr(c.status, LC_DEVSTAT_TIMEOUT);
-        *c.abort_flag = 1;
-        __threadfence_block();
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ bool wait_bar(const Ctx &c, uint32_t bar, uint32_t parity) {
-  if (lcptx::mbar_try_wait(bar, parity)) return true;
-  return wait_bar_slow(c, bar, parity);
-}
-
-// Warp-uniform form for warps whose lanes then run .sync.aligned tcgen05 ops
-// together: every lane waits, and the warp fails as one if any lane failed.
-__device__ __forceinline__ bool wait_warp(const Ctx &c, uint32_t bar, uint32_t parity) {
-  return __all_sync(0xffffffffu, wait_bar(c, bar, parity)) != 0;
-}
+using lcsm100::Ctx;
+using lcsm100::wait_bar;
+using lcsm100::wait_warp;
 
 struct Item {
   int b, h, seg, row0, seg_len, len;
@@ -260,78 +228,9 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// One 16-byte chunk (8 bf16 channels, packed pairs in wds) of a token row:
-// optional RMSNorm (inv = 1/rms of the row, w8 = the chunk's 8 weights), then
-// the rotation of its 4 channel pairs, rounded back to bf16.
-__device__ __forceinline__ void rot_chunk_bf16(uint32_t (&wds)[4], const float4 cc,
-                                               const float4 ss, bool norm, float inv,
-                                               const float (&w8)[8]) {
-  const float cs[4] = {cc.x, cc.y, cc.z, cc.w}, sn[4] = {ss.x, ss.y, ss.z, ss.w};
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    float a = __uint_as_float(wds[q] << 16);
-    float b = __uint_as_float(wds[q] & 0xFFFF0000u);
-    if (norm) {
-      a = lc_rms_apply(a, inv, w8[2 * q]);
-      b = lc_rms_apply(b, inv, w8[2 * q + 1]);
-    }
-    float xr, yr;
-    lc_rot_pair(a, b, cs[q], sn[q], xr, yr);
-    __nv_bfloat162 o2 = __floats2bfloat162_rn(xr, yr);
-    wds[q] = *reinterpret_cast<uint32_t *>(&o2);
-  }
-}
-
-// Sum of squares of the 8 bf16 channels of a chunk.
-__device__ __forceinline__ float sumsq_chunk_bf16(const uint32_t (&wds)[4]) {
-  float v[8];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    v[2 * q] = __uint_as_float(wds[q] << 16);
-    v[2 * q + 1] = __uint_as_float(wds[q] & 0xFFFF0000u);
-  }
-  return lc_sumsq8(v);
-}
-
-// Rotate one token row (64 bf16 channels, 128-byte swizzled) in place, after
-// an RMSNorm with the 64 weights nw when nw is not NULL.
-__device__ __forceinline__ void rope_row(uint8_t *tile, int r, int n, const float *tab,
-                                         const Sm100Params &p, const float *nw) {
-  const int t = lc_div(n, p.div_hw);
-  const int rem = n - t * p.div_hw.d;
-  const int hh = lc_div(rem, p.div_w);
-  const int w = rem - hh * p.div_w.d;
-  const float *cT = tab + t * 8, *sT = tab + p.T * 8 + t * 8;
-  const float *cH = tab + p.T * 16 + hh * 12, *sH = cH + p.H * 12;
-  const float *cW = tab + p.T * 16 + p.H * 24 + w * 12, *sW = cW + p.W * 12;
-  uint8_t *rowp = tile + r * 128;
-  const int x = r & 7;
-  float inv = 1.f;
-  if (nw) {
-    float c8[8];
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(rowp + ((ch ^ x) << 4));
-      const uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-      c8[ch] = sumsq_chunk_bf16(wds);
-    }
-    inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
-  }
-#pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
-    const float *c = ch < 2 ? cT + 4 * ch : (ch < 5 ? cH + 4 * (ch - 2) : cW + 4 * (ch - 5));
-    const float *s = ch < 2 ? sT + 4 * ch : (ch < 5 ? sH + 4 * (ch - 2) : sW + 4 * (ch - 5));
-    uint4 *ptr = reinterpret_cast<uint4 *>(rowp + ((ch ^ x) << 4));
-    const uint4 raw = *ptr;
-    uint32_t wds[4] = {raw.x, raw.y, raw.z, raw.w};
-    float w8[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w8[e] = nw ? nw[8 * ch + e] : 1.f;
-    rot_chunk_bf16(wds, *reinterpret_cast<const float4 *>(c), *reinterpret_cast<const float4 *>(s),
-                   nw != nullptr, inv, w8);
-    *ptr = make_uint4(wds[0], wds[1], wds[2], wds[3]);
-  }
-}
+using lcsm100::rope_row;
+using lcsm100::rot_chunk_bf16;
+using lcsm100::sumsq_chunk_bf16;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -1002,8 +901,6 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// Tensor map over one segment of a [B, ntot, heads, 64] bf16 tensor: tokens
-// [tok0, tok0 + nseg) of every batch entry; boxes of 64 tokens x 1 head.
 lc_status encode_segment(CUtensorMap *m, const void *base, int batch, long long ntot,
                          long long tok0, long long nseg, int heads) {
   EncodeTiledFn fn = get_encode_fn();
@@ -1093,6 +990,11 @@ lc_status launch_rope_k(const void *src, void *dst, int batch, long long ntok, i
 }
 
 }  // namespace
+
+lc_status lc_encode_segment(CUtensorMap *m, const void *base, int batch, long long ntot,
+                            long long tok0, long long nseg, int heads) {
+  return encode_segment(m, base, batch, ntot, tok0, nseg, heads);
+}
 
 // ------------------------------------------------------------ no-alloc scratch
 // Fixed device scratch for lc_bsa_forward_noalloc, for callers that must not

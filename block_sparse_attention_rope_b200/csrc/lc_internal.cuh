@@ -41,6 +41,15 @@ struct lc_bsa_plan_s {
   int *col_ptr;             // [nq + 1]  transpose (CSC): query blocks attending key block c
   int *row_idx;             // [nnz]     ascending
   int *col_cnt;             // [nq]      planner work array
+  // Backward work lists: key groups of 2 consecutive key blocks of one
+  // segment (kgc condition groups, then kgn noisy ones), each with the sorted
+  // union of the query blocks attending either member (entry = query block id
+  // | member mask << 24), and the groups ranked longest list first.
+  int kgc, kgn, KG;
+  int *kgrp_ptr;            // [KG + 1]
+  int *kgrp_cnt;            // [KG]
+  uint32_t *kgrp_ent;       // [nnz]     (upper bound of the union lists)
+  int *kgrp_order;          // [KG]
   unsigned long long *pairs;  // [2] attended token pairs: all rows, noisy rows
   int *err;                 // [1] planner consistency flag
   long long pairs_host[2];
@@ -172,6 +181,19 @@ lc_status lc_launch_backward(const void *q, const void *k, const void *v, const 
                              const float *lse, const void *dout, void *dq, void *dk, void *dv,
                              int batch, int heads, float scale, lc_dtype dtype,
                              const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
+                             const lc_rope3d_s *rope, cudaStream_t stream);
+// The tensor-core backward (attn_bwd_sm100.cu, bf16), and the pieces of the
+// backward shared by both paths (attn_bwd.cu): D = rowsum(dO * O) per row, and
+// dq = norm_q^T(R^T dq_acc) cast to dtype.
+lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, const void *out,
+                                   const float *lse, const void *dout, void *dq, void *dk,
+                                   void *dv, int batch, int heads, float scale,
+                                   const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
+                                   const lc_rope3d_s *rope, cudaStream_t stream);
+lc_status lc_bwd_delta(const void *out, const void *dout, float *delta, int batch, long long N,
+                       int heads, lc_dtype dtype, cudaStream_t stream);
+lc_status lc_bwd_dq_finalize(const float *dq_acc, const void *q, void *dq, int batch, long long N,
+                             int heads, lc_dtype dtype, const lc_qk_norm &norm,
                              const lc_rope3d_s *rope, cudaStream_t stream);
 // Rotate x [batch, ntok, heads, 64] of dtype (token n of x = sequence token
 // n + tok_offset) into out, after an RMSNorm with norm_w when not NULL

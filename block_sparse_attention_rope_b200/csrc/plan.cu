@@ -27,6 +27,7 @@ namespace {
 
 struct PlanGeom {
   int Nc, Nn, Cb, Nb, nq, gc, gn, G, local, stride;
+  int kgc, kgn, KG;  // key groups of 2 blocks (backward)
 };
 
 __device__ __forceinline__ bool attends(int r, int c, const PlanGeom &g) {
@@ -50,6 +51,62 @@ __device__ __forceinline__ void group_members(int gi, const PlanGeom &g, int *fi
   } else {
     *first = g.Cb + 4 * (gi - g.gc);
     *cnt = min(4, g.Nb - 4 * (gi - g.gc));
+  }
+}
+
+// Key group ki covers key blocks first..first+cnt-1 (global block ids).
+__device__ __forceinline__ void kgroup_members(int ki, const PlanGeom &g, int *first, int *cnt) {
+  if (ki < g.kgc) {
+    *first = 2 * ki;
+    *cnt = min(2, g.Cb - 2 * ki);
+  } else {
+    *first = g.Cb + 2 * (ki - g.kgc);
+    *cnt = min(2, g.Nb - 2 * (ki - g.kgc));
+  }
+}
+
+// One warp per key group: size of the union of its members' query lists.
+__global__ void kgroup_count_kernel(PlanGeom g, int *cnt_out) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= g.KG) return;
+  int first, cnt;
+  kgroup_members(warp, g, &first, &cnt);
+  int n = 0;
+  for (int r0 = 0; r0 < g.nq; r0 += 32) {
+    int r = r0 + lane;
+    bool any = false;
+    if (r < g.nq)
+      for (int m = 0; m < cnt; ++m) any |= attends(r, first + m, g);
+    n += __popc(__ballot_sync(0xffffffffu, any));
+  }
+  if (lane == 0) cnt_out[warp] = n;
+}
+
+// One warp per key group: union entries (query block id | member mask << 24).
+__global__ void kgroup_fill_kernel(PlanGeom g, const int *ptr, uint32_t *ent, long long cap,
+                                   int *err) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int lane = threadIdx.x & 31;
+  if (warp >= g.KG) return;
+  int first, cnt;
+  kgroup_members(warp, g, &first, &cnt);
+  long long pos = ptr[warp];
+  long long end = ptr[warp + 1];
+  for (int r0 = 0; r0 < g.nq; r0 += 32) {
+    int r = r0 + lane;
+    uint32_t mask = 0;
+    if (r < g.nq)
+      for (int m = 0; m < cnt; ++m) mask |= attends(r, first + m, g) ? (1u << m) : 0u;
+    unsigned bal = __ballot_sync(0xffffffffu, mask != 0);
+    if (mask) {
+      long long at = pos + __popc(bal & ((1u << lane) - 1u));
+      if (at < end && at < cap)
+        ent[at] = (uint32_t)r | (mask << 24);
+      else
+        atomicOr(err, 64);
+    }
+    pos += __popc(bal);
   }
 }
 
@@ -133,8 +190,8 @@ __device__ void block_exclusive_scan(const int *in, int *out, int n, long long *
 }
 
 __global__ void scan_kernel(PlanGeom g, const int *row_cnt, int *row_ptr, const int *grp_cnt,
-                            int *grp_ptr, const int *col_cnt, int *col_ptr, long long nnz_expect,
-                            int *err) {
+                            int *grp_ptr, const int *col_cnt, int *col_ptr, const int *kgrp_cnt,
+                            int *kgrp_ptr, long long nnz_expect, int *err) {
   __shared__ long long tot;
   block_exclusive_scan(row_cnt, row_ptr, g.nq, &tot);
   __syncthreads();
@@ -147,6 +204,10 @@ __global__ void scan_kernel(PlanGeom g, const int *row_cnt, int *row_ptr, const 
   block_exclusive_scan(col_cnt, col_ptr, g.nq, &tot);
   __syncthreads();
   if (threadIdx.x == 0 && tot != nnz_expect) atomicOr(err, 16);
+  __syncthreads();
+  block_exclusive_scan(kgrp_cnt, kgrp_ptr, g.KG, &tot);
+  __syncthreads();
+  if (threadIdx.x == 0 && tot > nnz_expect) atomicOr(err, 128);
 }
 
 // Transpose of the pattern, one warp per key block c: how many query blocks
@@ -237,12 +298,12 @@ __global__ void group_fill_kernel(PlanGeom g, const int *grp_ptr, uint32_t *ent,
   }
 }
 
-__global__ void order_kernel(PlanGeom g, const int *grp_cnt, int *order) {
+__global__ void order_kernel(int n, const int *grp_cnt, int *order) {
   int gi = blockIdx.x * blockDim.x + threadIdx.x;
-  if (gi >= g.G) return;
+  if (gi >= n) return;
   int mine = grp_cnt[gi];
   int rank = 0;
-  for (int o = 0; o < g.G; ++o) {
+  for (int o = 0; o < n; ++o) {
     int c = grp_cnt[o];
     rank += (c > mine) || (c == mine && o < gi);
   }
@@ -293,6 +354,9 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->gc = (p->Cb + 3) / 4;
   p->gn = (p->Nb + 3) / 4;
   p->G = p->gc + p->gn;
+  p->kgc = (p->Cb + 1) / 2;
+  p->kgn = (p->Nb + 1) / 2;
+  p->KG = p->kgc + p->kgn;
   long long nnz = (long long)p->Cb * p->Cb + (long long)p->Nb * p->Cb;
   for (long long i = 0; i < p->Nb; ++i) nnz += noisy_row_count(i, p->Nb, local, stride);
   p->nnz = nnz;
@@ -306,6 +370,8 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   carve<int>(probe, p->G + 1); carve<int>(probe, p->G); carve<uint32_t>(probe, nnz);
   carve<int>(probe, p->G); carve<unsigned long long>(probe, 2); carve<int>(probe, 1);
   carve<int>(probe, p->nq + 1); carve<int>(probe, nnz); carve<int>(probe, p->nq);
+  carve<int>(probe, p->KG + 1); carve<int>(probe, p->KG); carve<uint32_t>(probe, nnz);
+  carve<int>(probe, p->KG);
   size_t bytes = reinterpret_cast<size_t>(probe);
   cudaError_t e = cudaMallocAsync(&p->mem, bytes, st);
   if (e != cudaSuccess) { delete p; return lc_from_cuda(e); }
@@ -322,23 +388,32 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->col_ptr = carve<int>(q, p->nq + 1);
   p->row_idx = carve<int>(q, nnz);
   p->col_cnt = carve<int>(q, p->nq);
+  p->kgrp_ptr = carve<int>(q, p->KG + 1);
+  p->kgrp_cnt = carve<int>(q, p->KG);
+  p->kgrp_ent = carve<uint32_t>(q, nnz);
+  p->kgrp_order = carve<int>(q, p->KG);
 
-  PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride};
+  PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride,
+             p->kgc, p->kgn, p->KG};
   e = cudaMemsetAsync(p->pairs, 0, 2 * sizeof(unsigned long long), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(p->err, 0, sizeof(int), st);
   const int tpb = 256;
   int row_blocks = (p->nq * 32 + tpb - 1) / tpb;
   int grp_blocks = (p->G * 32 + tpb - 1) / tpb;
+  int kgrp_blocks = (p->KG * 32 + tpb - 1) / tpb;
   if (e == cudaSuccess) {
     row_scan_kernel<<<row_blocks, tpb, 0, st>>>(g, p->row_cnt, p->pairs);
     group_count_kernel<<<grp_blocks, tpb, 0, st>>>(g, p->grp_cnt);
     col_scan_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_cnt);
+    kgroup_count_kernel<<<kgrp_blocks, tpb, 0, st>>>(g, p->kgrp_cnt);
     scan_kernel<<<1, 1024, 0, st>>>(g, p->row_cnt, p->row_ptr, p->grp_cnt, p->grp_ptr,
-                                    p->col_cnt, p->col_ptr, nnz, p->err);
+                                    p->col_cnt, p->col_ptr, p->kgrp_cnt, p->kgrp_ptr, nnz, p->err);
     col_fill_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_ptr, p->row_idx, nnz, p->err);
     row_fill_kernel<<<row_blocks, tpb, 0, st>>>(g, p->row_ptr, p->col_idx, nnz, p->err);
     group_fill_kernel<<<grp_blocks, tpb, 0, st>>>(g, p->grp_ptr, p->grp_ent, nnz, p->err);
-    order_kernel<<<(p->G + 127) / 128, 128, 0, st>>>(g, p->grp_cnt, p->grp_order);
+    order_kernel<<<(p->G + 127) / 128, 128, 0, st>>>(p->G, p->grp_cnt, p->grp_order);
+    kgroup_fill_kernel<<<kgrp_blocks, tpb, 0, st>>>(g, p->kgrp_ptr, p->kgrp_ent, nnz, p->err);
+    order_kernel<<<(p->KG + 127) / 128, 128, 0, st>>>(p->KG, p->kgrp_cnt, p->kgrp_order);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p->ready, cudaEventDisableTiming);

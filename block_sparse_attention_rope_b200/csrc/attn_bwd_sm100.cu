@@ -5,8 +5,9 @@
 // The gradients are the chain rule through the forward's definition (see
 // attn_bwd.cu for the formulas and the pages that motivate them).  Layout of
 // the work, one persistent CTA per SM:
-//   work item = (batch, head, key group of 2 key blocks = 128 keys), handed
-//               out longest query list first; the group walks the sorted
+//   work item = (batch, head, key group of up to 2 key blocks = 128 keys
+//               with alike query lists), handed out longest query list
+//               first; the group walks the sorted
 //               union of the query blocks attending either key block (the
 //               plan's key-group lists), two query blocks (128 queries) per
 //               step.
@@ -60,6 +61,13 @@ constexpr uint32_t kIdescKQ = lcptx::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP
 constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A in TMEM)
 constexpr uint32_t kIdescDQ = lcptx::idesc_bf16_f32(128, 64, 1, 1);   // dQ (A = dS, MN-major)
 constexpr float kLog2e = 1.4426950408889634f;
+// Register split (setmaxnreg, per warpgroup): the elementwise warpgroup holds
+// two 32-column TMEM loads and their results; producer / MMA / RoPE need few;
+// the dQ warpgroup holds one 64-column row.  The host refuses to launch unless
+// the block's registers cover the split.
+constexpr int kRegsEw = 232, kRegsCtl = 96, kRegsDq = 136;
+constexpr int kRegsAtLaunchMin = (128 * (kRegsEw + kRegsCtl + kRegsDq) + kThreads - 1) / kThreads;
+static_assert(128 * (kRegsEw + kRegsCtl + kRegsDq) <= 65536, "register split");
 
 struct __align__(64) BwdParams {
   CUtensorMap tmQ[2], tmK[2], tmV[2], tmG[2];  // [0] condition segment, [1] noisy; G = dO
@@ -67,6 +75,7 @@ struct __align__(64) BwdParams {
   const int *kg_ptr;
   const uint32_t *kg_ent;
   const int *kg_order;
+  const int2 *kg_blk;
   int *work_counter;
   int *status;
   const float *lse;    // [B, heads, N] natural log (the forward's)
@@ -121,7 +130,9 @@ static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
 constexpr int kSchedConsumers = 4 + 1 + 2 + 4;  // elementwise, MMA, RoPE, dQ warps
 
 struct KItem {
-  int b, h, seg, kb0, cnt, krow0, seg_len, len;
+  int b, h, seg, cnt, seg_len, len;
+  int krow0, krow1;  // first row (in the segment) of each key block; past the end if absent
+  __device__ int krow(int half) const { return half ? krow1 : krow0; }
   const uint32_t *ent;
 };
 
@@ -133,12 +144,12 @@ __device__ __forceinline__ KItem decode_kitem(const BwdParams &p, int item) {
   it.b = bh / p.heads;
   it.h = bh - it.b * p.heads;
   it.seg = g < p.kgc ? 0 : 1;
-  const int j = it.seg ? g - p.kgc : g;  // group index within the segment
-  const int nblk = it.seg ? (p.Nn + 63) / 64 : p.Cb;
-  it.kb0 = (it.seg ? p.Cb : 0) + 2 * j;
-  it.cnt = min(2, nblk - 2 * j);
-  it.krow0 = 128 * j;
+  const int2 kb = p.kg_blk[g];  // global key block ids
+  const int base = it.seg ? p.Cb : 0;
   it.seg_len = it.seg ? p.Nn : p.Nc;
+  it.cnt = kb.y >= 0 ? 2 : 1;
+  it.krow0 = 64 * (kb.x - base);
+  it.krow1 = kb.y >= 0 ? 64 * (kb.y - base) : it.seg_len;
   const int lo = p.kg_ptr[g];
   it.len = p.kg_ptr[g + 1] - lo;
   it.ent = p.kg_ent + lo;
@@ -262,6 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   lcptx::tc_fence_after();
   const uint32_t tmem = misc[0];
 
+  if (warp >= kWarpProducer && warp < kWarpDq) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
   if (warp == kWarpProducer) {
     // ======================= TMA producer (one thread) =======================
     if (lane == 0) {
@@ -287,9 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t dv = lcptx::smem_addr(sV + kb * kTileBytes);
           // rows past the segment end (a missing second block) read as zeros
           lcptx::tma_load_4d(dk, &p.tmK[it.seg], bar, 0, it.h, it.krow0, it.b);
-          lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[it.seg], bar, 0, it.h, it.krow0 + 64, it.b);
+          lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[it.seg], bar, 0, it.h, it.krow1, it.b);
           lcptx::tma_load_4d(dv, &p.tmV[it.seg], bar, 0, it.h, it.krow0, it.b);
-          lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[it.seg], bar, 0, it.h, it.krow0 + 64, it.b);
+          lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[it.seg], bar, 0, it.h, it.krow1, it.b);
           kv_valid |= 1u << kb;
           kv_par = (kv_par & ~(1u << kb)) | (kph << kb);
         }
@@ -423,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       drain_wait(ctx.bar(B_DRAIN), 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp == kWarpRope || warp == kWarpRope + 1) {
+  } else {
     // ======================= RoPE warps: K per item, Q + lse / D per step ====
     const int rt = tid - kWarpRope * 32;
     const float *q_nw = p.q_norm_w ? s_normw : nullptr;
@@ -442,8 +455,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       if (!ok) break;
       const int seg_tok = it.seg ? p.Nc : 0;
       for (int r = rt; r < 128; r += kRopeThreads)
-        if (it.krow0 + r < it.seg_len && (r >> 6) < it.cnt)
-          rope_row(sK + kb * kTileBytes, r, seg_tok + it.krow0 + r, tab, p, k_nw);
+        if ((r >> 6) < it.cnt && it.krow(r >> 6) + (r & 63) < it.seg_len)
+          rope_row(sK + kb * kTileBytes, r, seg_tok + it.krow(r >> 6) + (r & 63), tab, p, k_nw);
       lcptx::fence_proxy_async_smem();
       lcptx::mbar_arrive(ctx.bar(B_KV_READY + kb));
       const int nsteps = (it.len + 1) >> 1;
@@ -475,7 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       if (!ok) break;
       ++item_it;
     }
+  }
   } else if (warp >= kWarpDq) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDq));
     // ======================= dQ warps: TMEM dQ -> fp32 atomics ================
     const int qrow = tid - kWarpDq * 32;  // TMEM lane == query row of the step
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -508,16 +523,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           qblock(p, __ldg(it.ent + e), qs, qr, qn);
           if ((qrow & 63) < qn) {
             const long long tok = (qs ? p.Nc : 0) + qr + (qrow & 63);
-            float4 *dst = reinterpret_cast<float4 *>(
-                p.dq_acc + (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM);
+            float *dst = p.dq_acc + (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              atomicAdd(dst + c, make_float4(__uint_as_float(a0[4 * c]), __uint_as_float(a0[4 * c + 1]),
-                                             __uint_as_float(a0[4 * c + 2]), __uint_as_float(a0[4 * c + 3])));
+              lcptx::red_add_v4_f32(dst + 4 * c, __uint_as_float(a0[4 * c]), __uint_as_float(a0[4 * c + 1]),
+                                    __uint_as_float(a0[4 * c + 2]), __uint_as_float(a0[4 * c + 3]));
 #pragma unroll
             for (int c = 0; c < 8; ++c)
-              atomicAdd(dst + 8 + c, make_float4(__uint_as_float(a1[4 * c]), __uint_as_float(a1[4 * c + 1]),
-                                                 __uint_as_float(a1[4 * c + 2]), __uint_as_float(a1[4 * c + 3])));
+              lcptx::red_add_v4_f32(dst + 32 + 4 * c, __uint_as_float(a1[4 * c]),
+                                    __uint_as_float(a1[4 * c + 1]), __uint_as_float(a1[4 * c + 2]),
+                                    __uint_as_float(a1[4 * c + 3]));
           }
         }
       }
@@ -525,6 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       ++item_it;
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
     // ======================= elementwise warps 0-3 (thread = key row) ========
     const int kr = tid;  // TMEM lane == key row of the group
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
@@ -539,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
       const KItem it = decode_kitem(p, item);
-      const bool key_valid = (kr >> 6) < it.cnt && it.krow0 + kr < it.seg_len;
+      const bool key_valid = (kr >> 6) < it.cnt && it.krow(kr >> 6) + (kr & 63) < it.seg_len;
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
       for (int t = 0; t < nsteps; ++t, ++q_it) {
@@ -610,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       ok = wait_warp(ctx, ctx.bar(B_ACC), item_it & 1);
       if (!ok) break;
       lcptx::tc_fence_after();
-      const int tok = (it.seg ? p.Nc : 0) + it.krow0 + kr;
+      const int tok = (it.seg ? p.Nc : 0) + it.krow(kr >> 6) + (kr & 63);
       const long long off = (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM;
       float dkv[64];
       {
@@ -711,6 +727,7 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   prm.kg_ptr = plan->kgrp_ptr;
   prm.kg_ent = plan->kgrp_ent;
   prm.kg_order = plan->kgrp_order;
+  prm.kg_blk = plan->kgrp_blk;
   prm.lse = lse;
   prm.dk = static_cast<__nv_bfloat16 *>(dk);
   prm.dv = static_cast<__nv_bfloat16 *>(dv);
@@ -741,6 +758,13 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   int dev = 0, n_sm = 0;
   LC_CUDA_TRY(cudaGetDevice(&dev));
   LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  static int regs_at_launch = -1;
+  if (regs_at_launch < 0) {
+    cudaFuncAttributes fa;
+    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, bsa_bwd_sm100_kernel));
+    regs_at_launch = fa.numRegs;
+  }
+  if (regs_at_launch < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;  // the split could never complete
   LC_CUDA_TRY(cudaFuncSetAttribute(bsa_bwd_sm100_kernel,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));

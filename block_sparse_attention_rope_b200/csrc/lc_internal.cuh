@@ -41,8 +41,9 @@ struct lc_bsa_plan_s {
   int *col_ptr;             // [nq + 1]  transpose (CSC): query blocks attending key block c
   int *row_idx;             // [nnz]     ascending
   int *col_cnt;             // [nq]      planner work array
-  // Backward work lists: key groups of 2 consecutive key blocks of one
-  // segment (kgc condition groups, then kgn noisy ones), each with the sorted
+  // Backward work lists: key groups of up to 2 key blocks of one segment
+  // with alike query lists (kgc condition groups, then kgn noisy ones; see
+  // kgroup_members in plan.cu), each with the sorted
   // union of the query blocks attending either member (entry = query block id
   // | member mask << 24), and the groups ranked longest list first.
   int kgc, kgn, KG;
@@ -50,6 +51,7 @@ struct lc_bsa_plan_s {
   int *kgrp_cnt;            // [KG]
   uint32_t *kgrp_ent;       // [nnz]     (upper bound of the union lists)
   int *kgrp_order;          // [KG]
+  int2 *kgrp_blk;           // [KG]      the group's key blocks (second -1 if none)
   unsigned long long *pairs;  // [2] attended token pairs: all rows, noisy rows
   int *err;                 // [1] planner consistency flag
   long long pairs_host[2];

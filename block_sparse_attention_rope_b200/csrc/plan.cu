@@ -54,15 +54,50 @@ __device__ __forceinline__ void group_members(int gi, const PlanGeom &g, int *fi
   }
 }
 
-// Key group ki covers key blocks first..first+cnt-1 (global block ids).
-__device__ __forceinline__ void kgroup_members(int ki, const PlanGeom &g, int *first, int *cnt) {
+// Key group ki: up to two key blocks (global block ids) of one segment whose
+// query lists are alike, so that the backward pass computes few masked
+// pairs.  Condition blocks pair in order (all are attended by every query
+// block).  In the noisy segment with strided globals, the global blocks
+// (j % stride == 0, attended by every noisy query block) pair with each
+// other, and the local-only blocks pair in order; otherwise blocks pair in
+// order.
+__device__ __forceinline__ void kgroup_members(int ki, const PlanGeom &g, int *blk, int *cnt) {
   if (ki < g.kgc) {
-    *first = 2 * ki;
+    blk[0] = 2 * ki;
     *cnt = min(2, g.Cb - 2 * ki);
-  } else {
-    *first = g.Cb + 2 * (ki - g.kgc);
-    *cnt = min(2, g.Nb - 2 * (ki - g.kgc));
+    blk[1] = blk[0] + 1;
+    return;
   }
+  const int gi = ki - g.kgc;
+  if (g.stride <= 1) {
+    blk[0] = g.Cb + 2 * gi;
+    *cnt = min(2, g.Nb - 2 * gi);
+    blk[1] = blk[0] + 1;
+    return;
+  }
+  const int s = g.stride;
+  const int n_glob = (g.Nb + s - 1) / s;
+  const int kg_glob = (n_glob + 1) / 2;
+  if (gi < kg_glob) {
+    blk[0] = g.Cb + (2 * gi) * s;
+    *cnt = min(2, n_glob - 2 * gi);
+    blk[1] = g.Cb + (2 * gi + 1) * s;
+  } else {
+    const int li = 2 * (gi - kg_glob);  // index among the non-multiples of s
+    const int n_loc = g.Nb - n_glob;
+    *cnt = min(2, n_loc - li);
+    blk[0] = g.Cb + (li / (s - 1)) * s + li % (s - 1) + 1;
+    blk[1] = g.Cb + ((li + 1) / (s - 1)) * s + (li + 1) % (s - 1) + 1;
+  }
+}
+
+// Key blocks of every key group, for the backward kernel: (first, second or -1).
+__global__ void kgroup_blocks_kernel(PlanGeom g, int2 *kg_blk) {
+  const int ki = blockIdx.x * blockDim.x + threadIdx.x;
+  if (ki >= g.KG) return;
+  int blk[2], cnt;
+  kgroup_members(ki, g, blk, &cnt);
+  kg_blk[ki] = make_int2(blk[0], cnt > 1 ? blk[1] : -1);
 }
 
 // One warp per key group: size of the union of its members' query lists.
@@ -70,14 +105,14 @@ __global__ void kgroup_count_kernel(PlanGeom g, int *cnt_out) {
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (warp >= g.KG) return;
-  int first, cnt;
-  kgroup_members(warp, g, &first, &cnt);
+  int blk[2], cnt;
+  kgroup_members(warp, g, blk, &cnt);
   int n = 0;
   for (int r0 = 0; r0 < g.nq; r0 += 32) {
     int r = r0 + lane;
     bool any = false;
     if (r < g.nq)
-      for (int m = 0; m < cnt; ++m) any |= attends(r, first + m, g);
+      for (int m = 0; m < cnt; ++m) any |= attends(r, blk[m], g);
     n += __popc(__ballot_sync(0xffffffffu, any));
   }
   if (lane == 0) cnt_out[warp] = n;
@@ -89,15 +124,15 @@ __global__ void kgroup_fill_kernel(PlanGeom g, const int *ptr, uint32_t *ent, lo
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   int lane = threadIdx.x & 31;
   if (warp >= g.KG) return;
-  int first, cnt;
-  kgroup_members(warp, g, &first, &cnt);
+  int blk[2], cnt;
+  kgroup_members(warp, g, blk, &cnt);
   long long pos = ptr[warp];
   long long end = ptr[warp + 1];
   for (int r0 = 0; r0 < g.nq; r0 += 32) {
     int r = r0 + lane;
     uint32_t mask = 0;
     if (r < g.nq)
-      for (int m = 0; m < cnt; ++m) mask |= attends(r, first + m, g) ? (1u << m) : 0u;
+      for (int m = 0; m < cnt; ++m) mask |= attends(r, blk[m], g) ? (1u << m) : 0u;
     unsigned bal = __ballot_sync(0xffffffffu, mask != 0);
     if (mask) {
       long long at = pos + __popc(bal & ((1u << lane) - 1u));
@@ -355,7 +390,12 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->gn = (p->Nb + 3) / 4;
   p->G = p->gc + p->gn;
   p->kgc = (p->Cb + 1) / 2;
-  p->kgn = (p->Nb + 1) / 2;
+  if (stride > 1) {  // global blocks pair with each other, the others in order
+    const int n_glob = (p->Nb + stride - 1) / stride;
+    p->kgn = (n_glob + 1) / 2 + (p->Nb - n_glob + 1) / 2;
+  } else {
+    p->kgn = (p->Nb + 1) / 2;
+  }
   p->KG = p->kgc + p->kgn;
   long long nnz = (long long)p->Cb * p->Cb + (long long)p->Nb * p->Cb;
   for (long long i = 0; i < p->Nb; ++i) nnz += noisy_row_count(i, p->Nb, local, stride);
@@ -371,7 +411,7 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   carve<int>(probe, p->G); carve<unsigned long long>(probe, 2); carve<int>(probe, 1);
   carve<int>(probe, p->nq + 1); carve<int>(probe, nnz); carve<int>(probe, p->nq);
   carve<int>(probe, p->KG + 1); carve<int>(probe, p->KG); carve<uint32_t>(probe, nnz);
-  carve<int>(probe, p->KG);
+  carve<int>(probe, p->KG); carve<int2>(probe, p->KG);
   size_t bytes = reinterpret_cast<size_t>(probe);
   cudaError_t e = cudaMallocAsync(&p->mem, bytes, st);
   if (e != cudaSuccess) { delete p; return lc_from_cuda(e); }
@@ -392,6 +432,7 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->kgrp_cnt = carve<int>(q, p->KG);
   p->kgrp_ent = carve<uint32_t>(q, nnz);
   p->kgrp_order = carve<int>(q, p->KG);
+  p->kgrp_blk = carve<int2>(q, p->KG);
 
   PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride,
              p->kgc, p->kgn, p->KG};
@@ -406,6 +447,7 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
     group_count_kernel<<<grp_blocks, tpb, 0, st>>>(g, p->grp_cnt);
     col_scan_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_cnt);
     kgroup_count_kernel<<<kgrp_blocks, tpb, 0, st>>>(g, p->kgrp_cnt);
+    kgroup_blocks_kernel<<<(p->KG + 127) / 128, 128, 0, st>>>(g, p->kgrp_blk);
     scan_kernel<<<1, 1024, 0, st>>>(g, p->row_cnt, p->row_ptr, p->grp_cnt, p->grp_ptr,
                                     p->col_cnt, p->col_ptr, p->kgrp_cnt, p->kgrp_ptr, nnz, p->err);
     col_fill_kernel<<<row_blocks, tpb, 0, st>>>(g, p->col_ptr, p->row_idx, nnz, p->err);

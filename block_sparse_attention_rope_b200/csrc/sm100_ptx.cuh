@@ -209,6 +209,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
       : "memory");
 }
 
+// Fire-and-forget add of four consecutive floats in global memory (16-byte
+// aligned): a reduction, no value comes back.
+__device__ __forceinline__ void red_add_v4_f32(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand tile
 // (rows of 128 bytes, 8-row atoms of 1024 bytes, tile base 1024-aligned).
 //   bits  0-13: start address >> 4     bits 16-29: leading byte offset >> 4

@@ -14,17 +14,18 @@
 //   per step, with keys as TMEM lanes (M = 128):
 //     S^T  = K' Q'^T        dP^T = V dO^T          (tcgen05, into TMEM)
 //     P^T  = exp(scale S^T - lse),  dS^T = P^T (dP^T - D) scale
-//                           (warps 0-3, one key row per thread; P^T and dS^T
-//                            written back as bf16 over the consumed columns,
+//                           (warps 0-7, one key row and query half per thread; P^T, dS^T
+//                            written back as bf16 over each half's consumed
+//                            columns,
 //                            dS^T also to shared memory for dQ)
 //     dV  += P^T dO         dK' += dS^T Q'         (A from TMEM)
 //     dQ'  = dS K'          (A = dS from shared memory, MN-major; queries as
 //                            TMEM lanes), added to the fp32 buffer by warps
-//                            8-11 with vector atomics
+//                            12-15 with vector reductions
 //   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
-//   warp 4: TMA producer (K, V per item, double-buffered; Q, dO per step,
-//   2 stages); warp 5: MMA issuer; warps 6-7: rotate K and Q tiles in shared
-//   memory and stage lse / D per step.
+//   warp 8: TMA producer (K, V per item, double-buffered; Q, dO per step,
+//   2 stages); warp 9: MMA issuer; warps 10-11: rotate K and Q tiles in
+//   shared memory and stage lse / D per step.
 //   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448).
 // Every mbarrier wait is bounded; on expiry the CTA stops, drains and frees
 // TMEM, and LC_DEVSTAT_TIMEOUT is set.
@@ -46,12 +47,13 @@ using lcsm100::rope_row;
 using lcsm100::wait_bar;
 using lcsm100::wait_warp;
 
-constexpr int kThreads = 384;
-constexpr int kWarpProducer = 4;
-constexpr int kWarpMma = 5;
-constexpr int kWarpRope = 6;  // and 7
+constexpr int kThreads = 512;
+constexpr int kEwWarps = 8;       // 0-7: elementwise, two warps per key row (query halves)
+constexpr int kWarpProducer = 8;
+constexpr int kWarpMma = 9;
+constexpr int kWarpRope = 10;     // and 11
 constexpr int kRopeThreads = 64;
-constexpr int kWarpDq = 8;    // 8-11
+constexpr int kWarpDq = 12;       // 12-15
 constexpr int kQStages = 2;
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kBoxBytes = 64 * 128;
@@ -61,13 +63,14 @@ constexpr uint32_t kIdescKQ = lcptx::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP
 constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A in TMEM)
 constexpr uint32_t kIdescDQ = lcptx::idesc_bf16_f32(128, 64, 1, 1);   // dQ (A = dS, MN-major)
 constexpr float kLog2e = 1.4426950408889634f;
-// Register split (setmaxnreg, per warpgroup): the elementwise warpgroup holds
-// two 32-column TMEM loads and their results; producer / MMA / RoPE need few;
-// the dQ warpgroup holds one 64-column row.  The host refuses to launch unless
-// the block's registers cover the split.
-constexpr int kRegsEw = 232, kRegsCtl = 96, kRegsDq = 136;
-constexpr int kRegsAtLaunchMin = (128 * (kRegsEw + kRegsCtl + kRegsDq) + kThreads - 1) / kThreads;
-static_assert(128 * (kRegsEw + kRegsCtl + kRegsDq) <= 65536, "register split");
+// Register split (setmaxnreg, per warpgroup): the two elementwise warpgroups
+// hold two 32-column TMEM loads and their results; producer / MMA / RoPE need
+// few; the dQ warpgroup holds one 64-column row.  The host refuses to launch
+// unless the block's registers cover the split.
+constexpr int kRegsEw = 152, kRegsCtl = 80, kRegsDq = 96;
+constexpr int kRegsTotal = 256 * kRegsEw + 128 * (kRegsCtl + kRegsDq);
+constexpr int kRegsAtLaunchMin = (kRegsTotal + kThreads - 1) / kThreads;
+static_assert(kRegsTotal <= 65536, "register split");
 
 struct __align__(64) BwdParams {
   CUtensorMap tmQ[2], tmK[2], tmV[2], tmG[2];  // [0] condition segment, [1] noisy; G = dO
@@ -117,17 +120,17 @@ enum {
   B_QG_READY = B_QG_FULL + kQStages,   // Q rotated, lse / D staged
   B_QG_EMPTY = B_QG_READY + kQStages,  // step's MMAs done with Q, dO
   B_SDP = B_QG_EMPTY + kQStages,    // S^T and dP^T in TMEM
-  B_PDS = B_SDP + 1,                // P^T, dS^T written (4 warps)
+  B_PDS = B_SDP + 1,                // P^T, dS^T written (8 warps)
   B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete
   B_DQ_FULL = B_STEP + 1,           // dQ of a step in TMEM
   B_DQ_EMPTY = B_DQ_FULL + 1,       // dQ read out (4 warps)
   B_ACC = B_DQ_EMPTY + 1,           // item's dK, dV complete
-  B_EPI_FREE = B_ACC + 1,           // dK, dV read out (4 warps)
+  B_EPI_FREE = B_ACC + 1,           // dK, dV read out (8 warps)
   B_DRAIN = B_EPI_FREE + 1,
   B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
-constexpr int kSchedConsumers = 4 + 1 + 2 + 4;  // elementwise, MMA, RoPE, dQ warps
+constexpr int kSchedConsumers = kEwWarps + 1 + 2 + 4;  // elementwise, MMA, RoPE, dQ warps
 
 struct KItem {
   int b, h, seg, cnt, seg_len, len;
@@ -205,6 +208,9 @@ __device__ __forceinline__ void pair_angle(const BwdParams &a, const float *tab,
   }
 }
 
+// kNorm: RMSNorm weights in use (the plain path is a separate instantiation
+// that carries none of that code).
+template <bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -247,12 +253,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       lcptx::mbar_init(ctx.bar(B_QG_EMPTY + s), 1);
     }
     lcptx::mbar_init(ctx.bar(B_SDP), 1);
-    lcptx::mbar_init(ctx.bar(B_PDS), 4);
+    lcptx::mbar_init(ctx.bar(B_PDS), kEwWarps);
     lcptx::mbar_init(ctx.bar(B_STEP), 1);
     lcptx::mbar_init(ctx.bar(B_DQ_FULL), 1);
     lcptx::mbar_init(ctx.bar(B_DQ_EMPTY), 4);
     lcptx::mbar_init(ctx.bar(B_ACC), 1);
-    lcptx::mbar_init(ctx.bar(B_EPI_FREE), 4);
+    lcptx::mbar_init(ctx.bar(B_EPI_FREE), kEwWarps);
     lcptx::mbar_init(ctx.bar(B_DRAIN), 1);
     lcptx::fence_mbar_init();
   }
@@ -403,14 +409,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             if (!ok) break;
           }
           lcptx::tc_fence_after();
+          // P^T / dS^T of query block h sit in columns [64 h, 64 h + 32) of S^T / dP^T
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ts(tmem + kColDV, tmem + kColST + 8 * kk, desc(g_mn + s * kTileLo + 128 * kk),
-                          kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+            lcptx::mma_ts(tmem + kColDV, tmem + kColST + 64 * (kk >> 2) + 8 * (kk & 3),
+                          desc(g_mn + s * kTileLo + 128 * kk), kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ts(tmem + kColDK, tmem + kColDPT + 8 * kk, desc(q_mn + s * kTileLo + 128 * kk),
-                          kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+            lcptx::mma_ts(tmem + kColDK, tmem + kColDPT + 64 * (kk >> 2) + 8 * (kk & 3),
+                          desc(q_mn + s * kTileLo + 128 * kk), kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
           if (k_step > 0) {  // the dQ warps have read the previous step's dQ
             ok = wait_bar(ctx, ctx.bar(B_DQ_EMPTY), (k_step - 1) & 1);
             if (!ok) break;
@@ -439,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   } else {
     // ======================= RoPE warps: K per item, Q + lse / D per step ====
     const int rt = tid - kWarpRope * 32;
-    const float *q_nw = p.q_norm_w ? s_normw : nullptr;
-    const float *k_nw = p.k_norm_w ? s_normw + 64 : nullptr;
+    const float *q_nw = (kNorm && p.q_norm_w) ? s_normw : nullptr;
+    const float *k_nw = (kNorm && p.k_norm_w) ? s_normw + 64 : nullptr;
     uint32_t item_it = 0, q_it = 0;
     for (;;) {
       const int slot = item_it & 1;
@@ -464,23 +471,34 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const float *del_bh = p.delta + ((long long)it.b * p.heads + it.h) * N;
       for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
         const int s = q_it % kQStages;
-        ok = wait_warp(ctx, ctx.bar(B_QG_FULL + s), (q_it / kQStages) & 1);
-        if (!ok) break;
-        for (int r = rt; r < 128; r += kRopeThreads) {
-          const int e = 2 * t + (r >> 6);
-          float l2 = 0.f, dl = 0.f;
+        // This thread's two query rows (rt of each query block): token, lse and
+        // D first, so that their global loads overlap the wait and the rotation.
+        int tokr[2];
+        float l2r[2], dlr[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          tokr[i] = -1;
+          l2r[i] = dlr[i] = 0.f;
+          const int e = 2 * t + i;
           if (e < it.len) {
             int qs, qr, qn;
             qblock(p, __ldg(it.ent + e), qs, qr, qn);
-            if ((r & 63) < qn) {
-              const int tok = (qs ? p.Nc : 0) + qr + (r & 63);
-              rope_row(sQ + s * kTileBytes, r, tok, tab, p, q_nw);
-              l2 = __ldg(lse_bh + tok) * kLog2e;
-              dl = __ldg(del_bh + tok);
+            if (rt < qn) {
+              tokr[i] = (qs ? p.Nc : 0) + qr + rt;
+              l2r[i] = __ldg(lse_bh + tokr[i]) * kLog2e;
+              dlr[i] = __ldg(del_bh + tokr[i]);
             }
           }
-          sLse[s * 128 + r] = l2;
-          sDel[s * 128 + r] = dl;
+        }
+        ok = wait_warp(ctx, ctx.bar(B_QG_FULL + s), (q_it / kQStages) & 1);
+        if (!ok) break;
+#pragma unroll 1
+        for (int i = 0; i < 2; ++i)
+          if (tokr[i] >= 0) rope_row(sQ + s * kTileBytes, rt + 64 * i, tokr[i], tab, p, q_nw);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          sLse[s * 128 + rt + 64 * i] = l2r[i];
+          sDel[s * 128 + rt + 64 * i] = dlr[i];
         }
         lcptx::fence_proxy_async_smem();
         lcptx::mbar_arrive(ctx.bar(B_QG_READY + s));
@@ -541,8 +559,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
-    // ======================= elementwise warps 0-3 (thread = key row) ========
-    const int kr = tid;  // TMEM lane == key row of the group
+    // ======================= elementwise warps 0-7 ===========================
+    // Thread = key row kr (TMEM lane); warps 0-3 take the step's first query
+    // block (columns 0-63), warps 4-7 the second: two warps per sub-partition
+    // keep the exp unit busy.
+    const int kr = tid & 127;
+    const int half = warp >> 2;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tST = tmem + lane_base + kColST, tDPT = tmem + lane_base + kColDPT;
     const float sl2 = p.scale * kLog2e;
@@ -560,19 +582,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       bool ok = true;
       for (int t = 0; t < nsteps; ++t, ++q_it) {
         const int s = q_it % kQStages;
-        // attended query tokens of the step's two query blocks, for this key row
-        int lim[2];
-#pragma unroll
-        for (int hq = 0; hq < 2; ++hq) {
-          lim[hq] = 0;
-          const int e = 2 * t + hq;
-          if (key_valid && e < it.len) {
-            const uint32_t ent = __ldg(it.ent + e);
-            if ((ent >> (24 + (kr >> 6))) & 1u) {
-              int qs, qr, qn;
-              qblock(p, ent, qs, qr, qn);
-              lim[hq] = qn;
-            }
+        // attended query tokens of this warp's query block, for this key row
+        int lim = 0;
+        const int e = 2 * t + half;
+        if (key_valid && e < it.len) {
+          const uint32_t ent = __ldg(it.ent + e);
+          if ((ent >> (24 + (kr >> 6))) & 1u) {
+            int qs, qr, qn;
+            qblock(p, ent, qs, qr, qn);
+            lim = qn;
           }
         }
         // the staged lse / D of this step (written by the RoPE warps), then S^T, dP^T
@@ -582,22 +600,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         sdp_ph ^= 1;
         lcptx::tc_fence_after();
         const float *l2 = sLse + s * 128, *dl = sDel + s * 128;
+        uint8_t *tile = sDS + half * kTileBytes;  // dS^T, this query block's MN-major chunk
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {  // 32 queries at a time
-          uint32_t sr[32], dr[32];
-          lcptx::tmem_ld32(tST + 32 * c, sr);
-          lcptx::tmem_ld32(tDPT + 32 * c, dr);
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {  // 16 queries at a time
+          uint32_t sr[16], dr[16];
+          lcptx::tmem_ld16(tST + 16 * c, sr);
+          lcptx::tmem_ld16(tDPT + 16 * c, dr);
           lcptx::tmem_wait_ld();
-          const int hq = c >> 1;
-          const int jb = (c & 1) * 32;  // first query of the chunk within its block
-          uint32_t pp[16], dd[16];
+          const int jb = (c & 3) * 16;  // first query of the chunk within its block
+          uint32_t pp[8], dd[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
+          for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int j = 32 * c + 2 * i + u;
-              const bool on = jb + 2 * i + u < lim[hq];
+              const int j = 16 * c + 2 * i + u;
+              const bool on = jb + 2 * i + u < lim;
               const float pe = on ? ex2(__uint_as_float(sr[2 * i + u]) * sl2 - l2[j]) : 0.f;
               pv[u] = pe;
               dv2[u] = pe * (__uint_as_float(dr[2 * i + u]) - dl[j]) * p.scale;
@@ -605,14 +623,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             pp[i] = pack_bf16(pv[0], pv[1]);
             dd[i] = pack_bf16(dv2[0], dv2[1]);
           }
-          lcptx::tmem_st16(tST + 16 * c, pp);
-          lcptx::tmem_st16(tDPT + 16 * c, dd);
-          // dS^T row kr, queries 32c..32c+31, into the MN-major dQ operand:
-          // tile hq (queries 64 hq .. 64 hq + 63), 16-byte chunks (c & 1) * 4 + i.
-          uint8_t *tile = sDS + hq * kTileBytes;
+          // P^T / dS^T of queries 16c..16c+15 go to columns 64 half + 8 (c & 3):
+          // inside this warp's own 64 columns, and already read
+          lcptx::tmem_st8(tST + 64 * half + 8 * (c & 3), pp);
+          lcptx::tmem_st8(tDPT + 64 * half + 8 * (c & 3), dd);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<uint4 *>(tile + swz(kr, (c & 1) * 4 + i)) =
+          for (int i = 0; i < 2; ++i)
+            *reinterpret_cast<uint4 *>(tile + swz(kr, (c & 3) * 2 + i)) =
                 make_uint4(dd[4 * i], dd[4 * i + 1], dd[4 * i + 2], dd[4 * i + 3]);
         }
         lcptx::fence_proxy_async_smem();
@@ -622,77 +639,78 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));
       }
       if (!ok) break;
-      // ---- epilogue: dK = R^T dK' (and the RMSNorm transpose), dV; stored bf16
+      // ---- epilogue: warps 0-3 store dV; warps 4-7 store dK = R^T dK' (and
+      // the RMSNorm transpose).  bf16 rows straight to global memory.
       ok = wait_warp(ctx, ctx.bar(B_ACC), item_it & 1);
       if (!ok) break;
       lcptx::tc_fence_after();
       const int tok = (it.seg ? p.Nc : 0) + it.krow(kr >> 6) + (kr & 63);
       const long long off = (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM;
-      float dkv[64];
+      float acc[64];
       {
         uint32_t a[32], b2[32];
-        lcptx::tmem_ld32(tmem + lane_base + kColDV, a);
-        lcptx::tmem_ld32(tmem + lane_base + kColDV + 32, b2);
-        lcptx::tmem_wait_ld();
-        if (key_valid) {
-          uint4 *gv = reinterpret_cast<uint4 *>(p.dv + off);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            gv[c] = make_uint4(pack_bf16(__uint_as_float(a[8 * c]), __uint_as_float(a[8 * c + 1])),
-                               pack_bf16(__uint_as_float(a[8 * c + 2]), __uint_as_float(a[8 * c + 3])),
-                               pack_bf16(__uint_as_float(a[8 * c + 4]), __uint_as_float(a[8 * c + 5])),
-                               pack_bf16(__uint_as_float(a[8 * c + 6]), __uint_as_float(a[8 * c + 7])));
-            gv[4 + c] = make_uint4(pack_bf16(__uint_as_float(b2[8 * c]), __uint_as_float(b2[8 * c + 1])),
-                                   pack_bf16(__uint_as_float(b2[8 * c + 2]), __uint_as_float(b2[8 * c + 3])),
-                                   pack_bf16(__uint_as_float(b2[8 * c + 4]), __uint_as_float(b2[8 * c + 5])),
-                                   pack_bf16(__uint_as_float(b2[8 * c + 6]), __uint_as_float(b2[8 * c + 7])));
-          }
-        }
-        lcptx::tmem_ld32(tmem + lane_base + kColDK, a);
-        lcptx::tmem_ld32(tmem + lane_base + kColDK + 32, b2);
+        const uint32_t col = half ? kColDK : kColDV;
+        lcptx::tmem_ld32(tmem + lane_base + col, a);
+        lcptx::tmem_ld32(tmem + lane_base + col + 32, b2);
         lcptx::tmem_wait_ld();
 #pragma unroll
         for (int d = 0; d < 32; ++d) {
-          dkv[d] = __uint_as_float(a[d]);
-          dkv[32 + d] = __uint_as_float(b2[d]);
+          acc[d] = __uint_as_float(a[d]);
+          acc[32 + d] = __uint_as_float(b2[d]);
         }
       }
       lcptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_EPI_FREE));
       if (key_valid) {
+        if (half) {
 #pragma unroll
-        for (int q2 = 0; q2 < 32; ++q2) {  // R^T: turn each pair back
-          float c, sn;
-          pair_angle(p, tab, tok, q2, c, sn);
-          const float u = dkv[2 * q2], w = dkv[2 * q2 + 1];
-          dkv[2 * q2] = fmaf(u, c, w * sn);
-          dkv[2 * q2 + 1] = fmaf(w, c, -u * sn);
-        }
-        if (p.k_norm_w) {  // y = x inv w:  dx = inv (w g) - x inv^3 / 64 * sum(g w x)
-          float c8[8];
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            float x8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x8[e] = __bfloat162float(p.k_raw[off + 8 * ch + e]);
-            c8[ch] = lc_sumsq8(x8);
+          for (int q2 = 0; q2 < 32; ++q2) {  // R^T: turn each pair back
+            float c, sn;
+            pair_angle(p, tab, tok, q2, c, sn);
+            const float u = acc[2 * q2], w = acc[2 * q2 + 1];
+            acc[2 * q2] = fmaf(u, c, w * sn);
+            acc[2 * q2 + 1] = fmaf(w, c, -u * sn);
           }
-          const float inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
-          float dot = 0.f;
+          if (kNorm && p.k_norm_w) {  // y = x inv w: dx = inv (w g) - x inv^3 / 64 sum(g w x)
+            const uint4 *xr = reinterpret_cast<const uint4 *>(p.k_raw + off);  // 8 bf16 per load
+            float c8[8], dot = 0.f;
 #pragma unroll
-          for (int d = 0; d < 64; ++d)
-            dot = fmaf(dkv[d] * s_normw[64 + d], __bfloat162float(p.k_raw[off + d]), dot);
-          const float k3 = inv * inv * inv * (1.f / 64.f) * dot;
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint4 raw = __ldg(xr + ch);
+              const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+              float x8[8];
 #pragma unroll
-          for (int d = 0; d < 64; ++d)
-            dkv[d] = inv * s_normw[64 + d] * dkv[d] - __bfloat162float(p.k_raw[off + d]) * k3;
+              for (int e2 = 0; e2 < 4; ++e2) {
+                x8[2 * e2] = __uint_as_float(wd[e2] << 16);
+                x8[2 * e2 + 1] = __uint_as_float(wd[e2] & 0xFFFF0000u);
+              }
+              c8[ch] = lc_sumsq8(x8);
+#pragma unroll
+              for (int e2 = 0; e2 < 8; ++e2)
+                dot = fmaf(acc[8 * ch + e2] * s_normw[64 + 8 * ch + e2], x8[e2], dot);
+            }
+            const float inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
+            const float k3 = inv * inv * inv * (1.f / 64.f) * dot;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+              const uint4 raw = __ldg(xr + ch);
+              const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+              for (int e2 = 0; e2 < 4; ++e2) {
+                const int d = 8 * ch + 2 * e2;
+                acc[d] = inv * s_normw[64 + d] * acc[d] - __uint_as_float(wd[e2] << 16) * k3;
+                acc[d + 1] = inv * s_normw[64 + d + 1] * acc[d + 1] -
+                             __uint_as_float(wd[e2] & 0xFFFF0000u) * k3;
+              }
+            }
+          }
         }
-        uint4 *gk = reinterpret_cast<uint4 *>(p.dk + off);
+        uint4 *dst = reinterpret_cast<uint4 *>((half ? p.dk : p.dv) + off);
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          gk[c] = make_uint4(pack_bf16(dkv[8 * c], dkv[8 * c + 1]), pack_bf16(dkv[8 * c + 2], dkv[8 * c + 3]),
-                             pack_bf16(dkv[8 * c + 4], dkv[8 * c + 5]), pack_bf16(dkv[8 * c + 6], dkv[8 * c + 7]));
+          dst[c] = make_uint4(pack_bf16(acc[8 * c], acc[8 * c + 1]), pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
+                              pack_bf16(acc[8 * c + 4], acc[8 * c + 5]), pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
       }
       ++item_it;
     }
@@ -758,15 +776,18 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   int dev = 0, n_sm = 0;
   LC_CUDA_TRY(cudaGetDevice(&dev));
   LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
-  static int regs_at_launch = -1;
-  if (regs_at_launch < 0) {
+  const bool with_norm = norm.q_w || norm.k_w;
+  void (*const kern)(const BwdParams) = with_norm ? bsa_bwd_sm100_kernel<true>
+                                                  : bsa_bwd_sm100_kernel<false>;
+  static int regs_at_launch[2] = {-1, -1};
+  int &regs = regs_at_launch[with_norm ? 1 : 0];
+  if (regs < 0) {
     cudaFuncAttributes fa;
-    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, bsa_bwd_sm100_kernel));
-    regs_at_launch = fa.numRegs;
+    LC_CUDA_TRY(cudaFuncGetAttributes(&fa, kern));
+    regs = fa.numRegs;
   }
-  if (regs_at_launch < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;  // the split could never complete
-  LC_CUDA_TRY(cudaFuncSetAttribute(bsa_bwd_sm100_kernel,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (regs < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;  // the split could never complete
+  LC_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));
   const size_t rows = (size_t)batch * N * heads;
@@ -789,7 +810,7 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
     prm.dq_acc = dq_acc;
     prm.work_counter = counter;
     const int grid = (int)(total < n_sm ? total : n_sm);
-    bsa_bwd_sm100_kernel<<<grid, kThreads, smem, stream>>>(prm);
+    kern<<<grid, kThreads, smem, stream>>>(prm);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && s == LC_OK)

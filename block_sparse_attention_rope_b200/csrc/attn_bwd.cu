@@ -20,7 +20,8 @@
 // per row), bwd_dq (one CTA per query block x head x batch, one thread per
 // query row, key blocks staged rotated in shared memory), bwd_dkdv (one CTA
 // per key block, one thread per key row, query blocks staged),
-// bwd_dq_finalize (dq from the tensor-core path's fp32 sums).  Every rotation uses the library's shared pair routine and
+// bwd_grad_finalize (dq, and dk under an RMSNorm, from the tensor-core
+// path's fp32 sums).  Every rotation uses the library's shared pair routine and
 // RMSNorm order, so q' and k' are the forward's values before rounding.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -315,9 +316,11 @@ __global__ void __launch_bounds__(64) bwd_dkdv_kernel(BwdArgs a) {
   }
 }
 
-// dq = norm_q^T(R^T dq_acc) for one (batch, token, head) row per thread.
+// g = norm^T(R^T acc) for one (batch, token, head) row per thread: dq from
+// the tensor-core path's fp32 dq sums (raw rows = q, weights = q's), or dk
+// from its fp32 dk' when k is normalised (raw rows = k).
 template <typename Tin>
-__global__ void bwd_dq_finalize_kernel(BwdArgs a, const float *acc, long long rows) {
+__global__ void bwd_grad_finalize_kernel(BwdArgs a, const float *acc, long long rows) {
   const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   if (i >= rows) return;
   const long long N = (long long)a.Nc + a.Nn;
@@ -368,14 +371,14 @@ lc_status lc_bwd_delta(const void *out, const void *dout, float *delta, int batc
   return lc_from_cuda(cudaGetLastError());
 }
 
-lc_status lc_bwd_dq_finalize(const float *dq_acc, const void *q, void *dq, int batch, long long N,
-                             int heads, lc_dtype dtype, const lc_qk_norm &norm,
-                             const lc_rope3d_s *rope, cudaStream_t stream) {
+lc_status lc_bwd_grad_finalize(const float *acc, const void *raw, void *grad, int batch,
+                               long long N, int heads, lc_dtype dtype, const float *nw, float eps,
+                               const lc_rope3d_s *rope, cudaStream_t stream) {
   BwdArgs a;
   memset(&a, 0, sizeof(a));
-  a.q = q; a.dq = dq; a.heads = heads; a.Nc = 0; a.Nn = (int)N;
+  a.q = raw; a.dq = grad; a.heads = heads; a.Nc = 0; a.Nn = (int)N;
   a.tab = rope->tab;
-  a.q_nw = norm.q_w; a.norm_eps = norm.eps;
+  a.q_nw = nw; a.norm_eps = eps;
   a.T = rope->T; a.H = rope->H; a.W = rope->W;
   a.div_hw = lc_make_divmod(rope->H * rope->W);
   a.div_w = lc_make_divmod(rope->W);
@@ -383,9 +386,9 @@ lc_status lc_bwd_dq_finalize(const float *dq_acc, const void *q, void *dq, int b
   if (rows == 0) return LC_OK;
   const unsigned grid = (unsigned)((rows + 127) / 128);
   if (dtype == LC_DTYPE_F32)
-    bwd_dq_finalize_kernel<float><<<grid, 128, 0, stream>>>(a, dq_acc, rows);
+    bwd_grad_finalize_kernel<float><<<grid, 128, 0, stream>>>(a, acc, rows);
   else
-    bwd_dq_finalize_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a, dq_acc, rows);
+    bwd_grad_finalize_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a, acc, rows);
   return lc_from_cuda(cudaGetLastError());
 }
 

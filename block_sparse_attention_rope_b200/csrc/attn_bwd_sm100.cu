@@ -23,9 +23,10 @@
 //                            TMEM lanes), added to the fp32 buffer by warps
 //                            12-15 with vector reductions
 //   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
-//   warp 8: TMA producer (K, V per item, double-buffered; Q, dO per step,
-//   2 stages); warp 9: MMA issuer; warps 10-11: rotate K and Q tiles in
-//   shared memory and stage lse / D per step.
+//   warp 8: TMA producer (K', V per item, double-buffered; Q', dO per step,
+//   2 stages); warp 9: MMA issuer; warps 10-11: stage lse / D per step.
+//   Q' = R(norm(q)) and K' = R(norm(k)) are formed once, before the kernel,
+//   by the one-pass rotation the forward uses for K (same arithmetic).
 //   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448).
 // Every mbarrier wait is bounded; on expiry the CTA stops, drains and frees
 // TMEM, and LC_DEVSTAT_TIMEOUT is set.
@@ -36,14 +37,12 @@
 
 #include "lc_internal.cuh"
 #include "sm100_ptx.cuh"
-#include "sm100_rope.cuh"
 #include "sm100_sync.cuh"
 
 namespace {
 
 using lcsm100::Ctx;
 using lcsm100::drain_wait;
-using lcsm100::rope_row;
 using lcsm100::wait_bar;
 using lcsm100::wait_warp;
 
@@ -54,7 +53,10 @@ constexpr int kWarpMma = 9;
 constexpr int kWarpRope = 10;     // and 11
 constexpr int kRopeThreads = 64;
 constexpr int kWarpDq = 12;       // 12-15
-constexpr int kQStages = 2;
+#ifndef LC_BWD_Q_STAGES
+#define LC_BWD_Q_STAGES 2
+#endif
+constexpr int kQStages = LC_BWD_Q_STAGES;
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kBoxBytes = 64 * 128;
 constexpr uint32_t kTmemCols = 512;
@@ -67,13 +69,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 // hold two 32-column TMEM loads and their results; producer / MMA / RoPE need
 // few; the dQ warpgroup holds one 64-column row.  The host refuses to launch
 // unless the block's registers cover the split.
-constexpr int kRegsEw = 152, kRegsCtl = 80, kRegsDq = 96;
+constexpr int kRegsEw = 152, kRegsCtl = 80, kRegsDq = 112;
 constexpr int kRegsTotal = 256 * kRegsEw + 128 * (kRegsCtl + kRegsDq);
 constexpr int kRegsAtLaunchMin = (kRegsTotal + kThreads - 1) / kThreads;
 static_assert(kRegsTotal <= 65536, "register split");
 
 struct __align__(64) BwdParams {
   CUtensorMap tmQ[2], tmK[2], tmV[2], tmG[2];  // [0] condition segment, [1] noisy; G = dO
+  CUtensorMap tmDQ;                            // fp32 dq sums, half rows (reduce-add target)
   const float *rope_tab;
   const int *kg_ptr;
   const uint32_t *kg_ent;
@@ -84,10 +87,8 @@ struct __align__(64) BwdParams {
   const float *lse;    // [B, heads, N] natural log (the forward's)
   const float *delta;  // [B, heads, N] rowsum(dO * O)
   float *dq_acc;       // [B, N, heads, 64] fp32, zero on entry
+  float *dk_acc;       // [B, N, heads, 64] fp32 dk' (under an RMSNorm of k), or NULL
   __nv_bfloat16 *dk, *dv;
-  const __nv_bfloat16 *k_raw;  // k as given (for the RMSNorm transpose)
-  const float *q_norm_w, *k_norm_w;
-  float norm_eps;
   long long timeout_ns;
   lc_divmod div_hw, div_w;
   int T, H, W;
@@ -101,23 +102,22 @@ struct SmemOffsets {
   static constexpr int q = v + 2 * kTileBytes;                 // [kQStages] query tiles (rotated)
   static constexpr int g = q + kQStages * kTileBytes;          // [kQStages] dO tiles
   static constexpr int ds = g + kQStages * kTileBytes;         // dS^T, two MN-major 64-query tiles
-  static constexpr int lse = ds + 2 * kTileBytes;              // [kQStages][128] lse * log2e
+  static constexpr int dq = ds + 2 * kTileBytes;               // dQ' staging: [block][half] 64 x 32 fp32
+  static constexpr int lse = dq + 2 * kTileBytes;              // [kQStages][128] lse * log2e
   static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] D
   static constexpr int bars = del + kQStages * 128 * 4;
   static constexpr int n_bars = 48;
   static constexpr int misc = bars + n_bars * 8;
-  static constexpr int normw = misc + 64;
-  static constexpr int tab = normw + 2 * 64 * 4;
+  static constexpr int tab = misc + 64;
 };
 
 enum {
   B_SCHED_FULL = 0,                 // [2]
   B_SCHED_EMPTY = 2,                // [2]
-  B_KV_FULL = 4,                    // [2] K, V landed
-  B_KV_READY = 6,                   // [2] K rotated
-  B_KV_EMPTY = 8,                   // [2] item's MMAs done with K, V
-  B_QG_FULL = 10,                   // [kQStages] Q, dO landed
-  B_QG_READY = B_QG_FULL + kQStages,   // Q rotated, lse / D staged
+  B_KV_FULL = 4,                    // [2] K', V landed
+  B_KV_EMPTY = 6,                   // [2] item's MMAs done with K', V
+  B_QG_FULL = 8,                    // [kQStages] Q', dO landed
+  B_QG_READY = B_QG_FULL + kQStages,   // lse / D staged
   B_QG_EMPTY = B_QG_READY + kQStages,  // step's MMAs done with Q, dO
   B_SDP = B_QG_EMPTY + kQStages,    // S^T and dP^T in TMEM
   B_PDS = B_SDP + 1,                // P^T, dS^T written (8 warps)
@@ -126,7 +126,9 @@ enum {
   B_DQ_EMPTY = B_DQ_FULL + 1,       // dQ read out (4 warps)
   B_ACC = B_DQ_EMPTY + 1,           // item's dK, dV complete
   B_EPI_FREE = B_ACC + 1,           // dK, dV read out (8 warps)
-  B_DRAIN = B_EPI_FREE + 1,
+  B_DQ_STAGED = B_EPI_FREE + 1,     // dQ' tile staged in shared memory (4 warps)
+  B_DQ_SMEM_FREE = B_DQ_STAGED + 1, // its reduce-add has read the staging tile
+  B_DRAIN = B_DQ_SMEM_FREE + 1,
   B_COUNT = B_DRAIN + 1
 };
 static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
@@ -208,8 +210,8 @@ __device__ __forceinline__ void pair_angle(const BwdParams &a, const float *tab,
   }
 }
 
-// kNorm: RMSNorm weights in use (the plain path is a separate instantiation
-// that carries none of that code).
+// kNorm: k is RMS-normalised, so dK' goes out in fp32 for the finalize pass
+// (the plain path is a separate instantiation without that branch).
 template <bool kNorm>
 __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -226,7 +228,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   float *sDel = reinterpret_cast<float *>(smem + SmemOffsets::del);
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SmemOffsets::misc);
   // misc[0] tmem base, misc[1..2] scheduled items, misc[3] abort flag
-  float *s_normw = reinterpret_cast<float *>(smem + SmemOffsets::normw);  // [q 64 | k 64]
   float *tab = reinterpret_cast<float *>(smem + SmemOffsets::tab);
   Ctx ctx;
   ctx.bar0 = lcptx::smem_addr(smem + SmemOffsets::bars);
@@ -236,15 +237,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   const long long N = (long long)p.Nc + p.Nn;
 
   for (int i = tid; i < p.tab_floats; i += kThreads) tab[i] = p.rope_tab[i];
-  if (tid < 64 && p.q_norm_w) s_normw[tid] = p.q_norm_w[tid];
-  if (tid < 64 && p.k_norm_w) s_normw[64 + tid] = p.k_norm_w[tid];
   if (tid == 0) {
     misc[3] = 0;
     for (int i = 0; i < 2; ++i) {
       lcptx::mbar_init(ctx.bar(B_SCHED_FULL + i), 1);
       lcptx::mbar_init(ctx.bar(B_SCHED_EMPTY + i), kSchedConsumers);
       lcptx::mbar_init(ctx.bar(B_KV_FULL + i), 1);
-      lcptx::mbar_init(ctx.bar(B_KV_READY + i), kRopeThreads);
       lcptx::mbar_init(ctx.bar(B_KV_EMPTY + i), 1);
     }
     for (int s = 0; s < kQStages; ++s) {
@@ -259,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     lcptx::mbar_init(ctx.bar(B_DQ_EMPTY), 4);
     lcptx::mbar_init(ctx.bar(B_ACC), 1);
     lcptx::mbar_init(ctx.bar(B_EPI_FREE), kEwWarps);
+    lcptx::mbar_init(ctx.bar(B_DQ_STAGED), 4);
+    lcptx::mbar_init(ctx.bar(B_DQ_SMEM_FREE), 1);
     lcptx::mbar_init(ctx.bar(B_DRAIN), 1);
     lcptx::fence_mbar_init();
   }
@@ -273,6 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       lcptx::tma_prefetch_desc(&p.tmV[i]);
       lcptx::tma_prefetch_desc(&p.tmG[i]);
     }
+    lcptx::tma_prefetch_desc(&p.tmDQ);
   }
   lcptx::tc_fence_before();
   __syncthreads();
@@ -377,12 +378,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         const KItem it = decode_kitem(p, item);
         const int kb = item_it & 1;
         const uint32_t kph = (item_it >> 1) & 1;
-        bool ok = wait_bar(ctx, ctx.bar(B_KV_READY + kb), kph);
+        bool ok = wait_bar(ctx, ctx.bar(B_KV_FULL + kb), kph);
         const int nsteps = (it.len + 1) >> 1;
         for (int t = 0; t < nsteps && ok; ++t, ++q_it, ++k_step) {
           const int s = q_it % kQStages;
           const uint32_t ph = (q_it / kQStages) & 1;
-          ok = wait_bar(ctx, ctx.bar(B_QG_READY + s), ph);
+          ok = wait_bar(ctx, ctx.bar(B_QG_FULL + s), ph);
           if (!ok) break;
           // S^T of this step overwrites P^T of the previous one: its P*V must be done.
           if (step_pending) {
@@ -444,10 +445,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     }
     __syncwarp();
   } else {
-    // ======================= RoPE warps: K per item, Q + lse / D per step ====
+    // ======================= warps 10-11: stage lse / D per step =============
     const int rt = tid - kWarpRope * 32;
-    const float *q_nw = (kNorm && p.q_norm_w) ? s_normw : nullptr;
-    const float *k_nw = (kNorm && p.k_norm_w) ? s_normw + 64 : nullptr;
     uint32_t item_it = 0, q_it = 0;
     for (;;) {
       const int slot = item_it & 1;
@@ -457,50 +456,38 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
       const KItem it = decode_kitem(p, item);
-      const int kb = item_it & 1;
-      bool ok = wait_warp(ctx, ctx.bar(B_KV_FULL + kb), (item_it >> 1) & 1);
-      if (!ok) break;
-      const int seg_tok = it.seg ? p.Nc : 0;
-      for (int r = rt; r < 128; r += kRopeThreads)
-        if ((r >> 6) < it.cnt && it.krow(r >> 6) + (r & 63) < it.seg_len)
-          rope_row(sK + kb * kTileBytes, r, seg_tok + it.krow(r >> 6) + (r & 63), tab, p, k_nw);
-      lcptx::fence_proxy_async_smem();
-      lcptx::mbar_arrive(ctx.bar(B_KV_READY + kb));
+      bool ok = true;
       const int nsteps = (it.len + 1) >> 1;
       const float *lse_bh = p.lse + ((long long)it.b * p.heads + it.h) * N;
       const float *del_bh = p.delta + ((long long)it.b * p.heads + it.h) * N;
       for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
         const int s = q_it % kQStages;
-        // This thread's two query rows (rt of each query block): token, lse and
-        // D first, so that their global loads overlap the wait and the rotation.
-        int tokr[2];
+        // This thread's two query rows (rt of each query block): lse and D of
+        // their tokens (0 for rows that do not exist; they are masked).
         float l2r[2], dlr[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          tokr[i] = -1;
           l2r[i] = dlr[i] = 0.f;
           const int e = 2 * t + i;
           if (e < it.len) {
             int qs, qr, qn;
             qblock(p, __ldg(it.ent + e), qs, qr, qn);
             if (rt < qn) {
-              tokr[i] = (qs ? p.Nc : 0) + qr + rt;
-              l2r[i] = __ldg(lse_bh + tokr[i]) * kLog2e;
-              dlr[i] = __ldg(del_bh + tokr[i]);
+              const int tok = (qs ? p.Nc : 0) + qr + rt;
+              l2r[i] = __ldg(lse_bh + tok) * kLog2e;
+              dlr[i] = __ldg(del_bh + tok);
             }
           }
         }
+        // the stage is free once its previous step's MMAs are done, which the
+        // producer's reload of it implies
         ok = wait_warp(ctx, ctx.bar(B_QG_FULL + s), (q_it / kQStages) & 1);
         if (!ok) break;
-#pragma unroll 1
-        for (int i = 0; i < 2; ++i)
-          if (tokr[i] >= 0) rope_row(sQ + s * kTileBytes, rt + 64 * i, tokr[i], tab, p, q_nw);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           sLse[s * 128 + rt + 64 * i] = l2r[i];
           sDel[s * 128 + rt + 64 * i] = dlr[i];
         }
-        lcptx::fence_proxy_async_smem();
         lcptx::mbar_arrive(ctx.bar(B_QG_READY + s));
       }
       if (!ok) break;
@@ -509,10 +496,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   }
   } else if (warp >= kWarpDq) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDq));
-    // ======================= dQ warps: TMEM dQ -> fp32 atomics ================
+    // ======================= dQ warps: TMEM dQ' -> shared -> TMA reduce-add ==
+    // Each step's dQ' tile (128 query rows x 64 fp32) is staged in shared
+    // memory as four 64-row x 32-channel swizzled boxes and added into the
+    // fp32 dq sums by the TMA engine (one thread issues; nothing per lane
+    // goes to global memory).  Rows of absent or padded queries are zero.
     const int qrow = tid - kWarpDq * 32;  // TMEM lane == query row of the step
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    uint32_t item_it = 0, dq_ph = 0;
+    uint8_t *sDQ = smem + SmemOffsets::dq;
+    uint32_t item_it = 0, dq_ph = 0, dq_step = 0;
+    bool issued = false;
     for (;;) {
       const int slot = item_it & 1;
       if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
@@ -523,40 +516,61 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const KItem it = decode_kitem(p, item);
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
-      for (int t = 0; t < nsteps; ++t) {
+      for (int t = 0; t < nsteps; ++t, ++dq_step) {
         ok = wait_warp(ctx, ctx.bar(B_DQ_FULL), dq_ph);
         if (!ok) break;
         dq_ph ^= 1;
         lcptx::tc_fence_after();
-        uint32_t a0[32], a1[32];
-        lcptx::tmem_ld32(tmem + lane_base + kColDQ, a0);
-        lcptx::tmem_ld32(tmem + lane_base + kColDQ + 32, a1);
+        uint32_t a[2][32];
+        lcptx::tmem_ld32(tmem + lane_base + kColDQ, a[0]);
+        lcptx::tmem_ld32(tmem + lane_base + kColDQ + 32, a[1]);
         lcptx::tmem_wait_ld();
         lcptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_DQ_EMPTY));
-        const int e = 2 * t + (qrow >> 6);
-        if (e < it.len) {
-          int qs, qr, qn;
-          qblock(p, __ldg(it.ent + e), qs, qr, qn);
-          if ((qrow & 63) < qn) {
-            const long long tok = (qs ? p.Nc : 0) + qr + (qrow & 63);
-            float *dst = p.dq_acc + (((long long)it.b * N + tok) * p.heads + it.h) * LC_HEAD_DIM;
+        // the previous step's reduce-add has finished reading the staging tile
+        ok = wait_warp(ctx, ctx.bar(B_DQ_SMEM_FREE), (dq_step & 1) ^ 1);
+        if (!ok) break;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              lcptx::red_add_v4_f32(dst + 4 * c, __uint_as_float(a0[4 * c]), __uint_as_float(a0[4 * c + 1]),
-                                    __uint_as_float(a0[4 * c + 2]), __uint_as_float(a0[4 * c + 3]));
+        for (int hd = 0; hd < 2; ++hd) {
+          uint8_t *tile = sDQ + ((qrow >> 6) * 2 + hd) * (64 * 128);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              lcptx::red_add_v4_f32(dst + 32 + 4 * c, __uint_as_float(a1[4 * c]),
-                                    __uint_as_float(a1[4 * c + 1]), __uint_as_float(a1[4 * c + 2]),
-                                    __uint_as_float(a1[4 * c + 3]));
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4 *>(tile + swz(qrow & 63, c)) =
+                make_uint4(a[hd][4 * c], a[hd][4 * c + 1], a[hd][4 * c + 2], a[hd][4 * c + 3]);
+        }
+        lcptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_DQ_STAGED));
+        if (qrow == 0) {
+          ok = wait_bar(ctx, ctx.bar(B_DQ_STAGED), dq_step & 1);
+          if (ok) {
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk) {
+              const int e = 2 * t + blk;
+              if (e >= it.len) continue;
+              int qs, qr, qn;
+              qblock(p, __ldg(it.ent + e), qs, qr, qn);
+              const int tok0 = (qs ? p.Nc : 0) + qr;
+#pragma unroll
+              for (int hd = 0; hd < 2; ++hd)
+                lcptx::tma_reduce_add_4d(&p.tmDQ,
+                                         lcptx::smem_addr(sDQ + (blk * 2 + hd) * (64 * 128)),
+                                         32 * hd, it.h, tok0, it.b);
+            }
+            lcptx::bulk_commit_group();
+            issued = true;
+            lcptx::bulk_wait_group_read0();
+            lcptx::mbar_arrive(ctx.bar(B_DQ_SMEM_FREE));
           }
         }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && !*ctx.abort_flag;
+        if (!ok) break;
       }
       if (!ok) break;
       ++item_it;
     }
+    if (qrow == 0 && issued) lcptx::bulk_wait_group0();  // every reduce-add complete
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsEw));
     // ======================= elementwise warps 0-7 ===========================
@@ -639,8 +653,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));
       }
       if (!ok) break;
-      // ---- epilogue: warps 0-3 store dV; warps 4-7 store dK = R^T dK' (and
-      // the RMSNorm transpose).  bf16 rows straight to global memory.
+      // ---- epilogue: warps 0-3 store dV; warps 4-7 store dK = R^T dK' as bf16
+      // rows straight to global memory, or, when k is normalised, dK' in fp32
+      // for the finalize pass (R^T and the RMSNorm transpose).
       ok = wait_warp(ctx, ctx.bar(B_ACC), item_it & 1);
       if (!ok) break;
       lcptx::tc_fence_after();
@@ -663,54 +678,30 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_EPI_FREE));
       if (key_valid) {
-        if (half) {
+        if (kNorm && half && p.dk_acc) {  // dk' as is; R^T and the norm transpose follow
+          float4 *dst = reinterpret_cast<float4 *>(p.dk_acc + off);
 #pragma unroll
-          for (int q2 = 0; q2 < 32; ++q2) {  // R^T: turn each pair back
-            float c, sn;
-            pair_angle(p, tab, tok, q2, c, sn);
-            const float u = acc[2 * q2], w = acc[2 * q2 + 1];
-            acc[2 * q2] = fmaf(u, c, w * sn);
-            acc[2 * q2 + 1] = fmaf(w, c, -u * sn);
-          }
-          if (kNorm && p.k_norm_w) {  // y = x inv w: dx = inv (w g) - x inv^3 / 64 sum(g w x)
-            const uint4 *xr = reinterpret_cast<const uint4 *>(p.k_raw + off);  // 8 bf16 per load
-            float c8[8], dot = 0.f;
+          for (int c = 0; c < 16; ++c)
+            dst[c] = make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+        } else {
+          if (half) {
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 raw = __ldg(xr + ch);
-              const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-              float x8[8];
-#pragma unroll
-              for (int e2 = 0; e2 < 4; ++e2) {
-                x8[2 * e2] = __uint_as_float(wd[e2] << 16);
-                x8[2 * e2 + 1] = __uint_as_float(wd[e2] & 0xFFFF0000u);
-              }
-              c8[ch] = lc_sumsq8(x8);
-#pragma unroll
-              for (int e2 = 0; e2 < 8; ++e2)
-                dot = fmaf(acc[8 * ch + e2] * s_normw[64 + 8 * ch + e2], x8[e2], dot);
-            }
-            const float inv = lc_rms_inv(lc_sumsq_tree8(c8), p.norm_eps);
-            const float k3 = inv * inv * inv * (1.f / 64.f) * dot;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint4 raw = __ldg(xr + ch);
-              const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-              for (int e2 = 0; e2 < 4; ++e2) {
-                const int d = 8 * ch + 2 * e2;
-                acc[d] = inv * s_normw[64 + d] * acc[d] - __uint_as_float(wd[e2] << 16) * k3;
-                acc[d + 1] = inv * s_normw[64 + d + 1] * acc[d + 1] -
-                             __uint_as_float(wd[e2] & 0xFFFF0000u) * k3;
-              }
+            for (int q2 = 0; q2 < 32; ++q2) {  // R^T: turn each pair back
+              float c, sn;
+              pair_angle(p, tab, tok, q2, c, sn);
+              const float u = acc[2 * q2], w = acc[2 * q2 + 1];
+              acc[2 * q2] = fmaf(u, c, w * sn);
+              acc[2 * q2 + 1] = fmaf(w, c, -u * sn);
             }
           }
+          uint4 *dst = reinterpret_cast<uint4 *>((half ? p.dk : p.dv) + off);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_uint4(pack_bf16(acc[8 * c], acc[8 * c + 1]),
+                                pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
+                                pack_bf16(acc[8 * c + 4], acc[8 * c + 5]),
+                                pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
         }
-        uint4 *dst = reinterpret_cast<uint4 *>((half ? p.dk : p.dv) + off);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          dst[c] = make_uint4(pack_bf16(acc[8 * c], acc[8 * c + 1]), pack_bf16(acc[8 * c + 2], acc[8 * c + 3]),
-                              pack_bf16(acc[8 * c + 4], acc[8 * c + 5]), pack_bf16(acc[8 * c + 6], acc[8 * c + 7]));
       }
       ++item_it;
     }
@@ -733,39 +724,9 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   BwdParams prm;
   memset(&prm, 0, sizeof(prm));
   const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
-  const void *src[4] = {q, k, v, dout};
-  CUtensorMap *maps[4] = {prm.tmQ, prm.tmK, prm.tmV, prm.tmG};
-  for (int i = 0; i < 4; ++i) {
-    lc_status s = lc_encode_segment(&maps[i][1], src[i], batch, N, Nc, Nn, heads);
-    if (s == LC_OK && Nc > 0) s = lc_encode_segment(&maps[i][0], src[i], batch, N, 0, Nc, heads);
-    if (s != LC_OK) return s;
-    if (Nc == 0) maps[i][0] = maps[i][1];  // unused, kept a valid descriptor
-  }
-  prm.rope_tab = rope->tab;
-  prm.kg_ptr = plan->kgrp_ptr;
-  prm.kg_ent = plan->kgrp_ent;
-  prm.kg_order = plan->kgrp_order;
-  prm.kg_blk = plan->kgrp_blk;
-  prm.lse = lse;
-  prm.dk = static_cast<__nv_bfloat16 *>(dk);
-  prm.dv = static_cast<__nv_bfloat16 *>(dv);
-  prm.k_raw = static_cast<const __nv_bfloat16 *>(k);
-  prm.q_norm_w = norm.q_w;
-  prm.k_norm_w = norm.k_w;
-  prm.norm_eps = norm.eps;
-  prm.timeout_ns = 2000000000LL;
-  prm.div_hw = lc_make_divmod(rope->H * rope->W);
-  prm.div_w = lc_make_divmod(rope->W);
-  prm.T = rope->T; prm.H = rope->H; prm.W = rope->W;
-  prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.kgc = plan->kgc;
-  prm.heads = heads;
-  prm.KG = plan->KG;
-  prm.tab_floats = (int)rope->n_floats;
-  prm.scale = scale;
   const long long total = (long long)batch * heads * plan->KG;
   if (total == 0) return LC_OK;
   if (total >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
-  prm.total_items = (int)total;
   const size_t smem = 1024 + SmemOffsets::tab + sizeof(float) * (size_t)rope->n_floats;
   if (smem > 227 * 1024) return LC_ERR_UNSUPPORTED;
   lc_status s = LC_OK;
@@ -773,10 +734,7 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   if (s != LC_OK) return s;
   cudaMemPool_t pool = lc_scratch_pool(&s);
   if (s != LC_OK) return s;
-  int dev = 0, n_sm = 0;
-  LC_CUDA_TRY(cudaGetDevice(&dev));
-  LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
-  const bool with_norm = norm.q_w || norm.k_w;
+  const bool with_norm = norm.k_w != nullptr;
   void (*const kern)(const BwdParams) = with_norm ? bsa_bwd_sm100_kernel<true>
                                                   : bsa_bwd_sm100_kernel<false>;
   static int regs_at_launch[2] = {-1, -1};
@@ -788,11 +746,19 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   }
   if (regs < kRegsAtLaunchMin) return LC_ERR_UNSUPPORTED;  // the split could never complete
   LC_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int dev = 0, n_sm = 0;
+  LC_CUDA_TRY(cudaGetDevice(&dev));
+  LC_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));
+
+  // Scratch from the library's pool: D, the fp32 dq sums, the scheduler
+  // counter, and Q' = R(norm(q)), K' = R(norm(k)).
   const size_t rows = (size_t)batch * N * heads;
-  float *delta = nullptr, *dq_acc = nullptr;
+  const size_t tbytes = rows * LC_HEAD_DIM * 2;
+  float *delta = nullptr, *dq_acc = nullptr, *dk_acc = nullptr;
   int *counter = nullptr;
+  void *q_rot = nullptr, *k_rot = nullptr;
   cudaError_t e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&delta), rows * sizeof(float),
                                           pool, stream);
   if (e == cudaSuccess)
@@ -800,21 +766,63 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
                                 rows * LC_HEAD_DIM * sizeof(float), pool, stream);
   if (e == cudaSuccess)
     e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&counter), sizeof(int), pool, stream);
+  if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&q_rot, tbytes, pool, stream);
+  if (e == cudaSuccess) e = cudaMallocFromPoolAsync(&k_rot, tbytes, pool, stream);
+  if (e == cudaSuccess && norm.k_w)  // dk' in fp32, normalised back by the finalize pass
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&dk_acc),
+                                rows * LC_HEAD_DIM * sizeof(float), pool, stream);
   if (e == cudaSuccess)
     e = cudaMemsetAsync(dq_acc, 0, rows * LC_HEAD_DIM * sizeof(float), stream);
   if (e == cudaSuccess) e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) s = lc_rope_rows_bf16(q, q_rot, batch, N, heads, 0, rope, norm.q_w, norm.eps, stream);
+  if (e == cudaSuccess && s == LC_OK)
+    s = lc_rope_rows_bf16(k, k_rot, batch, N, heads, 0, rope, norm.k_w, norm.eps, stream);
+  if (e == cudaSuccess && s == LC_OK)
     s = lc_bwd_delta(out, dout, delta, batch, N, heads, LC_DTYPE_BF16, stream);
+  if (e == cudaSuccess && s == LC_OK) s = lc_encode_f32_halfrows(&prm.tmDQ, dq_acc, batch, N, heads);
+  const void *src[4] = {q_rot, k_rot, v, dout};
+  CUtensorMap *maps[4] = {prm.tmQ, prm.tmK, prm.tmV, prm.tmG};
+  for (int i = 0; i < 4 && e == cudaSuccess && s == LC_OK; ++i) {
+    s = lc_encode_segment(&maps[i][1], src[i], batch, N, Nc, Nn, heads);
+    if (s == LC_OK && Nc > 0) s = lc_encode_segment(&maps[i][0], src[i], batch, N, 0, Nc, heads);
+    if (Nc == 0) maps[i][0] = maps[i][1];  // unused, kept a valid descriptor
+  }
   if (e == cudaSuccess && s == LC_OK) {
+    prm.rope_tab = rope->tab;
+    prm.kg_ptr = plan->kgrp_ptr;
+    prm.kg_ent = plan->kgrp_ent;
+    prm.kg_order = plan->kgrp_order;
+    prm.kg_blk = plan->kgrp_blk;
+    prm.lse = lse;
     prm.delta = delta;
     prm.dq_acc = dq_acc;
+    prm.dk_acc = dk_acc;
     prm.work_counter = counter;
+    prm.dk = static_cast<__nv_bfloat16 *>(dk);
+    prm.dv = static_cast<__nv_bfloat16 *>(dv);
+    prm.timeout_ns = 2000000000LL;
+    prm.div_hw = lc_make_divmod(rope->H * rope->W);
+    prm.div_w = lc_make_divmod(rope->W);
+    prm.T = rope->T; prm.H = rope->H; prm.W = rope->W;
+    prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.kgc = plan->kgc;
+    prm.heads = heads;
+    prm.KG = plan->KG;
+    prm.total_items = (int)total;
+    prm.tab_floats = (int)rope->n_floats;
+    prm.scale = scale;
     const int grid = (int)(total < n_sm ? total : n_sm);
     kern<<<grid, kThreads, smem, stream>>>(prm);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess && s == LC_OK)
-    s = lc_bwd_dq_finalize(dq_acc, q, dq, batch, N, heads, LC_DTYPE_BF16, norm, rope, stream);
+    s = lc_bwd_grad_finalize(dq_acc, q, dq, batch, N, heads, LC_DTYPE_BF16, norm.q_w, norm.eps,
+                             rope, stream);
+  if (e == cudaSuccess && s == LC_OK && dk_acc)
+    s = lc_bwd_grad_finalize(dk_acc, k, dk, batch, N, heads, LC_DTYPE_BF16, norm.k_w, norm.eps,
+                             rope, stream);
+  if (dk_acc) cudaFreeAsync(dk_acc, stream);
+  if (k_rot) cudaFreeAsync(k_rot, stream);
+  if (q_rot) cudaFreeAsync(q_rot, stream);
   if (counter) cudaFreeAsync(counter, stream);
   if (dq_acc) cudaFreeAsync(dq_acc, stream);
   if (delta) cudaFreeAsync(delta, stream);

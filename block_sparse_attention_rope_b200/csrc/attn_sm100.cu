@@ -283,38 +283,6 @@ __device__ __forceinline__ float row_max(const float (&s)[128]) {
   return max3(max3(mc[0], mc[1], mc[2]), max3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
 }
 
-// P = 2^(s * scale_log2 - m) for a 128-column row, written as bf16 pairs to
-// TMEM (64 columns at tP) in four 32-key chunks as they are produced; returns
-// the fp32 row sum of P.
-__device__ __forceinline__ float exp_pass_store(const float (&s)[128], float sl2, float m,
-                                                uint32_t tP) {
-  const float2 sc2 = make_float2(sl2, sl2);
-  const float2 nm2 = make_float2(-m, -m);
-  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                   make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t pk[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int jj = 16 * c + j;  // column pair
-      const float2 x = __ffma2_rn(make_float2(s[2 * jj], s[2 * jj + 1]), sc2, nm2);
-      float2 e;
-      if (kPolyMask & (1u << (jj & 7))) {
-        e = exp2_poly2(x);
-      } else {
-        e.x = ex2(x.x);
-        e.y = ex2(x.y);
-      }
-      acc[j & 3] = __fadd2_rn(acc[j & 3], e);
-      pk[j] = pack_bf16(e.x, e.y);
-    }
-    lcptx::tmem_st16(tP + 16 * c, pk);
-  }
-  const float2 a = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-  return a.x + a.y;
-}
-
 // Mask limits of tile tt of an item for the rows of query block `qsub`:
 // bits 0-7 = attended tokens of the tile's first key block (0 when the block
 // is not attended), bits 8-15 = same for the second block.
@@ -994,6 +962,29 @@ lc_status launch_rope_k(const void *src, void *dst, int batch, long long ntok, i
 lc_status lc_encode_segment(CUtensorMap *m, const void *base, int batch, long long ntot,
                             long long tok0, long long nseg, int heads) {
   return encode_segment(m, base, batch, ntot, tok0, nseg, heads);
+}
+
+lc_status lc_encode_f32_halfrows(CUtensorMap *m, const float *base, int batch, long long ntot,
+                                 int heads) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return LC_ERR_CUDA;
+  const long long row_bytes = (long long)heads * LC_HEAD_DIM * 4;
+  cuuint64_t dims[4] = {LC_HEAD_DIM, (cuuint64_t)heads, (cuuint64_t)ntot, (cuuint64_t)batch};
+  cuuint64_t strides[3] = {LC_HEAD_DIM * 4, (cuuint64_t)row_bytes, (cuuint64_t)(ntot * row_bytes)};
+  cuuint32_t box[4] = {32, 1, 64, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LC_OK : LC_ERR_CUDA;
+}
+
+lc_status lc_rope_rows_bf16(const void *src, void *dst, int batch, long long ntok, int heads,
+                            int tok_offset, const lc_rope3d_s *rope, const float *nw, float eps,
+                            cudaStream_t stream) {
+  if (ntok <= 0) return LC_OK;
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, rope->ready, 0));
+  return launch_rope_k(src, dst, batch, ntok, heads, tok_offset, rope, stream, nw, eps);
 }
 
 // ------------------------------------------------------------ no-alloc scratch

@@ -186,17 +186,22 @@ lc_status lc_launch_backward(const void *q, const void *k, const void *v, const 
                              const lc_rope3d_s *rope, cudaStream_t stream);
 // The tensor-core backward (attn_bwd_sm100.cu, bf16), and the pieces of the
 // backward shared by both paths (attn_bwd.cu): D = rowsum(dO * O) per row, and
-// dq = norm_q^T(R^T dq_acc) cast to dtype.
+// grad = norm^T(R^T acc) cast to dtype (dq; dk under an RMSNorm).
 lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, const void *out,
                                    const float *lse, const void *dout, void *dq, void *dk,
                                    void *dv, int batch, int heads, float scale,
                                    const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
                                    const lc_rope3d_s *rope, cudaStream_t stream);
+// R(norm(x)) of a bf16 [batch, ntok, heads, 64] tensor into dst, with the
+// attention kernels' exact arithmetic (attn_sm100.cu).
+lc_status lc_rope_rows_bf16(const void *src, void *dst, int batch, long long ntok, int heads,
+                            int tok_offset, const lc_rope3d_s *rope, const float *nw, float eps,
+                            cudaStream_t stream);
 lc_status lc_bwd_delta(const void *out, const void *dout, float *delta, int batch, long long N,
                        int heads, lc_dtype dtype, cudaStream_t stream);
-lc_status lc_bwd_dq_finalize(const float *dq_acc, const void *q, void *dq, int batch, long long N,
-                             int heads, lc_dtype dtype, const lc_qk_norm &norm,
-                             const lc_rope3d_s *rope, cudaStream_t stream);
+lc_status lc_bwd_grad_finalize(const float *acc, const void *raw, void *grad, int batch,
+                               long long N, int heads, lc_dtype dtype, const float *nw, float eps,
+                               const lc_rope3d_s *rope, cudaStream_t stream);
 // Rotate x [batch, ntok, heads, 64] of dtype (token n of x = sequence token
 // n + tok_offset) into out, after an RMSNorm with norm_w when not NULL
 // (rope.cu; the public lc_rope3d_apply is this without the norm).  Arguments

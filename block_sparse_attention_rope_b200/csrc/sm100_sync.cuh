@@ -67,3 +67,8 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, long l
 // 128-byte swizzle, zero fill out of range (attn_sm100.cu).
 lc_status lc_encode_segment(CUtensorMap *m, const void *base, int batch, long long ntot,
                             long long tok0, long long nseg, int heads);
+// Tensor map over an fp32 [B, ntot, heads, 64] tensor: boxes of 64 tokens x
+// 1 head x 32 channels (128 bytes, 128-byte swizzle), for TMA reduce-adds of
+// half rows (attn_sm100.cu).
+lc_status lc_encode_f32_halfrows(CUtensorMap *m, const float *base, int batch, long long ntot,
+                                 int heads);

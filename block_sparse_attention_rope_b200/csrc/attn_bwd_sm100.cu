@@ -615,13 +615,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         lcptx::tc_fence_after();
         const float *l2 = sLse + s * 128, *dl = sDel + s * 128;
         uint8_t *tile = sDS + half * kTileBytes;  // dS^T, this query block's MN-major chunk
-#pragma unroll 1
-        for (int c = 4 * half; c < 4 * half + 4; ++c) {  // 16 queries at a time
-          uint32_t sr[16], dr[16];
-          lcptx::tmem_ld16(tST + 16 * c, sr);
-          lcptx::tmem_ld16(tDPT + 16 * c, dr);
-          lcptx::tmem_wait_ld();
-          const int jb = (c & 3) * 16;  // first query of the chunk within its block
+        // 16 queries at a time; the next chunk's TMEM loads are in flight while
+        // this one is computed (double buffer)
+        uint32_t sr[2][16], dr[2][16];
+        lcptx::tmem_ld16(tST + 64 * half, sr[0]);
+        lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
+        lcptx::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c = 4 * half + k;
+          if (k < 3) {
+            lcptx::tmem_ld16(tST + 64 * half + 16 * (k + 1), sr[(k + 1) & 1]);
+            lcptx::tmem_ld16(tDPT + 64 * half + 16 * (k + 1), dr[(k + 1) & 1]);
+          }
+          const uint32_t(&scur)[16] = sr[k & 1];
+          const uint32_t(&dcur)[16] = dr[k & 1];
+          const int jb = k * 16;  // first query of the chunk within its block
           uint32_t pp[8], dd[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -630,21 +639,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             for (int u = 0; u < 2; ++u) {
               const int j = 16 * c + 2 * i + u;
               const bool on = jb + 2 * i + u < lim;
-              const float pe = on ? ex2(__uint_as_float(sr[2 * i + u]) * sl2 - l2[j]) : 0.f;
+              const float pe = on ? ex2(__uint_as_float(scur[2 * i + u]) * sl2 - l2[j]) : 0.f;
               pv[u] = pe;
-              dv2[u] = pe * (__uint_as_float(dr[2 * i + u]) - dl[j]) * p.scale;
+              dv2[u] = pe * (__uint_as_float(dcur[2 * i + u]) - dl[j]) * p.scale;
             }
             pp[i] = pack_bf16(pv[0], pv[1]);
             dd[i] = pack_bf16(dv2[0], dv2[1]);
           }
-          // P^T / dS^T of queries 16c..16c+15 go to columns 64 half + 8 (c & 3):
+          // P^T / dS^T of queries 16c..16c+15 go to columns 64 half + 8 k:
           // inside this warp's own 64 columns, and already read
-          lcptx::tmem_st8(tST + 64 * half + 8 * (c & 3), pp);
-          lcptx::tmem_st8(tDPT + 64 * half + 8 * (c & 3), dd);
+          lcptx::tmem_st8(tST + 64 * half + 8 * k, pp);
+          lcptx::tmem_st8(tDPT + 64 * half + 8 * k, dd);
 #pragma unroll
           for (int i = 0; i < 2; ++i)
-            *reinterpret_cast<uint4 *>(tile + swz(kr, (c & 3) * 2 + i)) =
+            *reinterpret_cast<uint4 *>(tile + swz(kr, k * 2 + i)) =
                 make_uint4(dd[4 * i], dd[4 * i + 1], dd[4 * i + 2], dd[4 * i + 3]);
+          if (k < 3) lcptx::tmem_wait_ld();
         }
         lcptx::fence_proxy_async_smem();
         lcptx::tmem_wait_st();

@@ -14,17 +14,16 @@
 //   per step, with keys as TMEM lanes (M = 128):
 //     S^T  = K' Q'^T        dP^T = V dO^T          (tcgen05, into TMEM)
 //     P^T  = exp(scale S^T - lse),  dS^T = P^T (dP^T - D) scale
-//                           (warps 0-7, one key row and query half per thread; P^T, dS^T
-//                            written back as bf16 over each half's consumed
-//                            columns,
-//                            dS^T also to shared memory for dQ)
-//     dV  += P^T dO         dK' += dS^T Q'         (A from TMEM)
+//                           (warps 0-7, one key row and query block per
+//                            thread; P^T and dS^T written as bf16 tiles to
+//                            shared memory, so the next step's S^T, dP^T can
+//                            be computed while they are formed)
+//     dV  += P^T dO         dK' += dS^T Q'         (A from shared memory)
 //     dQ'  = dS K'          (A = dS from shared memory, MN-major; queries as
 //                            TMEM lanes), added to the fp32 buffer by warps
 //                            12-15 with vector reductions
 //   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
-//   warp 8: TMA producer (K', V per item, double-buffered; Q', dO per step,
-//   2 stages); warp 9: MMA issuer; warps 10-11: stage lse / D per step.
+//   warp 8: TMA producer (K', V per item; Q', dO per step, 2 stages); warp 9: MMA issuer; warps 10-11: stage lse / D per step.
 //   Q' = R(norm(q)) and K' = R(norm(k)) are formed once, before the kernel,
 //   by the one-pass rotation the forward uses for K (same arithmetic).
 //   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448).
@@ -62,7 +61,7 @@ constexpr int kBoxBytes = 64 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
 constexpr uint32_t kIdescKQ = lcptx::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
-constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A in TMEM)
+constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A K-major)
 constexpr uint32_t kIdescDQ = lcptx::idesc_bf16_f32(128, 64, 1, 1);   // dQ (A = dS, MN-major)
 constexpr float kLog2e = 1.4426950408889634f;
 // Register split (setmaxnreg, per warpgroup): the two elementwise warpgroups
@@ -97,11 +96,12 @@ struct __align__(64) BwdParams {
 };
 
 struct SmemOffsets {
-  static constexpr int k = 0;                                  // [2] key tiles (rotated)
-  static constexpr int v = k + 2 * kTileBytes;                 // [2]
-  static constexpr int q = v + 2 * kTileBytes;                 // [kQStages] query tiles (rotated)
+  static constexpr int k = 0;                                  // key tile K' (one item)
+  static constexpr int v = k + kTileBytes;                     // value tile
+  static constexpr int q = v + kTileBytes;                     // [kQStages] query tiles Q'
   static constexpr int g = q + kQStages * kTileBytes;          // [kQStages] dO tiles
-  static constexpr int ds = g + kQStages * kTileBytes;         // dS^T, two MN-major 64-query tiles
+  static constexpr int pt = g + kQStages * kTileBytes;         // P^T, two 64-query tiles
+  static constexpr int ds = pt + 2 * kTileBytes;               // dS^T, two 64-query tiles
   static constexpr int dq = ds + 2 * kTileBytes;               // dQ' staging: [block][half] 64 x 32 fp32
   static constexpr int lse = dq + 2 * kTileBytes;              // [kQStages][128] lse * log2e
   static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] D
@@ -114,14 +114,15 @@ struct SmemOffsets {
 enum {
   B_SCHED_FULL = 0,                 // [2]
   B_SCHED_EMPTY = 2,                // [2]
-  B_KV_FULL = 4,                    // [2] K', V landed
-  B_KV_EMPTY = 6,                   // [2] item's MMAs done with K', V
+  B_KV_FULL = 4,                    // K', V landed
+  B_KV_EMPTY = 5,                   // item's MMAs done with K', V
+  B_ST_FREE = 6,                    // S^T, dP^T read out of TMEM (8 warps)
   B_QG_FULL = 8,                    // [kQStages] Q', dO landed
   B_QG_READY = B_QG_FULL + kQStages,   // lse / D staged
   B_QG_EMPTY = B_QG_READY + kQStages,  // step's MMAs done with Q, dO
   B_SDP = B_QG_EMPTY + kQStages,    // S^T and dP^T in TMEM
-  B_PDS = B_SDP + 1,                // P^T, dS^T written (8 warps)
-  B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete
+  B_PDS = B_SDP + 1,                // P^T, dS^T written to shared memory (8 warps)
+  B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete (P^T, dS^T tiles free)
   B_DQ_FULL = B_STEP + 1,           // dQ of a step in TMEM
   B_DQ_EMPTY = B_DQ_FULL + 1,       // dQ read out (4 warps)
   B_ACC = B_DQ_EMPTY + 1,           // item's dK, dV complete
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   uint8_t *sV = smem + SmemOffsets::v;
   uint8_t *sQ = smem + SmemOffsets::q;
   uint8_t *sG = smem + SmemOffsets::g;
+  uint8_t *sP = smem + SmemOffsets::pt;
   uint8_t *sDS = smem + SmemOffsets::ds;
   float *sLse = reinterpret_cast<float *>(smem + SmemOffsets::lse);
   float *sDel = reinterpret_cast<float *>(smem + SmemOffsets::del);
@@ -242,9 +244,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     for (int i = 0; i < 2; ++i) {
       lcptx::mbar_init(ctx.bar(B_SCHED_FULL + i), 1);
       lcptx::mbar_init(ctx.bar(B_SCHED_EMPTY + i), kSchedConsumers);
-      lcptx::mbar_init(ctx.bar(B_KV_FULL + i), 1);
-      lcptx::mbar_init(ctx.bar(B_KV_EMPTY + i), 1);
     }
+    lcptx::mbar_init(ctx.bar(B_KV_FULL), 1);
+    lcptx::mbar_init(ctx.bar(B_KV_EMPTY), 1);
+    lcptx::mbar_init(ctx.bar(B_ST_FREE), kEwWarps);
     for (int s = 0; s < kQStages; ++s) {
       lcptx::mbar_init(ctx.bar(B_QG_FULL + s), 1);
       lcptx::mbar_init(ctx.bar(B_QG_READY + s), kRopeThreads);
@@ -296,22 +299,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         lcptx::mbar_arrive(ctx.bar(B_SCHED_FULL + slot));
         if (item < 0) break;
         const KItem it = decode_kitem(p, item);
-        const int kb = item_it & 1;
-        const uint32_t kph = (item_it >> 1) & 1;
-        bool ok = wait_bar(ctx, ctx.bar(B_KV_EMPTY + kb), kph ^ 1);
+        const uint32_t kph = item_it & 1;
+        bool ok = wait_bar(ctx, ctx.bar(B_KV_EMPTY), kph ^ 1);
         if (!ok) break;
         {
-          const uint32_t bar = ctx.bar(B_KV_FULL + kb);
+          const uint32_t bar = ctx.bar(B_KV_FULL);
           lcptx::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
-          const uint32_t dk = lcptx::smem_addr(sK + kb * kTileBytes);
-          const uint32_t dv = lcptx::smem_addr(sV + kb * kTileBytes);
+          const uint32_t dk = lcptx::smem_addr(sK);
+          const uint32_t dv = lcptx::smem_addr(sV);
           // rows past the segment end (a missing second block) read as zeros
           lcptx::tma_load_4d(dk, &p.tmK[it.seg], bar, 0, it.h, it.krow0, it.b);
           lcptx::tma_load_4d(dk + kBoxBytes, &p.tmK[it.seg], bar, 0, it.h, it.krow1, it.b);
           lcptx::tma_load_4d(dv, &p.tmV[it.seg], bar, 0, it.h, it.krow0, it.b);
           lcptx::tma_load_4d(dv + kBoxBytes, &p.tmV[it.seg], bar, 0, it.h, it.krow1, it.b);
-          kv_valid |= 1u << kb;
-          kv_par = (kv_par & ~(1u << kb)) | (kph << kb);
+          kv_valid = 1u;
+          kv_par = kph;
         }
         const int nsteps = (it.len + 1) >> 1;
         for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
@@ -342,8 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         ++item_it;
       }
       // Drain: every load this thread issued must land before the CTA exits.
-      for (int i = 0; i < 2; ++i)
-        if ((kv_valid >> i) & 1u) drain_wait(ctx.bar(B_KV_FULL + i), (kv_par >> i) & 1u, p.timeout_ns);
+      if (kv_valid) drain_wait(ctx.bar(B_KV_FULL), kv_par, p.timeout_ns);
       for (int s = 0; s < kQStages; ++s)
         if ((q_valid >> s) & 1u) drain_wait(ctx.bar(B_QG_FULL + s), (q_par >> s) & 1u, p.timeout_ns);
     }
@@ -351,8 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     // ======================= MMA issuer (one thread) =========================
     if (lane == 0) {
       uint32_t item_it = 0, q_it = 0, k_step = 0;
-      uint32_t pds_ph = 0, step_ph = 0;
-      bool step_pending = false;
+      uint32_t pds_ph = 0;
       constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
       constexpr uint32_t kTileLo = kTileBytes >> 4;
       auto desc = [](uint32_t lo) -> uint64_t {
@@ -369,6 +369,29 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const uint32_t q_mn = (lcptx::smem_addr(sQ) >> 4) | (512u << 16);
       const uint32_t g_mn = (lcptx::smem_addr(sG) >> 4) | (512u << 16);
       const uint32_t ds_mn = (lcptx::smem_addr(sDS) >> 4) | ((uint32_t)(kTileBytes >> 4) << 16);
+      const uint32_t pt_km = (lcptx::smem_addr(sP) >> 4) | (1u << 16);
+      const uint32_t ds_km = (lcptx::smem_addr(sDS) >> 4) | (1u << 16);
+      uint32_t st_free_ph = 0;
+      // S^T = K' Q'^T and dP^T = V dO^T of step q (stage s) into TMEM, once the
+      // previous step's S^T / dP^T have been read out.
+      auto issue_sdp = [&](int s, uint32_t ph, bool wait_free) -> bool {
+        if (!wait_bar(ctx, ctx.bar(B_QG_FULL + s), ph)) return false;
+        if (wait_free) {
+          if (!wait_bar(ctx, ctx.bar(B_ST_FREE), st_free_ph)) return false;
+          st_free_ph ^= 1;
+        }
+        lcptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          lcptx::mma_ss(tmem + kColST, desc(k_km + 2 * kk), desc(q_km + s * kTileLo + 2 * kk),
+                        kIdescKQ, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          lcptx::mma_ss(tmem + kColDPT, desc(v_km + 2 * kk), desc(g_km + s * kTileLo + 2 * kk),
+                        kIdescKQ, kk > 0);
+        lcptx::mma_commit(ctx.bar(B_SDP));
+        return true;
+      };
       for (;;) {
         const int slot = item_it & 1;
         if (!wait_bar(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
@@ -376,32 +399,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
         if (item < 0) break;
         const KItem it = decode_kitem(p, item);
-        const int kb = item_it & 1;
-        const uint32_t kph = (item_it >> 1) & 1;
-        bool ok = wait_bar(ctx, ctx.bar(B_KV_FULL + kb), kph);
+        bool ok = wait_bar(ctx, ctx.bar(B_KV_FULL), item_it & 1);
         const int nsteps = (it.len + 1) >> 1;
+        if (ok) ok = issue_sdp(q_it % kQStages, (q_it / kQStages) & 1, k_step > 0);
         for (int t = 0; t < nsteps && ok; ++t, ++q_it, ++k_step) {
           const int s = q_it % kQStages;
-          const uint32_t ph = (q_it / kQStages) & 1;
-          ok = wait_bar(ctx, ctx.bar(B_QG_FULL + s), ph);
-          if (!ok) break;
-          // S^T of this step overwrites P^T of the previous one: its P*V must be done.
-          if (step_pending) {
-            ok = wait_bar(ctx, ctx.bar(B_STEP), step_ph);
+          // the next step's S^T / dP^T overlap this step's elementwise pass
+          if (t + 1 < nsteps) {
+            ok = issue_sdp((q_it + 1) % kQStages, ((q_it + 1) / kQStages) & 1, true);
             if (!ok) break;
-            step_ph ^= 1;
-            step_pending = false;
           }
-          lcptx::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            lcptx::mma_ss(tmem + kColST, desc(k_km + kb * kTileLo + 2 * kk),
-                          desc(q_km + s * kTileLo + 2 * kk), kIdescKQ, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            lcptx::mma_ss(tmem + kColDPT, desc(v_km + kb * kTileLo + 2 * kk),
-                          desc(g_km + s * kTileLo + 2 * kk), kIdescKQ, kk > 0);
-          lcptx::mma_commit(ctx.bar(B_SDP));
           ok = wait_bar(ctx, ctx.bar(B_PDS), pds_ph);
           if (!ok) break;
           pds_ph ^= 1;
@@ -410,14 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             if (!ok) break;
           }
           lcptx::tc_fence_after();
-          // P^T / dS^T of query block h sit in columns [64 h, 64 h + 32) of S^T / dP^T
+          // dV += P^T dO, dK' += dS^T Q': A = the 64-query tiles in shared memory
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ts(tmem + kColDV, tmem + kColST + 64 * (kk >> 2) + 8 * (kk & 3),
+            lcptx::mma_ss(tmem + kColDV, desc(pt_km + (kk >> 2) * kTileLo + 2 * (kk & 3)),
                           desc(g_mn + s * kTileLo + 128 * kk), kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ts(tmem + kColDK, tmem + kColDPT + 64 * (kk >> 2) + 8 * (kk & 3),
+            lcptx::mma_ss(tmem + kColDK, desc(ds_km + (kk >> 2) * kTileLo + 2 * (kk & 3)),
                           desc(q_mn + s * kTileLo + 128 * kk), kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
           if (k_step > 0) {  // the dQ warps have read the previous step's dQ
             ok = wait_bar(ctx, ctx.bar(B_DQ_EMPTY), (k_step - 1) & 1);
@@ -426,15 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ss(tmem + kColDQ, desc(ds_mn + 128 * kk), desc(k_mn + kb * kTileLo + 128 * kk),
-                          kIdescDQ, kk > 0);
+            lcptx::mma_ss(tmem + kColDQ, desc(ds_mn + 128 * kk), desc(k_mn + 128 * kk), kIdescDQ,
+                          kk > 0);
           lcptx::mma_commit(ctx.bar(B_DQ_FULL));
           lcptx::mma_commit(ctx.bar(B_QG_EMPTY + s));
           lcptx::mma_commit(ctx.bar(B_STEP));
-          step_pending = true;
           if (t + 1 == nsteps) {
             lcptx::mma_commit(ctx.bar(B_ACC));
-            lcptx::mma_commit(ctx.bar(B_KV_EMPTY + kb));
+            lcptx::mma_commit(ctx.bar(B_KV_EMPTY));
           }
         }
         if (!ok) break;
@@ -617,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         uint8_t *tile = sDS + half * kTileBytes;  // dS^T, this query block's MN-major chunk
         // 16 queries at a time; the next chunk's TMEM loads are in flight while
         // this one is computed (double buffer)
+        uint8_t *ptile = sP + half * kTileBytes;  // P^T, this query block's tile
         uint32_t sr[2][16], dr[2][16];
         lcptx::tmem_ld16(tST + 64 * half, sr[0]);
         lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
@@ -627,6 +634,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           if (k < 3) {
             lcptx::tmem_ld16(tST + 64 * half + 16 * (k + 1), sr[(k + 1) & 1]);
             lcptx::tmem_ld16(tDPT + 64 * half + 16 * (k + 1), dr[(k + 1) & 1]);
+          } else {  // every TMEM load of the step has landed: S^T, dP^T may be overwritten
+            lcptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_ST_FREE));
           }
           const uint32_t(&scur)[16] = sr[k & 1];
           const uint32_t(&dcur)[16] = dr[k & 1];
@@ -646,19 +657,26 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             pp[i] = pack_bf16(pv[0], pv[1]);
             dd[i] = pack_bf16(dv2[0], dv2[1]);
           }
-          // P^T / dS^T of queries 16c..16c+15 go to columns 64 half + 8 k:
-          // inside this warp's own 64 columns, and already read
-          lcptx::tmem_st8(tST + 64 * half + 8 * k, pp);
-          lcptx::tmem_st8(tDPT + 64 * half + 8 * k, dd);
+          if (k == 0 && q_it > 0) {  // the previous step's MMAs are done with the tiles
+            ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
+            if (!ok) {
+              lcptx::tmem_wait_ld();  // nothing of this warp stays in flight
+              break;
+            }
+          }
+          // row kr of the P^T and dS^T tiles: 64 queries of this block, 128-byte
+          // swizzled; K-major for dV / dK, MN-major (dS) for dQ
 #pragma unroll
-          for (int i = 0; i < 2; ++i)
+          for (int i = 0; i < 2; ++i) {
+            *reinterpret_cast<uint4 *>(ptile + swz(kr, k * 2 + i)) =
+                make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
             *reinterpret_cast<uint4 *>(tile + swz(kr, k * 2 + i)) =
                 make_uint4(dd[4 * i], dd[4 * i + 1], dd[4 * i + 2], dd[4 * i + 3]);
+          }
           if (k < 3) lcptx::tmem_wait_ld();
         }
+        if (!ok) break;
         lcptx::fence_proxy_async_smem();
-        lcptx::tmem_wait_st();
-        lcptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));
       }

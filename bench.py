@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-extra", action="store_true", help="skip the 86,400-token line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward pass of --workload (one JSON line; for profiling)")
     return ap.parse_args()
 
 
@@ -218,7 +220,8 @@ def time_backward(api, synthetic, torch, name, steps, warmup, stream):
     return {"workload": name, "ms_per_layer": round(ms, 3),
             "attended_tflops": round(flops / (ms * 1e-3) / 1e12, 3),
             "work": "10*64 FLOP per attended pair and head",
-            "kernels": "bwd_delta, bsa_bwd_sm100_kernel (tcgen05), bwd_dq_finalize"}
+            "kernels": "rope_k_kernel (Q', K'), bwd_delta, bsa_bwd_sm100_kernel (tcgen05), "
+                       "bwd_grad_finalize"}
 
 
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):
@@ -489,6 +492,14 @@ def main():
     a = parse()
     if a.impl == "reference":
         run_reference(a)
+    elif a.backward_only:
+        import torch
+        torch.cuda.set_device(0)
+        from block_sparse_attention_rope_b200 import api, synthetic
+        r = time_backward(api, synthetic, torch, a.workload, a.steps, a.warmup,
+                          torch.cuda.current_stream())
+        print(json.dumps(dict(metric="backward ms per layer", value=r["ms_per_layer"], unit="ms",
+                              higher_is_better=False, **r)), flush=True)
     else:
         run_ours(a)
 

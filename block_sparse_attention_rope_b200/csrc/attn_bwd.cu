@@ -146,21 +146,59 @@ __device__ __forceinline__ void rotate_norm_transpose(const BwdArgs &a, float *g
   }
 }
 
-// D[b, h, n] = <dO_n, O_n>.
+// Eight consecutive values of a row (16 or 32 bytes) as fp32.
+__device__ __forceinline__ void ld8(const __nv_bfloat16 *p, float (&v)[8]) {
+  const uint4 raw = *reinterpret_cast<const uint4 *>(p);
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    v[2 * e] = __uint_as_float(w[e] << 16);
+    v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void ld8(const float *p, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void st8(__nv_bfloat16 *p, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    w[e] = *reinterpret_cast<uint32_t *>(&t);
+  }
+  *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+__device__ __forceinline__ void st8(float *p, const float (&v)[8]) {
+  reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// D[b, h, n] = <dO_n, O_n>; eight lanes per (batch, token, head) row, each
+// on one 8-channel chunk (coalesced vector loads), combined by shuffles.
 template <typename Tin>
 __global__ void bwd_delta_kernel(BwdArgs a, long long rows) {
-  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (i >= rows) return;
-  const int h = (int)(i % a.heads);
-  const long long bn = i / a.heads;  // b * N + n
-  const long long N = (long long)a.Nc + a.Nn;
-  const int n = (int)(bn % N), b = (int)(bn / N);
-  const Tin *o = static_cast<const Tin *>(a.o) + i * LC_HEAD_DIM;
-  const Tin *g = static_cast<const Tin *>(a.dout) + i * LC_HEAD_DIM;
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long i = gid >> 3;
+  const int ch = (int)(gid & 7);
+  if (i >= rows) return;  // rows are whole 8-lane groups: the group leaves together
+  const unsigned group = 0xFFu << (threadIdx.x & 24);
+  float o[8], g[8];
+  ld8(static_cast<const Tin *>(a.o) + i * LC_HEAD_DIM + 8 * ch, o);
+  ld8(static_cast<const Tin *>(a.dout) + i * LC_HEAD_DIM + 8 * ch, g);
   float acc = 0.f;
-#pragma unroll 16
-  for (int d = 0; d < LC_HEAD_DIM; ++d) acc = fmaf(ld(o, d), ld(g, d), acc);
-  a.delta[((long long)b * a.heads + h) * N + n] = acc;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc = fmaf(o[e], g[e], acc);
+  acc += __shfl_xor_sync(group, acc, 1);
+  acc += __shfl_xor_sync(group, acc, 2);
+  acc += __shfl_xor_sync(group, acc, 4);
+  if (ch == 0) {
+    const int h = (int)(i % a.heads);
+    const long long bn = i / a.heads;  // b * N + n
+    const long long N = (long long)a.Nc + a.Nn;
+    const int n = (int)(bn % N), b = (int)(bn / N);
+    a.delta[((long long)b * a.heads + h) * N + n] = acc;
+  }
 }
 
 // Shared memory rows are padded to 65 floats: a thread walking its own row
@@ -316,34 +354,53 @@ __global__ void __launch_bounds__(64) bwd_dkdv_kernel(BwdArgs a) {
   }
 }
 
-// g = norm^T(R^T acc) for one (batch, token, head) row per thread: dq from
-// the tensor-core path's fp32 dq sums (raw rows = q, weights = q's), or dk
-// from its fp32 dk' when k is normalised (raw rows = k).
+// g = norm^T(R^T acc) per (batch, token, head) row: dq from the tensor-core
+// path's fp32 dq sums (raw rows = q, weights = q's), or dk from its fp32 dk'
+// when k is normalised (raw rows = k).  Eight lanes per row, one 8-channel
+// chunk (4 RoPE pairs) each; the norm's row sums by shuffles.
 template <typename Tin>
 __global__ void bwd_grad_finalize_kernel(BwdArgs a, const float *acc, long long rows) {
-  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
-  if (i >= rows) return;
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long i = gid >> 3;
+  const int ch = (int)(gid & 7);
+  if (i >= rows) return;  // rows are whole 8-lane groups: the group leaves together
+  const unsigned group = 0xFFu << (threadIdx.x & 24);
   const long long N = (long long)a.Nc + a.Nn;
   const int n = (int)((i / a.heads) % N);
-  float g[LC_HEAD_DIM], x[LC_HEAD_DIM];
-  const float4 *src = reinterpret_cast<const float4 *>(acc + i * LC_HEAD_DIM);
+  float g[8];
+  ld8(acc + i * LC_HEAD_DIM + 8 * ch, g);
+  const Pos pos = decode(a, n);
 #pragma unroll
-  for (int c = 0; c < LC_HEAD_DIM / 4; ++c) {
-    const float4 v = src[c];
-    g[4 * c] = v.x; g[4 * c + 1] = v.y; g[4 * c + 2] = v.z; g[4 * c + 3] = v.w;
+  for (int q2 = 0; q2 < 4; ++q2) {  // R^T: turn each pair back
+    float c, sn;
+    pair_angle(a, pos, 4 * ch + q2, c, sn);
+    const float u = g[2 * q2], w = g[2 * q2 + 1];
+    g[2 * q2] = fmaf(u, c, w * sn);
+    g[2 * q2 + 1] = fmaf(w, c, -u * sn);
   }
-  const Tin *Q = static_cast<const Tin *>(a.q) + i * LC_HEAD_DIM;
+  if (a.q_nw) {  // y = x inv w:  dx = inv (w g) - x inv^3 / 64 * sum(g w x)
+    float x[8], w8[8];
+    ld8(static_cast<const Tin *>(a.q) + i * LC_HEAD_DIM + 8 * ch, x);
 #pragma unroll
-  for (int d = 0; d < LC_HEAD_DIM; ++d) x[d] = a.q_nw ? ld(Q, d) : 0.f;
-  rotate_norm_transpose(a, g, x, n, a.q_nw);
+    for (int e = 0; e < 8; ++e) w8[e] = __ldg(a.q_nw + 8 * ch + e);
+    const float inv = lc_rms_inv(lc_sumsq_lanes8(lc_sumsq8(x), group), a.norm_eps);
+    float dot = 0.f;
 #pragma unroll
-  for (int d = 0; d < LC_HEAD_DIM; ++d) st<Tin>(a.dq, i * LC_HEAD_DIM + d, g[d]);
+    for (int e = 0; e < 8; ++e) dot = fmaf(g[e] * w8[e], x[e], dot);
+    dot += __shfl_xor_sync(group, dot, 1);
+    dot += __shfl_xor_sync(group, dot, 2);
+    dot += __shfl_xor_sync(group, dot, 4);
+    const float k3 = inv * inv * inv * (1.f / LC_HEAD_DIM) * dot;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g[e] = inv * w8[e] * g[e] - x[e] * k3;
+  }
+  st8(static_cast<Tin *>(a.dq) + i * LC_HEAD_DIM + 8 * ch, g);
 }
 
 template <typename Tin>
 lc_status launch_all(const BwdArgs &a, int batch, int nq, cudaStream_t st) {
   const long long rows = (long long)batch * (a.Nc + a.Nn) * a.heads;
-  bwd_delta_kernel<Tin><<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(a, rows);
+  bwd_delta_kernel<Tin><<<(unsigned)((rows * 8 + 255) / 256), 256, 0, st>>>(a, rows);
   dim3 grid(nq, a.heads, batch);
   LC_CUDA_TRY(cudaFuncSetAttribute(bwd_dq_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kBwdSmem));
@@ -364,10 +421,11 @@ lc_status lc_bwd_delta(const void *out, const void *dout, float *delta, int batc
   a.Nc = 0; a.Nn = (int)N;
   const long long rows = (long long)batch * N * heads;
   if (rows == 0) return LC_OK;
+  const unsigned grid = (unsigned)((rows * 8 + 255) / 256);  // 8 lanes per row
   if (dtype == LC_DTYPE_F32)
-    bwd_delta_kernel<float><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a, rows);
+    bwd_delta_kernel<float><<<grid, 256, 0, stream>>>(a, rows);
   else
-    bwd_delta_kernel<__nv_bfloat16><<<(unsigned)((rows + 255) / 256), 256, 0, stream>>>(a, rows);
+    bwd_delta_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a, rows);
   return lc_from_cuda(cudaGetLastError());
 }
 
@@ -384,11 +442,11 @@ lc_status lc_bwd_grad_finalize(const float *acc, const void *raw, void *grad, in
   a.div_w = lc_make_divmod(rope->W);
   const long long rows = (long long)batch * N * heads;
   if (rows == 0) return LC_OK;
-  const unsigned grid = (unsigned)((rows + 127) / 128);
+  const unsigned grid = (unsigned)((rows * 8 + 255) / 256);  // 8 lanes per row
   if (dtype == LC_DTYPE_F32)
-    bwd_grad_finalize_kernel<float><<<grid, 128, 0, stream>>>(a, acc, rows);
+    bwd_grad_finalize_kernel<float><<<grid, 256, 0, stream>>>(a, acc, rows);
   else
-    bwd_grad_finalize_kernel<__nv_bfloat16><<<grid, 128, 0, stream>>>(a, acc, rows);
+    bwd_grad_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(a, acc, rows);
   return lc_from_cuda(cudaGetLastError());
 }
 

@@ -68,6 +68,11 @@ def _load():
                                 vp]),
         "lc_bsa_plan_copy_csc": (S, [vp, vp, vp, vp]),
         "lc_bsa_forward_noalloc": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp]),
+        "lc_bsa_plan_create_shard": (S, [ctypes.POINTER(vp), I, I, I, I, I, I, I, I, I, I, I,
+                                         vp]),
+        "lc_bsa_plan_token_range": (S, [vp] + [ctypes.POINTER(LL)] * 4),
+        "lc_bsa_forward_shard": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp, vp]),
+        "lc_bsa_lse_merge": (S, [vp, vp, vp, vp, vp, I, LL, I, I, I, ctypes.c_uint, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
         "lc_status_string": (ctypes.c_char_p, [S]),
@@ -126,16 +131,33 @@ def _check_bmhk(name: str, t: torch.Tensor, shape, dtype):
 
 
 class Plan:
-    """Device-resident block-sparse plan (lc_bsa_plan_create)."""
+    """Device-resident block-sparse plan (lc_bsa_plan_create), or, with
+    q_blocks / k_blocks, the plan of one shard pair of ring context
+    parallelism (lc_bsa_plan_create_shard): query blocks [lo, hi) against key
+    blocks [lo, hi)."""
 
     def __init__(self, T: int, H: int, W: int, *, local: int, stride: int, n_cond: int = 0,
-                 block: int = 64, stream=None):
+                 block: int = 64, q_blocks: Optional[Tuple[int, int]] = None,
+                 k_blocks: Optional[Tuple[int, int]] = None, stream=None):
         self.T, self.H, self.W, self.n_cond = T, H, W, n_cond
         self.local, self.stride, self.block = local, stride, block
         h = ctypes.c_void_p()
-        _check(lib.lc_bsa_plan_create(ctypes.byref(h), T, H, W, block, local, stride, n_cond,
-                                      _stream(stream)), "lc_bsa_plan_create")
+        if q_blocks is None and k_blocks is None:
+            _check(lib.lc_bsa_plan_create(ctypes.byref(h), T, H, W, block, local, stride, n_cond,
+                                          _stream(stream)), "lc_bsa_plan_create")
+        else:
+            if q_blocks is None or k_blocks is None:
+                raise ValueError("q_blocks and k_blocks go together")
+            _check(lib.lc_bsa_plan_create_shard(ctypes.byref(h), T, H, W, block, local, stride,
+                                                n_cond, int(q_blocks[0]), int(q_blocks[1]),
+                                                int(k_blocks[0]), int(k_blocks[1]),
+                                                _stream(stream)), "lc_bsa_plan_create_shard")
         self.handle = h
+        r = [ctypes.c_longlong() for _ in range(4)]
+        _check(lib.lc_bsa_plan_token_range(self.handle, *[ctypes.byref(x) for x in r]),
+               "lc_bsa_plan_token_range")
+        self.q_tokens = (r[0].value, r[1].value)  # whole-sequence token range of the queries
+        self.k_tokens = (r[2].value, r[3].value)  # and of the keys
 
     def info(self) -> PlanInfo:
         inf = PlanInfo()
@@ -390,6 +412,59 @@ def forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Pla
                                       float(softmax_scale), plan.handle, rope.handle,
                                       _stream(stream)), "lc_bsa_forward_noalloc")
     return out
+
+
+def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D,
+                  *, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                  softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
+                  k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None):
+    """Partial attention of one shard pair (lc_bsa_forward_shard): q holds the
+    shard plan's query tokens [B, nq, heads, 64], k / v its key tokens
+    [B, nk, heads, 64] (pre-RoPE, bf16).  Returns (out, lse); rows that attend
+    no key of the shard get out 0 and lse -inf."""
+    B, nq, heads, hd = q.shape
+    nk = plan.k_tokens[1] - plan.k_tokens[0]
+    _check_bmhk("q", q, (B, plan.q_tokens[1] - plan.q_tokens[0], heads, hd), q.dtype)
+    for name, t in (("k", k), ("v", v)):
+        _check_bmhk(name, t, (B, nk, heads, hd), q.dtype)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, heads, nq, dtype=torch.float32, device=q.device)
+    _check_bmhk("out", out, q.shape, q.dtype)
+    _check_bmhk("lse", lse, (B, heads, nq), torch.float32)
+    opts = _opts(0, q_norm, k_norm, norm_eps, hd)
+    _check(lib.lc_bsa_forward_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, heads, hd, _dtype_code(q),
+                                    float(softmax_scale),
+                                    None if opts is None else ctypes.byref(opts), plan.handle,
+                                    rope.handle, _stream(stream)), "lc_bsa_forward_shard")
+    return out, lse
+
+
+MERGE_INIT = 1  # LC_MERGE_INIT
+
+
+def lse_merge(o_acc: Optional[torch.Tensor], lse_acc: torch.Tensor, o_part: torch.Tensor,
+              lse_part: torch.Tensor, *, out: Optional[torch.Tensor] = None, init: bool = False,
+              stream=None):
+    """Fold a partial result (o_part [B, n, heads, 64] bf16/fp32, lse_part
+    [B, heads, n]) into a running one (o_acc fp32, lse_acc) by log-sum-exp
+    (lc_bsa_lse_merge).  With `out` the merged o goes there (rounded to
+    o_part's dtype) instead of o_acc; with init the running result is not read."""
+    B, n, heads, hd = o_part.shape
+    _check_bmhk("o_part", o_part, o_part.shape, o_part.dtype)
+    _check_bmhk("lse_part", lse_part, (B, heads, n), torch.float32)
+    _check_bmhk("lse_acc", lse_acc, (B, heads, n), torch.float32)
+    if o_acc is not None:
+        _check_bmhk("o_acc", o_acc, o_part.shape, torch.float32)
+    if out is not None:
+        _check_bmhk("out", out, o_part.shape, o_part.dtype)
+    _check(lib.lc_bsa_lse_merge(_ptr(o_acc), lse_acc.data_ptr(), o_part.data_ptr(),
+                                lse_part.data_ptr(), _ptr(out), B, n, heads, hd,
+                                _dtype_code(o_part), MERGE_INIT if init else 0, _stream(stream)),
+           "lc_bsa_lse_merge")
+    return out if out is not None else o_acc
 
 
 def last_device_status(stream=None) -> int:

@@ -12,10 +12,12 @@ int *g_status[kMaxDevices] = {nullptr};
 
 bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+// A shard plan is accepted by lc_bsa_forward_shard only (allow_shard).
 lc_status check_common(const lc_bsa_plan_s *plan, const lc_rope3d_s *rope, int batch, int heads,
-                       int head_dim, lc_dtype dtype) {
+                       int head_dim, lc_dtype dtype, bool allow_shard = false) {
   if (!plan || !rope || batch <= 0 || heads <= 0 || head_dim <= 0)
     return LC_ERR_INVALID_ARGUMENT;
+  if (!allow_shard && lc_plan_is_shard(plan)) return LC_ERR_INVALID_ARGUMENT;
   if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
   if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
   if (plan->T != rope->T || plan->H != rope->H || plan->W != rope->W)
@@ -261,6 +263,59 @@ extern "C" lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const 
   return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale,
                                  LC_FWD_FULL, false, lc_qk_norm(), plan, rope, scratch + 1, st,
                                  scratch);
+}
+
+extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void *out,
+                                          float *lse, int batch, int heads, int head_dim,
+                                          lc_dtype dtype, float softmax_scale,
+                                          const lc_bsa_opts *opts, lc_bsa_plan plan,
+                                          lc_rope3d rope, void *stream) {
+  lc_status s = check_common(plan, rope, batch, heads, head_dim, dtype, true);
+  if (s != LC_OK) return s;
+  unsigned flags;
+  lc_qk_norm norm;
+  if (!parse_opts(opts, 0u, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
+  if (!q || !k || !v || !out || !lse) return LC_ERR_INVALID_ARGUMENT;
+  if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return LC_ERR_INVALID_ARGUMENT;
+  if (!(softmax_scale == softmax_scale)) return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16) return LC_ERR_UNSUPPORTED;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 0.125f;
+  lc_shard_view sv;
+  sv.q_lo = lc_block_token(plan, plan->qlo);
+  sv.q_n = lc_block_token(plan, plan->qhi) - sv.q_lo;
+  sv.k_lo = lc_block_token(plan, plan->klo);
+  sv.k_n = lc_block_token(plan, plan->khi) - sv.k_lo;
+  if (sv.q_n == 0) return LC_OK;
+  int *dev_status = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Rows of groups without entries (out = 0, lse = -inf); the kernel writes the rest.
+  s = lc_launch_shard_fill(plan, out, lse, batch, heads, dtype, st);
+  if (s != LC_OK || plan->G_active == 0) return s;
+  return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale,
+                                 LC_FWD_SHARD, false, norm, plan, rope, dev_status, st, nullptr,
+                                 &sv);
+}
+
+extern "C" lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
+                                      const float *lse_part, void *out, int batch,
+                                      long long n_tokens, int heads, int head_dim, lc_dtype dtype,
+                                      unsigned flags, void *stream) {
+  if (batch <= 0 || heads <= 0 || head_dim <= 0 || n_tokens < 0) return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
+  if (flags & ~(unsigned)LC_MERGE_INIT) return LC_ERR_INVALID_ARGUMENT;
+  if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
+  const bool init = (flags & LC_MERGE_INIT) != 0;
+  if (!lse_acc || !o_part || !lse_part || (!o_acc && !(init && out)))
+    return LC_ERR_INVALID_ARGUMENT;
+  if (misaligned(o_acc) || misaligned(o_part) || misaligned(out) ||
+      ((reinterpret_cast<uintptr_t>(lse_acc) | reinterpret_cast<uintptr_t>(lse_part)) & 3u))
+    return LC_ERR_INVALID_ARGUMENT;
+  if ((long long)batch * n_tokens * heads >= (1LL << 40)) return LC_ERR_UNSUPPORTED;
+  return lc_launch_lse_merge(o_acc, lse_acc, o_part, lse_part, out, batch, n_tokens, heads, dtype,
+                             init, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" lc_status lc_last_device_status(void *stream) {

@@ -113,7 +113,9 @@ struct __align__(64) Sm100Params {
   int heads, n_groups_active, total_items;
   int group_offset;        // first rank of grp_order this launch works on
   int lse_nq;              // rows of the lse tensor per (batch, head)
-  int q_row_offset_noisy;  // row of the q/out/lse tensors holding noisy token 0
+  int lse_base[2];         // lse row of segment row 0, per segment ([0] condition, [1] noisy)
+  int q_row_off[2];        // row of the q/out maps' row 0 within its segment (shards)
+  int k_row_off[2];        // same for the k/v maps
   int tab_floats;
   int k_prerotated;        // K tensors already hold R(k): skip the K rotation
   float scale_log2;
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           const uint32_t bq = ctx.bar(B_QFULL + qi);
           lcptx::mbar_arrive_expect_tx(bq, kTileBytes);
           const uint32_t dst = lcptx::smem_addr(sQ + qi * kTileBytes);
-          const int r = it.row0 + 128 * i;
+          const int r = it.row0 + 128 * i - p.q_row_off[it.seg];
           lcptx::tma_load_4d(dst, &p.tmQ[it.seg], bq, 0, it.h, r, it.b);
           lcptx::tma_load_4d(dst + kBoxBytes, &p.tmQ[it.seg], bq, 0, it.h, r + 64, it.b);
           q_valid |= 1u << qi;
@@ -416,11 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           const uint32_t ph = (kv_it / kStages) & 1;
           int sa, ra, na, sb, rb, nb;
           entry_block(p, __ldg(it.ent + 2 * t), sa, ra, na);
+          ra -= p.k_row_off[sa];
           if (2 * t + 1 < it.len) {
             entry_block(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
-          } else {  // no second block: a box entirely past the segment end reads zeros
+            rb -= p.k_row_off[sb];
+          } else {  // no second block: a box far past every map's end reads zeros
             sb = 1;
-            rb = p.Nn;
+            rb = 1 << 24;
           }
           ok = wait_bar(ctx, ctx.bar(B_KEMPTY + s), ph ^ 1);
           if (!ok) break;
@@ -816,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       lcptx::tc_fence_before();
       const int qrow = it.row0 + 128 * wg + row;  // row within the segment
       if (p.lse && qrow < it.seg_len) {
-        const int out_row = (it.seg ? p.q_row_offset_noisy : 0) + qrow;
+        const int out_row = p.lse_base[it.seg] + qrow;
         p.lse[((long long)it.b * p.heads + it.h) * p.lse_nq + out_row] =
             ((m_ref == -INFINITY ? 0.f : m_ref) + __log2f(l_sum)) * 0.69314718055994530942f;
       }
@@ -826,10 +830,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         ok = wait_bar(ctx, ctx.bar(B_EPI + wg), item_it & 1);
         if (ok) {
           const uint32_t src = lcptx::smem_addr(stage);
-          const int r0 = it.row0 + 128 * wg;
-          if (r0 < it.seg_len) lcptx::tma_store_4d(&p.tmO[it.seg], src, 0, it.h, r0, it.b);
+          const int r0 = it.row0 + 128 * wg;  // row within the segment
+          const int c0 = r0 - p.q_row_off[it.seg];  // row of the out map (>= 0: groups lie in the shard)
+          if (r0 < it.seg_len) lcptx::tma_store_4d(&p.tmO[it.seg], src, 0, it.h, c0, it.b);
           if (r0 + 64 < it.seg_len)
-            lcptx::tma_store_4d(&p.tmO[it.seg], src + kBoxBytes, 0, it.h, r0 + 64, it.b);
+            lcptx::tma_store_4d(&p.tmO[it.seg], src + kBoxBytes, 0, it.h, c0 + 64, it.b);
           lcptx::bulk_commit_group();
           lcptx::bulk_wait_group_read0();
           lcptx::mbar_arrive(ctx.bar(B_QEMPTY + 2 * buf + wg));
@@ -1027,20 +1032,53 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
                                   float scale, lc_fwd_mode mode, bool cond_k_rotated,
                                   const lc_qk_norm &norm, const lc_bsa_plan_s *plan,
                                   const lc_rope3d_s *rope, int *dev_status, cudaStream_t stream,
-                                  int *counter_scratch) {
+                                  int *counter_scratch, const lc_shard_view *shard) {
   Sm100Params prm;
   memset(&prm, 0, sizeof(prm));
   const long long Nc = plan->Nc, Nn = plan->Nn, N = Nc + Nn;
   const bool cached = mode == LC_FWD_CACHED, cond_only = mode == LC_FWD_COND;
+  const bool sharded = mode == LC_FWD_SHARD;
   if (counter_scratch && mode != LC_FWD_FULL) return LC_ERR_UNSUPPORTED;
+  if (sharded != (shard != nullptr)) return LC_ERR_INVALID_ARGUMENT;
   if (cond_only && Nc == 0) return LC_OK;
   lc_status s = LC_OK;
-  if (cond_only) {  // condition queries over condition keys only
+  // Shard maps: per segment, the part of a shard buffer (tokens [lo, lo + n))
+  // that lies in the segment; row_off[seg] = that part's first row counted
+  // from the segment start (the kernel subtracts it from segment rows).
+  const long long seg_lo[2] = {0, Nc}, seg_hi[2] = {Nc, N};
+  auto encode_shard = [&](CUtensorMap *maps, const void *base, long long lo, long long n,
+                          int *row_off) -> lc_status {
+    bool have[2] = {false, false};
+    for (int sg = 0; sg < 2; ++sg) {
+      const long long a = lo > seg_lo[sg] ? lo : seg_lo[sg];
+      const long long b = lo + n < seg_hi[sg] ? lo + n : seg_hi[sg];
+      if (a >= b) continue;
+      lc_status r = encode_segment(&maps[sg], base, batch, n, a - lo, b - a, heads);
+      if (r != LC_OK) return r;
+      if (row_off) row_off[sg] = (int)(a - seg_lo[sg]);
+      have[sg] = true;
+    }
+    if (!have[0] && !have[1]) return LC_ERR_INVALID_ARGUMENT;
+    if (!have[0]) maps[0] = maps[1];  // unused segment: a valid descriptor, never read
+    if (!have[1]) maps[1] = maps[0];
+    return LC_OK;
+  };
+  if (sharded) {
+    s = encode_shard(prm.tmQ, q, shard->q_lo, shard->q_n, prm.q_row_off);
+    if (s == LC_OK) s = encode_shard(prm.tmO, out, shard->q_lo, shard->q_n, nullptr);
+    if (s == LC_OK) s = encode_shard(prm.tmK, k, shard->k_lo, shard->k_n, prm.k_row_off);
+    if (s == LC_OK) s = encode_shard(prm.tmV, v, shard->k_lo, shard->k_n, nullptr);
+    prm.lse_base[0] = (int)(seg_lo[0] - shard->q_lo);
+    prm.lse_base[1] = (int)(seg_lo[1] - shard->q_lo);
+    prm.lse_nq = (int)shard->q_n;
+    prm.group_offset = 0;
+    prm.n_groups_active = plan->G_active;  // groups with entries rank first
+  } else if (cond_only) {  // condition queries over condition keys only
     s = encode_segment(&prm.tmQ[0], q, batch, Nc, 0, Nc, heads);
     if (s == LC_OK) s = encode_segment(&prm.tmO[0], out, batch, Nc, 0, Nc, heads);
     if (s == LC_OK) s = encode_segment(&prm.tmK[0], cond_k, batch, Nc, 0, Nc, heads);
     if (s == LC_OK) s = encode_segment(&prm.tmV[0], cond_v, batch, Nc, 0, Nc, heads);
-    prm.q_row_offset_noisy = 0;
+    prm.lse_base[0] = 0;
     prm.lse_nq = (int)Nc;
     // grp_order ranks noisy groups first (every noisy list holds all Cb
     // condition blocks plus at least one noisy block, so it is longer than
@@ -1056,7 +1094,7 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
       s = encode_segment(&prm.tmK[0], cond_k, batch, Nc, 0, Nc, heads);
       if (s == LC_OK) s = encode_segment(&prm.tmV[0], cond_v, batch, Nc, 0, Nc, heads);
     }
-    prm.q_row_offset_noisy = 0;
+    prm.lse_base[1] = 0;
     prm.lse_nq = (int)Nn;
     prm.group_offset = 0;
     prm.n_groups_active = plan->gn;
@@ -1071,13 +1109,16 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
       if (s == LC_OK) s = encode_segment(&prm.tmK[0], k, batch, N, 0, Nc, heads);
       if (s == LC_OK) s = encode_segment(&prm.tmV[0], v, batch, N, 0, Nc, heads);
     }
-    prm.q_row_offset_noisy = (int)Nc;
+    prm.lse_base[0] = 0;
+    prm.lse_base[1] = (int)Nc;
     prm.lse_nq = (int)N;
     prm.group_offset = 0;
     prm.n_groups_active = plan->G;
   }
   if (s != LC_OK) return s;
-  if (cond_only) {  // keep the unused noisy maps valid descriptors
+  if (sharded) {
+    // encode_shard filled every map
+  } else if (cond_only) {  // keep the unused noisy maps valid descriptors
     prm.tmQ[1] = prm.tmQ[0]; prm.tmK[1] = prm.tmK[0];
     prm.tmV[1] = prm.tmV[0]; prm.tmO[1] = prm.tmO[0];
   } else if (Nc == 0) {  // keep the unused condition maps valid descriptors
@@ -1153,13 +1194,14 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   cudaError_t e = cudaStreamWaitEvent(stream, rope->ready, 0);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, plan->ready, 0);
   if (e == cudaSuccess && k_prepass) {
-    // K of the query-side tensor (all tokens, or the noisy ones).
+    // K of the query-side tensor (all tokens, the noisy ones, or the shard's).
     if (!cond_only) {
-      const size_t kb = (size_t)batch * (cached ? Nn : N) * heads * LC_HEAD_DIM * 2;
-      e = cudaMallocFromPoolAsync(&k_rot, kb, pool, stream);
+      const long long kn = sharded ? shard->k_n : (cached ? Nn : N);
+      const int k_tok0 = sharded ? (int)shard->k_lo : (cached ? (int)Nc : 0);
+      e = cudaMallocFromPoolAsync(&k_rot, (size_t)batch * kn * heads * LC_HEAD_DIM * 2, pool,
+                                  stream);
       if (e == cudaSuccess)
-        s = launch_rope_k(k, k_rot, batch, cached ? Nn : N, heads, cached ? (int)Nc : 0, rope,
-                          stream, norm.k_w, norm.eps);
+        s = launch_rope_k(k, k_rot, batch, kn, heads, k_tok0, rope, stream, norm.k_w, norm.eps);
     }
     // Separately supplied condition K, unless the caller rotated it already.
     if (e == cudaSuccess && s == LC_OK && (cached || cond_only) && Nc > 0 && !cond_k_rotated) {
@@ -1170,7 +1212,9 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
     }
     if (e == cudaSuccess && s == LC_OK) {
       if (ck_rot) s = encode_segment(&prm.tmK[0], ck_rot, batch, Nc, 0, Nc, heads);
-      if (cond_only) {
+      if (sharded) {
+        s = encode_shard(prm.tmK, k_rot, shard->k_lo, shard->k_n, prm.k_row_off);
+      } else if (cond_only) {
         prm.tmK[1] = prm.tmK[0];
       } else if (cached) {
         if (s == LC_OK) s = encode_segment(&prm.tmK[1], k_rot, batch, Nn, 0, Nn, heads);

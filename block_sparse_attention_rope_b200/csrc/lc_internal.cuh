@@ -27,6 +27,8 @@ struct lc_bsa_plan_s {
   int T, H, W, block, local, stride, n_cond;
   int Nc, Nn, Cb, Nb, nq;
   int gc, gn, G;            // groups in the condition / noisy segment, total
+  int qlo, qhi, klo, khi;   // block ranges the plan covers (a shard plan: part of the pattern)
+  int G_active;             // groups with at least one entry (the first G_active of grp_order)
   long long nnz;            // CSR entries (host closed form, checked on device)
   int device;
   cudaEvent_t ready;        // recorded after the planner kernels
@@ -57,6 +59,18 @@ struct lc_bsa_plan_s {
   long long pairs_host[2];
   bool info_cached;
 };
+
+// A plan restricted to part of the pattern (lc_bsa_plan_create_shard).
+inline bool lc_plan_is_shard(const lc_bsa_plan_s *p) {
+  return p->qlo != 0 || p->qhi != p->nq || p->klo != 0 || p->khi != p->nq;
+}
+// First token of block r in the whole sequence (r == nq: the token count).
+inline long long lc_block_token(const lc_bsa_plan_s *p, int r) {
+  const long long t = r < p->Cb ? (long long)LC_BLOCK * r
+                                : (long long)p->Nc + (long long)LC_BLOCK * (r - p->Cb);
+  const long long n = (long long)p->Nc + p->Nn;
+  return t < n ? t : n;
+}
 
 // RoPE tables: fp32 [cos_t T*dt/2][sin_t][cos_h H*dh/2][sin_h][cos_w W*dw/2][sin_w].
 struct lc_rope3d_s {
@@ -152,8 +166,15 @@ __device__ __forceinline__ float lc_rms_apply(float x, float inv, float w) {
 //                  tokens' K/V come from cond_k / cond_v ([B, Nc, heads, 64]).
 //   LC_FWD_COND    only the condition queries: q and out hold the Nc condition
 //                  tokens, K/V come from cond_k / cond_v (k and v unused).
+//   LC_FWD_SHARD   one shard of the whole-sequence attention (context
+//                  parallelism): q and out hold tokens [q_lo, q_lo + q_n), k
+//                  and v tokens [k_lo, k_lo + k_n) (lc_shard_view); the plan
+//                  is a shard plan over those blocks (bf16 only).
 // cond_k_rotated: cond_k already holds R(k) (CACHED and COND only).
-enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2 };
+enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2, LC_FWD_SHARD = 3 };
+struct lc_shard_view {
+  long long q_lo, q_n, k_lo, k_n;
+};
 
 // RMSNorm of q and k ahead of the rotation: device fp32 weights [64] or NULL.
 struct lc_qk_norm {
@@ -177,7 +198,16 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v,
                                   bool cond_k_rotated, const lc_qk_norm &norm,
                                   const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
                                   int *dev_status, cudaStream_t stream,
-                                  int *counter_scratch = nullptr);
+                                  int *counter_scratch = nullptr,
+                                  const lc_shard_view *shard = nullptr);
+// Context parallelism pieces (ring.cu): rows of a shard plan's query range
+// that no launch writes (groups without entries) get out = 0, lse = -inf;
+// the online-softmax merge of a partial result into a running one.
+lc_status lc_launch_shard_fill(const lc_bsa_plan_s *plan, void *out, float *lse, int batch,
+                               int heads, lc_dtype dtype, cudaStream_t stream);
+lc_status lc_launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
+                              const float *lse_part, void *out, int batch, long long n, int heads,
+                              lc_dtype dtype, bool init, cudaStream_t stream);
 // Gradients dq, dk, dv of the whole-sequence attention (attn_bwd.cu).
 lc_status lc_launch_backward(const void *q, const void *k, const void *v, const void *out,
                              const float *lse, const void *dout, void *dq, void *dk, void *dv,

@@ -28,9 +28,13 @@ namespace {
 struct PlanGeom {
   int Nc, Nn, Cb, Nb, nq, gc, gn, G, local, stride;
   int kgc, kgn, KG;  // key groups of 2 blocks (backward)
+  int qlo, qhi, klo, khi;  // the plan covers query blocks [qlo, qhi) x key blocks [klo, khi)
 };
 
-__device__ __forceinline__ bool attends(int r, int c, const PlanGeom &g) {
+// The pattern (query block r attends key block c), restricted to the plan's
+// block ranges.  Same rule on the host (sizing) and the device.
+__host__ __device__ __forceinline__ bool attends(int r, int c, const PlanGeom &g) {
+  if (r < g.qlo || r >= g.qhi || c < g.klo || c >= g.khi) return false;
   if (r < g.Cb) return c < g.Cb;
   if (c < g.Cb) return true;
   int i = r - g.Cb, j = c - g.Cb;
@@ -365,8 +369,10 @@ T *carve(char *&p, long long n) {
 
 }  // namespace
 
-extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, int block,
-                                        int local, int stride, int n_cond_frames, void *stream) {
+// Builds the plan of query blocks [qlo, qhi) against key blocks [klo, khi)
+// (qhi / khi < 0: through the last block).
+static lc_status plan_create(lc_bsa_plan *out, int T, int H, int W, int block, int local, int stride,
+                      int n_cond_frames, int qlo, int qhi, int klo, int khi, void *stream) {
   if (!out || T <= 0 || H <= 0 || W <= 0 || local < 0 || n_cond_frames < 0 ||
       n_cond_frames >= T || block <= 0)
     return LC_ERR_INVALID_ARGUMENT;
@@ -397,8 +403,46 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
     p->kgn = (p->Nb + 1) / 2;
   }
   p->KG = p->kgc + p->kgn;
-  long long nnz = (long long)p->Cb * p->Cb + (long long)p->Nb * p->Cb;
-  for (long long i = 0; i < p->Nb; ++i) nnz += noisy_row_count(i, p->Nb, local, stride);
+  if (qhi < 0) qhi = p->nq;
+  if (khi < 0) khi = p->nq;
+  if (qlo < 0 || klo < 0 || qlo > qhi || klo > khi || qhi > p->nq || khi > p->nq) {
+    delete p;
+    return LC_ERR_INVALID_ARGUMENT;
+  }
+  // Shard query ranges start and end on group boundaries (4 blocks within a
+  // segment, or a segment end), so every group lies wholly inside or outside.
+  auto group_edge = [&](int b) {
+    return b == p->Cb || b == p->nq || (b < p->Cb ? b % 4 == 0 : (b - p->Cb) % 4 == 0);
+  };
+  if (!group_edge(qlo) || !group_edge(qhi)) {
+    delete p;
+    return LC_ERR_INVALID_ARGUMENT;
+  }
+  p->qlo = qlo; p->qhi = qhi; p->klo = klo; p->khi = khi;
+  PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride,
+             p->kgc, p->kgn, p->KG, qlo, qhi, klo, khi};
+  long long nnz = 0;
+  p->G_active = p->G;
+  if (qlo == 0 && qhi == p->nq && klo == 0 && khi == p->nq) {  // closed form
+    nnz = (long long)p->Cb * p->Cb + (long long)p->Nb * p->Cb;
+    for (long long i = 0; i < p->Nb; ++i) nnz += noisy_row_count(i, p->Nb, local, stride);
+  } else {  // a shard: count on the host (block pairs; groups with any pair)
+    p->G_active = 0;
+    for (int gi = 0; gi < p->G; ++gi) {
+      const int first = gi < p->gc ? 4 * gi : p->Cb + 4 * (gi - p->gc);
+      const int cnt = gi < p->gc ? std::min(4, p->Cb - 4 * gi) : std::min(4, p->Nb - 4 * (gi - p->gc));
+      bool any = false;
+      for (int r = first; r < first + cnt; ++r) {
+        if (r < qlo || r >= qhi) continue;
+        for (int c = klo; c < khi; ++c)
+          if (attends(r, c, g)) {
+            ++nnz;
+            any = true;
+          }
+      }
+      p->G_active += any ? 1 : 0;
+    }
+  }
   p->nnz = nnz;
   if (nnz >= (1LL << 31)) { delete p; return LC_ERR_INVALID_ARGUMENT; }
 
@@ -434,8 +478,6 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
   p->kgrp_order = carve<int>(q, p->KG);
   p->kgrp_blk = carve<int2>(q, p->KG);
 
-  PlanGeom g{p->Nc, p->Nn, p->Cb, p->Nb, p->nq, p->gc, p->gn, p->G, local, stride,
-             p->kgc, p->kgn, p->KG};
   e = cudaMemsetAsync(p->pairs, 0, 2 * sizeof(unsigned long long), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(p->err, 0, sizeof(int), st);
   const int tpb = 256;
@@ -466,6 +508,30 @@ extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, i
     return lc_from_cuda(e);
   }
   *out = p;
+  return LC_OK;
+}
+
+extern "C" lc_status lc_bsa_plan_create(lc_bsa_plan *out, int T, int H, int W, int block,
+                                        int local, int stride, int n_cond_frames, void *stream) {
+  return plan_create(out, T, H, W, block, local, stride, n_cond_frames, 0, -1, 0, -1, stream);
+}
+
+extern "C" lc_status lc_bsa_plan_create_shard(lc_bsa_plan *out, int T, int H, int W, int block,
+                                              int local, int stride, int n_cond_frames,
+                                              int q_block_lo, int q_block_hi, int k_block_lo,
+                                              int k_block_hi, void *stream) {
+  if (q_block_hi < 0 || k_block_hi < 0) return LC_ERR_INVALID_ARGUMENT;
+  return plan_create(out, T, H, W, block, local, stride, n_cond_frames, q_block_lo, q_block_hi,
+                     k_block_lo, k_block_hi, stream);
+}
+
+extern "C" lc_status lc_bsa_plan_token_range(lc_bsa_plan plan, long long *q_lo, long long *q_hi,
+                                             long long *k_lo, long long *k_hi) {
+  if (!plan || !q_lo || !q_hi || !k_lo || !k_hi) return LC_ERR_INVALID_ARGUMENT;
+  *q_lo = lc_block_token(plan, plan->qlo);
+  *q_hi = lc_block_token(plan, plan->qhi);
+  *k_lo = lc_block_token(plan, plan->klo);
+  *k_hi = lc_block_token(plan, plan->khi);
   return LC_OK;
 }
 

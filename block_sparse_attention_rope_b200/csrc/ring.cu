@@ -1,0 +1,151 @@
+// ring.cu -- device pieces of ring context parallelism: the sequence is cut
+// into contiguous shards, each rank keeps its queries and passes the K/V
+// shards around a ring, and the partial results over the K/V shards are
+// combined by their log-sum-exp (myzaker / QbitAI "背后技术原理": block-sparse
+// attention combined with context-parallel ring block-sparse attention).
+//
+//   shard_fill   rows of a shard plan's query range that no key of the K/V
+//                shard reaches as a group (no plan entries): out = 0,
+//                lse = -inf, so every row of a shard result is defined.
+//   lse_merge    (o, lse) <- merge((o, lse), (o_p, lse_p)): with
+//                m = max(lse, lse_p), w = e^(lse - m), w_p = e^(lse_p - m):
+//                o = (w o + w_p o_p) / (w + w_p), lse = m + log(w + w_p).
+//                Both -inf: the row stays (0, -inf).
+// Both are HBM-bound elementwise passes; eight lanes per (batch, token, head)
+// row, each on 8 channels with 16- / 32-byte vector accesses.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "lc_internal.cuh"
+#include "lc_vec8.cuh"
+
+namespace {
+
+using lcvec::ld8;
+using lcvec::st8;
+
+struct FillArgs {
+  const int *grp_ptr;
+  int G, gc, Cb, Nc, Nn;
+  int qlo, qhi;         // the plan's query blocks
+  long long q_lo, q_n;  // its query tokens
+  int batch, heads;
+};
+
+// One CTA per group; groups outside the query range or with entries return.
+template <typename T>
+__global__ void shard_fill_kernel(FillArgs a, T *out, float *lse) {
+  const int g = blockIdx.x;
+  const int first = g < a.gc ? 4 * g : a.Cb + 4 * (g - a.gc);
+  if (first < a.qlo || first >= a.qhi) return;
+  if (a.grp_ptr[g + 1] != a.grp_ptr[g]) return;
+  const long long seg_end = g < a.gc ? a.Nc : (long long)a.Nc + a.Nn;
+  const long long t0 = g < a.gc ? 256LL * g : a.Nc + 256LL * (g - a.gc);
+  const long long t1 = t0 + 256 < seg_end ? t0 + 256 : seg_end;
+  long long r0 = t0 - a.q_lo, r1 = t1 - a.q_lo;  // rows of the shard buffers
+  r0 = r0 < 0 ? 0 : r0;
+  r1 = r1 > a.q_n ? a.q_n : r1;
+  if (r0 >= r1) return;
+  // out[b, r0:r1] is one contiguous span per batch entry.
+  const long long span = (r1 - r0) * a.heads * LC_HEAD_DIM;  // elements
+  const long long vec = span * (long long)sizeof(T) / 16;
+  for (int b = 0; b < a.batch; ++b) {
+    uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)b * a.q_n + r0) * a.heads * LC_HEAD_DIM);
+    for (long long i = threadIdx.x; i < vec; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+    const long long nl = (r1 - r0) * a.heads;
+    for (long long i = threadIdx.x; i < nl; i += blockDim.x) {
+      const int h = (int)(i / (r1 - r0));
+      const long long r = r0 + i % (r1 - r0);
+      lse[((long long)b * a.heads + h) * a.q_n + r] = -INFINITY;
+    }
+  }
+}
+
+template <typename T>
+__global__ void lse_merge_kernel(float *o_acc, float *lse_acc, const T *o_part,
+                                 const float *lse_part, T *out, long long rows, long long n,
+                                 int heads, int init) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long i = gid >> 3;  // (b * n + t) * heads + h
+  const int ch = (int)(gid & 7);
+  if (i >= rows) return;
+  const int h = (int)(i % heads);
+  const long long bt = i / heads;
+  const long long b = bt / n, t = bt - b * n;
+  const long long li = (b * heads + h) * n + t;
+  const long long oi = i * LC_HEAD_DIM + 8 * ch;
+  float p[8], o[8];
+  ld8(o_part + oi, p);
+  const float lp = lse_part[li];
+  float l;
+  if (init) {
+    l = lp;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = lp == -INFINITY ? 0.f : p[e];
+  } else {
+    ld8(o_acc + oi, o);
+    const float la = lse_acc[li];
+    const float m = fmaxf(la, lp);
+    if (m == -INFINITY) {
+      l = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = 0.f;
+    } else {
+      const float wa = expf(la - m), wp = expf(lp - m);  // one of them is 1
+      const float inv = 1.f / (wa + wp);
+      const float ca = wa * inv, cp = wp * inv;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        o[e] = (wa > 0.f ? ca * o[e] : 0.f) + (wp > 0.f ? cp * p[e] : 0.f);
+      l = m + logf(wa + wp);
+    }
+  }
+  if (out)
+    st8(out + oi, o);
+  else
+    st8(o_acc + oi, o);
+  if (ch == 0) lse_acc[li] = l;
+}
+
+}  // namespace
+
+lc_status lc_launch_shard_fill(const lc_bsa_plan_s *plan, void *out, float *lse, int batch,
+                               int heads, lc_dtype dtype, cudaStream_t stream) {
+  if (plan->G_active == plan->G) return LC_OK;  // every group has entries
+  FillArgs a;
+  a.grp_ptr = plan->grp_ptr;
+  a.G = plan->G; a.gc = plan->gc; a.Cb = plan->Cb; a.Nc = plan->Nc; a.Nn = plan->Nn;
+  a.qlo = plan->qlo; a.qhi = plan->qhi;
+  a.q_lo = lc_block_token(plan, plan->qlo);
+  a.q_n = lc_block_token(plan, plan->qhi) - a.q_lo;
+  a.batch = batch; a.heads = heads;
+  if (a.q_n <= 0) return LC_OK;
+  LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
+  if (dtype == LC_DTYPE_F32)
+    shard_fill_kernel<float><<<plan->G, 256, 0, stream>>>(a, static_cast<float *>(out), lse);
+  else
+    shard_fill_kernel<__nv_bfloat16><<<plan->G, 256, 0, stream>>>(
+        a, static_cast<__nv_bfloat16 *>(out), lse);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}
+
+lc_status lc_launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
+                              const float *lse_part, void *out, int batch, long long n, int heads,
+                              lc_dtype dtype, bool init, cudaStream_t stream) {
+  const long long rows = (long long)batch * n * heads;
+  if (rows == 0) return LC_OK;
+  const long long threads = rows * 8;
+  const unsigned grid = (unsigned)((threads + 255) / 256);
+  if (dtype == LC_DTYPE_F32)
+    lse_merge_kernel<float><<<grid, 256, 0, stream>>>(o_acc, lse_acc,
+                                                      static_cast<const float *>(o_part), lse_part,
+                                                      static_cast<float *>(out), rows, n, heads,
+                                                      init ? 1 : 0);
+  else
+    lse_merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        o_acc, lse_acc, static_cast<const __nv_bfloat16 *>(o_part), lse_part,
+        static_cast<__nv_bfloat16 *>(out), rows, n, heads, init ? 1 : 0);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}

@@ -307,6 +307,71 @@ lc_status lc_bsa_forward_noalloc(const void *q, const void *k, const void *v, vo
                                  void *stream);
 
 /*
+ * Context parallelism (myzaker / QbitAI "背后技术原理": block-sparse attention
+ * is combined with context-parallel ring block-sparse attention for the
+ * high-resolution pass).  The sequence's blocks are cut into contiguous
+ * shards, one per rank; each rank keeps its query shard, the K/V shards
+ * travel around a ring of ranks, and each step's partial result over one K/V
+ * shard is merged into the rank's running result by log-sum-exp.  The pages
+ * give no more than this; the pieces below are the device half of it (the
+ * ring itself is the Python driver's send/recv over NCCL).
+ *
+ * lc_bsa_plan_create_shard -- the plan of lc_bsa_plan_create restricted to
+ * query blocks [q_block_lo, q_block_hi) and key blocks [k_block_lo,
+ * k_block_hi) (block ids as in lc_bsa_plan_create: condition blocks first).
+ * The query bounds must be group boundaries: 0, multiples of 4 below Cb, Cb,
+ * Cb + multiples of 4, or the block count (LC_ERR_INVALID_ARGUMENT
+ * otherwise).  The key bounds are free.  A shard plan is accepted by
+ * lc_bsa_forward_shard only; lc_bsa_plan_info reports its counts (nnz and
+ * attended pairs of the shard) and lc_bsa_plan_copy_csr / _csc its entries.
+ */
+lc_status lc_bsa_plan_create_shard(lc_bsa_plan *out, int T, int H, int W, int block, int local,
+                                   int stride, int n_cond_frames, int q_block_lo, int q_block_hi,
+                                   int k_block_lo, int k_block_hi, void *stream);
+
+/* Token ranges a plan covers: queries [*q_lo, *q_hi), keys [*k_lo, *k_hi)
+ * (whole-sequence token indices; a full plan covers [0, N) twice). */
+lc_status lc_bsa_plan_token_range(lc_bsa_plan plan, long long *q_lo, long long *q_hi,
+                                  long long *k_lo, long long *k_hi);
+
+/*
+ * lc_bsa_forward_shard -- attention of the query tokens of a shard plan over
+ * the key tokens of that plan only: q and out hold [batch, q_hi - q_lo,
+ * heads, 64] (the plan's query token range, lc_bsa_plan_token_range), k and
+ * v hold [batch, k_hi - k_lo, heads, 64] (pre-RoPE, like lc_bsa_forward's k;
+ * they are rotated at their whole-sequence positions), lse (required) is
+ * [batch, heads, q_hi - q_lo].  Rows that attend no key of the shard get
+ * out = 0 and lse = -inf, so lc_bsa_lse_merge can take every shard's result
+ * as it is.  opts: the RMSNorm weights of lc_bsa_forward_ex, flags 0.
+ * bf16 only (LC_DTYPE_F32: LC_ERR_UNSUPPORTED).  Errors as lc_bsa_forward.
+ */
+lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void *out, float *lse,
+                               int batch, int heads, int head_dim, lc_dtype dtype,
+                               float softmax_scale, const lc_bsa_opts *opts, lc_bsa_plan plan,
+                               lc_rope3d rope, void *stream);
+
+#define LC_MERGE_INIT 1u  /* the running result is not read: it starts as the part */
+
+/*
+ * lc_bsa_lse_merge -- fold one partial attention result (o_part of dtype,
+ * lse_part fp32) into a running one (o_acc fp32, lse_acc fp32), per (batch,
+ * token, head) row:  m = max(lse_acc, lse_part), w = e^(lse_acc - m),
+ * w_p = e^(lse_part - m);  o = (w o_acc + w_p o_part) / (w + w_p),
+ * lse = m + log(w + w_p); a row with both lse -inf stays (0, -inf).  The
+ * result over a partition of the keys equals the attention over all of them.
+ * Layouts: o_acc, o_part, out [batch, n_tokens, heads, 64]; lse_acc, lse_part
+ * [batch, heads, n_tokens].  out NULL: o goes to o_acc; out given: o goes to
+ * out, rounded to dtype, and o_acc is not written (the last step of a ring).
+ * flags: LC_MERGE_INIT (o_acc and lse_acc not read; o_acc may then be NULL
+ * when out is given).  lse_acc always receives the merged lse.  Errors:
+ * LC_ERR_INVALID_ARGUMENT (NULL or misaligned pointer, bad sizes or flags),
+ * LC_ERR_UNSUPPORTED (head_dim != 64).
+ */
+lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
+                           const float *lse_part, void *out, int batch, long long n_tokens,
+                           int heads, int head_dim, lc_dtype dtype, unsigned flags, void *stream);
+
+/*
  * lc_last_device_status -- synchronise `stream`, then report and clear the
  * current device's status word, which the kernels set when a bounded wait
  * timed out (LC_ERR_TIMEOUT) or an in-kernel check failed

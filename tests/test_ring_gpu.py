@@ -1,0 +1,231 @@
+"""Ring context parallelism on the GPU: shard plans, the shard forward
+(lc_bsa_forward_shard), the log-sum-exp merge (lc_bsa_lse_merge) and the
+whole ring, one process standing in for every rank (each rank's K/V shard is
+taken from the full tensors instead of arriving over NCCL; the exchange itself
+is covered on CPU with gloo), against the fp64 oracle.
+
+Tolerances: bf16 as the forward's (|out - ref| <= 1.5e-2, mean <= 1e-3; lse
+<= 5e-2), plus at most one more bf16 rounding of the merged output; the merge
+kernel alone works in fp32 on exact inputs: 1e-6 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import ring as orng
+from block_sparse_attention_rope_b200 import ring, synthetic
+from block_sparse_attention_rope_b200.synthetic import Workload
+
+pytestmark = pytest.mark.gpu
+
+SMALL = Workload("ring_small", T=5, H=8, W=40, n_cond=2, heads=2, local=1, stride=2,
+                 dtype="bf16")                       # Cb 10, Nb 15: 25 blocks, ragged tails
+RAGGED = Workload("ring_ragged", T=6, H=13, W=21, n_cond=1, heads=2, local=2, stride=3,
+                  dtype="bf16", batch=2)
+
+
+@pytest.fixture(scope="module")
+def api():
+    from block_sparse_attention_rope_b200 import build
+    build.build()
+    from block_sparse_attention_rope_b200 import api as a
+    return a
+
+
+def geo(w):
+    return dict(T=w.T, H=w.H, W=w.W, n_cond=w.n_cond, local=w.local, stride=w.stride)
+
+
+def blocks(w):
+    Nc, Nn, Cb, Nb = oracle.segment_sizes(w.T, w.H, w.W, w.n_cond)
+    return Cb, Nb
+
+
+def test_shard_plans_partition_the_full_plan(api):
+    w = SMALL
+    Cb, Nb = blocks(w)
+    full = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rp, ci = (x.numpy() for x in full.csr())
+    fi = full.info()
+    shards = [(0, 4), (4, 10), (10, 18), (18, 25)]
+    nnz = pairs = 0
+    for qs in shards:
+        for ks in shards:
+            p = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                         q_blocks=qs, k_blocks=ks)
+            inf = p.info()
+            srp, sci = (x.numpy() for x in p.csr())
+            # the shard's CSR is the full CSR with rows and columns restricted (bit-exact)
+            for r in range(Cb + Nb):
+                row = ci[rp[r]:rp[r + 1]]
+                want = row[(row >= ks[0]) & (row < ks[1])] if qs[0] <= r < qs[1] else row[:0]
+                assert np.array_equal(sci[srp[r]:srp[r + 1]], want)
+            nnz += inf.nnz
+            pairs += inf.attended_token_pairs
+    assert nnz == fi.nnz and pairs == fi.attended_token_pairs
+
+
+def test_shard_plan_argument_errors(api):
+    w = SMALL
+    with pytest.raises(api.LcError):   # query bound inside a group
+        api.Plan(w.T, w.H, w.W, local=1, stride=2, n_cond=2, q_blocks=(0, 6), k_blocks=(0, 25))
+    with pytest.raises(api.LcError):   # past the last block
+        api.Plan(w.T, w.H, w.W, local=1, stride=2, n_cond=2, q_blocks=(0, 4), k_blocks=(0, 26))
+    p = api.Plan(w.T, w.H, w.W, local=1, stride=2, n_cond=2, q_blocks=(4, 10), k_blocks=(3, 7))
+    assert p.q_tokens == (256, 640) and p.k_tokens == (192, 448)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    x = synthetic.make_inputs(w)
+    q = x["q"].cuda()
+    # a shard plan is refused by the whole-sequence entry points
+    with pytest.raises(api.LcError):
+        api.forward(q, x["k"].cuda(), x["v"].cuda(), p, rope)
+    with pytest.raises(api.LcError):   # fp32 shards are not supported
+        qf = torch.zeros(1, 384, 2, 64, device="cuda")
+        kf = torch.zeros(1, 256, 2, 64, device="cuda")
+        api.forward_shard(qf, kf, kf, p, rope)
+
+
+def _shard_case(api, w, x, rope, qs, ks):
+    p = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                 q_blocks=qs, k_blocks=ks)
+    (qa, qb), (ka, kb) = p.q_tokens, p.k_tokens
+    d = {n: x[n].cuda() for n in ("q", "k", "v")}
+    out = torch.full((w.batch, qb - qa, w.heads, 64), float("nan"), dtype=torch.bfloat16,
+                     device="cuda")
+    lse = torch.full((w.batch, w.heads, qb - qa), float("nan"), device="cuda")
+    api.forward_shard(d["q"][:, qa:qb].contiguous(), d["k"][:, ka:kb].contiguous(),
+                      d["v"][:, ka:kb].contiguous(), p, rope, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    ref_o, ref_l = orng.partial_attention(x["q"][:, qa:qb], x["k"][:, ka:kb], x["v"][:, ka:kb],
+                                          q_tokens=(qa, qb), k_tokens=(ka, kb), **geo(w))
+    return out.double().cpu().numpy(), lse.double().cpu().numpy(), ref_o, ref_l
+
+
+@pytest.mark.parametrize("qs,ks", [((4, 10), (0, 25)), ((10, 18), (10, 18)), ((0, 4), (10, 25)),
+                                   ((18, 25), (3, 11)), ((10, 14), (20, 25)), ((0, 10), (0, 3))])
+def test_forward_shard_matches_oracle(api, qs, ks):
+    w = SMALL
+    x = synthetic.make_inputs(w)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    o, l, ref_o, ref_l = _shard_case(api, w, x, rope, qs, ks)
+    empty = ref_l == -np.inf
+    # rows that attend no key of the shard: exactly (0, -inf); every other row is written
+    assert np.array_equal(l == -np.inf, empty)
+    assert np.all(o.transpose(0, 2, 1, 3)[empty] == 0)
+    assert not np.isnan(o).any() and not np.isnan(l).any()
+    err = np.abs(o - ref_o)
+    assert err.max() <= 1.5e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    fin = ~empty
+    if fin.any():
+        assert np.abs(l[fin] - ref_l[fin]).max() <= 5e-2
+
+
+def test_lse_merge_kernel(api):
+    g = torch.Generator().manual_seed(5)
+    B, n, heads = 2, 300, 3
+    o_a = torch.randn(B, n, heads, 64, generator=g)
+    l_a = 3 * torch.randn(B, heads, n, generator=g)
+    o_b = torch.randn(B, n, heads, 64, generator=g).bfloat16()
+    l_b = 3 * torch.randn(B, heads, n, generator=g)
+    l_a[0, 0, :7] = -float("inf")          # empty running rows
+    o_a[0, :7, 0] = 0
+    l_b[1, 2, 10:20] = -float("inf")       # empty part rows (their o is 0)
+    o_b[1, 10:20, 2] = 0
+    l_a[1, 1, 30:33] = l_b[1, 1, 30:33] = -float("inf")
+    o_a[1, 30:33, 1] = 0
+    o_b[1, 30:33, 1] = 0
+    ref_o, ref_l = orng.lse_merge(o_a.double().numpy(), l_a.double().numpy(),
+                                  o_b.double().numpy(), l_b.double().numpy())
+    acc_o, acc_l = o_a.cuda(), l_a.cuda()
+    api.lse_merge(acc_o, acc_l, o_b.cuda(), l_b.cuda())
+    torch.cuda.synchronize()
+    assert np.abs(acc_o.double().cpu().numpy() - ref_o).max() <= 1e-6 * np.abs(ref_o).max()
+    gl = acc_l.double().cpu().numpy()
+    assert np.array_equal(gl == -np.inf, ref_l == -np.inf)
+    fin = np.isfinite(ref_l)
+    assert np.abs(gl[fin] - ref_l[fin]).max() <= 1e-6 * np.abs(ref_l[fin]).max()
+    # init: the part is copied (empty rows -> 0); out: the merged o in the part's dtype
+    acc_o2, acc_l2 = torch.full_like(acc_o, float("nan")), torch.full_like(acc_l, float("nan"))
+    api.lse_merge(acc_o2, acc_l2, o_b.cuda(), l_b.cuda(), init=True)
+    torch.cuda.synchronize()
+    assert torch.equal(acc_o2.cpu(), o_b.float()) and torch.equal(acc_l2.cpu(), l_b)
+    out = torch.empty_like(o_b).cuda()
+    acc_o3, acc_l3 = o_a.cuda(), l_a.cuda()
+    api.lse_merge(acc_o3, acc_l3, o_b.cuda(), l_b.cuda(), out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(acc_o3.cpu(), o_a)  # not written when out is given
+    assert torch.equal(out.cpu(), torch.from_numpy(ref_o).float().bfloat16()) or \
+        np.abs(out.double().cpu().numpy() - ref_o).max() <= 2 ** -8 * np.abs(ref_o).max()
+
+
+def run_ring(api, w, x, shards, rope, dev):
+    """Every rank of the ring in this process; returns out [B, N, heads, 64], lse."""
+    d = {n: x[n].to(dev) for n in ("q", "k", "v")}
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(w.batch, w.heads, w.n_tokens, device=dev)
+    for rank in range(len(shards)):
+        sched, partial, merge = ring.gpu_steps(api, w.T, w.H, w.W, local=w.local,
+                                               stride=w.stride, n_cond=w.n_cond, shards=shards,
+                                               rank=rank, rope=rope)
+        a, b = sched.tokens[rank]
+
+        def fetch(src):
+            ka, kb = sched.tokens[src]
+            return d["k"][:, ka:kb].contiguous(), d["v"][:, ka:kb].contiguous()
+        k0, v0 = fetch(rank)
+        o, l = ring.ring_forward(sched, d["q"][:, a:b].contiguous(), k0, v0, partial, merge,
+                                 fetch=fetch)
+        out[:, a:b] = o
+        lse[:, :, a:b] = l
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    return out, lse
+
+
+@pytest.mark.parametrize("w,world", [(SMALL, 2), (SMALL, 4), (RAGGED, 3)])
+def test_ring_matches_oracle_and_full_forward(api, w, world):
+    x = synthetic.make_inputs(w)
+    Cb, Nb = blocks(w)
+    rp, _ = oracle.block_csr(w.T, w.H, w.W, 64, w.local, w.stride, w.n_cond)
+    shards = ring.balanced_shards(np.diff(rp), Cb, world)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    out, lse = run_ring(api, w, x, shards, rope, "cuda")
+    ref_o, ref_l = oracle.forward(x["q"], x["k"], x["v"], **geo(w))
+    o = out.double().cpu().numpy()
+    err = np.abs(o - ref_o)
+    assert err.max() <= 1.5e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    assert np.abs(lse.double().cpu().numpy() - ref_l).max() <= 5e-2
+    # and next to the single-launch forward: the same up to one more rounding
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    full_o, full_l = api.forward(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), plan, rope,
+                                 return_lse=True)
+    assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
+    assert (lse - full_l).abs().max().item() <= 1e-2
+
+
+def test_ring_full_size_sampled(api):
+    """I2V 480p (37,440 tokens, 32 heads) over 8 ring ranks in one process:
+    sampled rows against the oracle, every row against the single launch."""
+    from parity import compare, oracle_rows, sample_rows
+    w = synthetic.get("i2v_480p")
+    x = synthetic.make_inputs(w)
+    rp, _ = oracle.block_csr(w.T, w.H, w.W, 64, w.local, w.stride, w.n_cond)
+    Cb, Nb = blocks(w)
+    shards = ring.balanced_shards(np.diff(rp), Cb, 8)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    out, lse = run_ring(api, w, x, shards, rope, "cuda")
+    rows = sample_rows(w, n_random_blocks=16)
+    # rows on both sides of every shard boundary
+    toks = orng.shard_tokens(shards, w.T, w.H, w.W, w.n_cond)
+    edge = np.array([t for a, _ in toks[1:] for t in (a - 1, a)], dtype=np.int64)
+    rows = np.unique(np.concatenate([rows, edge]))
+    heads = [0, 31]
+    ref_o, ref_l = oracle_rows(w, x, rows, heads)
+    compare(w, out.cpu(), lse.cpu(), ref_o, ref_l, rows, heads)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    full_o, full_l = api.forward(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), plan, rope,
+                                 return_lse=True)
+    assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
+    assert (lse - full_l).abs().max().item() <= 1e-2

@@ -226,10 +226,11 @@ def time_backward(api, synthetic, torch, name, steps, warmup, stream):
 
 def time_ring(api, synthetic, torch, name, world, stream, reps=3):
     """Ring context parallelism over `world` ranks, every rank run in turn on
-    this GPU with its K/V shards already resident (the NCCL exchange is left
-    out: on NVLink it overlaps the compute).  Per rank: device time of its
-    shard forwards and merges; the slowest rank bounds a real ring's step.
-    Compared with one whole-sequence launch divided by `world`."""
+    this GPU with the K/V shards it receives already resident (the NCCL
+    exchange is left out: on NVLink it overlaps the compute).  Per rank: device
+    time of its own q / k rotation, its shard forwards and the final merge;
+    the slowest rank bounds a real ring's step.  Compared with one
+    whole-sequence launch divided by `world`."""
     import numpy as np
     from block_sparse_attention_rope_b200 import ring
     w = synthetic.get(name)
@@ -238,31 +239,26 @@ def time_ring(api, synthetic, torch, name, world, stream, reps=3):
     rope = api.Rope3D(w.T, w.H, w.W)
     rp, _ = plan.csr()
     shards = ring.balanced_shards(np.diff(rp.numpy()), plan.info().num_cond_blocks, world)
-    ranks = []
-    for r in range(world):
-        sched, partial, merge = ring.gpu_steps(api, w.T, w.H, w.W, local=w.local,
-                                               stride=w.stride, n_cond=w.n_cond, shards=shards,
-                                               rank=r, rope=rope)
-        kv = {}
-        for src in range(world):
-            a_, b_ = sched.tokens[src]
-            kv[src] = (x["k"][:, a_:b_].contiguous(), x["v"][:, a_:b_].contiguous())
-        a_, b_ = sched.tokens[r]
-        ranks.append((sched, partial, merge, x["q"][:, a_:b_].contiguous(), kv))
+    ranks = [ring.GpuRingRank(api, w.T, w.H, w.W, local=w.local, stride=w.stride,
+                              n_cond=w.n_cond, shards=shards, rank=r, rope=rope, batch=w.batch,
+                              heads=w.heads) for r in range(world)]
+    toks = ranks[0].sched.tokens
+    own = [{n: x[n][:, a:b].contiguous() for n in ("q", "k", "v")} for a, b in toks]
+    k_rot = [ranks[s].rotate(own[s]["k"], s, None) for s in range(world)]  # as received
 
-    def run_rank(sched, partial, merge, q, kv):
-        return ring.ring_forward(sched, q, kv[sched.rank][0], kv[sched.rank][1], partial, merge,
-                                 fetch=lambda src: kv[src])
+    def run_rank(r):
+        return ranks[r].forward(own[r]["q"], own[r]["k"], own[r]["v"],
+                                fetch=lambda src: (k_rot[src], own[src]["v"]))
     per = []
     with torch.cuda.stream(stream):
-        for rk in ranks:
-            run_rank(*rk)  # warm-up
+        for r in range(world):
+            run_rank(r)  # warm-up
         torch.cuda.synchronize()
-        for rk in ranks:
+        for r in range(world):
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
             ev[0].record(stream)
             for _ in range(reps):
-                run_rank(*rk)
+                run_rank(r)
             ev[1].record(stream)
             torch.cuda.synchronize()
             per.append(ev[0].elapsed_time(ev[1]) / reps)
@@ -277,13 +273,14 @@ def time_ring(api, synthetic, torch, name, world, stream, reps=3):
     if api.last_device_status() != 0:
         raise RuntimeError("device status set by the ring")
     full = ev[0].elapsed_time(ev[1]) / reps
-    steps = sum(sum(rk[0].computes) for rk in ranks)
+    steps = sum(sum(rr.sched.computes) for rr in ranks)
     return {"workload": name, "ranks": world, "shards_blocks": shards,
             "computing_steps": steps, "skipped_steps": world * world - steps,
             "ms_per_rank_max": round(max(per), 3), "ms_per_rank_mean": round(sum(per) / world, 3),
             "whole_sequence_ms": round(full, 3), "ideal_ms": round(full / world, 3),
             "compute_efficiency": round(full / world / max(per), 3),
-            "kernels": "per step: shard_fill, rope_k_kernel, bsa_sm100_kernel, lse_merge"}
+            "kernels": "per rank: rope_apply (q, k once); per step: bsa_sm100_kernel "
+                       "(shard_fill where a group has no entry); lse_merge_parts once"}
 
 
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):
@@ -477,6 +474,8 @@ def run_ours(a):
         extra["backward_i2v_480p"] = time_backward(api, synthetic, torch, "i2v_480p", 2, 1,
                                                    stream)
         extra["ring_8_ranks_i2v_480p"] = time_ring(api, synthetic, torch, "i2v_480p", 8, stream)
+        extra["ring_8_ranks_refine_720p"] = time_ring(api, synthetic, torch, "refine_720p", 8,
+                                                      stream)
     w = main["w"]
     ms = main["total_ms"] / a.steps
     value = world * main["flops"] * a.steps / (main["total_ms"] * 1e-3) / 1e12

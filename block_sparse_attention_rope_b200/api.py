@@ -73,6 +73,8 @@ def _load():
         "lc_bsa_plan_token_range": (S, [vp] + [ctypes.POINTER(LL)] * 4),
         "lc_bsa_forward_shard": (S, [vp, vp, vp, vp, vp, I, I, I, I, F, vp, vp, vp, vp]),
         "lc_bsa_lse_merge": (S, [vp, vp, vp, vp, vp, I, LL, I, I, I, ctypes.c_uint, vp]),
+        "lc_bsa_lse_merge_parts": (S, [vp, vp, I, vp, vp, I, LL, I, I, I, vp]),
+        "lc_rope3d_apply_ex": (S, [vp, vp, I, LL, I, I, LL, I, vp, F, vp, vp]),
         "lc_last_device_status": (S, [vp]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
         "lc_status_string": (ctypes.c_char_p, [S]),
@@ -86,6 +88,8 @@ def _load():
 
 lib = _load()
 COND_K_ROTATED = 1  # LC_FLAG_COND_K_ROTATED
+Q_ROTATED = 2       # LC_FLAG_Q_ROTATED
+K_ROTATED = 4       # LC_FLAG_K_ROTATED
 
 
 def status_string(s: int) -> str:
@@ -221,14 +225,25 @@ class Rope3D:
         return out
 
     def apply(self, x: torch.Tensor, tok_offset: int = 0, out: Optional[torch.Tensor] = None,
+              norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
               stream=None) -> torch.Tensor:
+        """R(x), or R(norm(x)) with RMSNorm weights `norm` (lc_rope3d_apply_ex);
+        token n of x is token n + tok_offset of the sequence."""
         B, n, heads, hd = x.shape
         if out is None:
             out = torch.empty_like(x)
         _check_bmhk("x", x, x.shape, x.dtype)
         _check_bmhk("out", out, x.shape, x.dtype)
-        _check(lib.lc_rope3d_apply(x.data_ptr(), out.data_ptr(), B, n, heads, hd, tok_offset,
-                                   _dtype_code(x), self.handle, _stream(stream)), "lc_rope3d_apply")
+        if norm is None:
+            _check(lib.lc_rope3d_apply(x.data_ptr(), out.data_ptr(), B, n, heads, hd, tok_offset,
+                                       _dtype_code(x), self.handle, _stream(stream)),
+                   "lc_rope3d_apply")
+        else:
+            _opts(0, norm, None, norm_eps, hd)  # checks the weight tensor
+            _check(lib.lc_rope3d_apply_ex(x.data_ptr(), out.data_ptr(), B, n, heads, hd,
+                                          tok_offset, _dtype_code(x), norm.data_ptr(),
+                                          float(norm_eps), self.handle, _stream(stream)),
+                   "lc_rope3d_apply_ex")
         return out
 
     def close(self, stream=None):
@@ -417,11 +432,13 @@ def forward_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Pla
 def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan, rope: Rope3D,
                   *, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                   softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
-                  k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6, stream=None):
+                  k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
+                  q_rotated: bool = False, k_rotated: bool = False, stream=None):
     """Partial attention of one shard pair (lc_bsa_forward_shard): q holds the
     shard plan's query tokens [B, nq, heads, 64], k / v its key tokens
-    [B, nk, heads, 64] (pre-RoPE, bf16).  Returns (out, lse); rows that attend
-    no key of the shard get out 0 and lse -inf."""
+    [B, nk, heads, 64] (pre-RoPE, bf16, or already normalised and rotated with
+    q_rotated / k_rotated).  Returns (out, lse); rows that attend no key of
+    the shard get out 0 and lse -inf."""
     B, nq, heads, hd = q.shape
     nk = plan.k_tokens[1] - plan.k_tokens[0]
     _check_bmhk("q", q, (B, plan.q_tokens[1] - plan.q_tokens[0], heads, hd), q.dtype)
@@ -433,7 +450,8 @@ def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
         lse = torch.empty(B, heads, nq, dtype=torch.float32, device=q.device)
     _check_bmhk("out", out, q.shape, q.dtype)
     _check_bmhk("lse", lse, (B, heads, nq), torch.float32)
-    opts = _opts(0, q_norm, k_norm, norm_eps, hd)
+    flags = (Q_ROTATED if q_rotated else 0) | (K_ROTATED if k_rotated else 0)
+    opts = _opts(flags, q_norm, k_norm, norm_eps, hd)
     _check(lib.lc_bsa_forward_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     lse.data_ptr(), B, heads, hd, _dtype_code(q),
                                     float(softmax_scale),
@@ -465,6 +483,26 @@ def lse_merge(o_acc: Optional[torch.Tensor], lse_acc: torch.Tensor, o_part: torc
                                 _dtype_code(o_part), MERGE_INIT if init else 0, _stream(stream)),
            "lc_bsa_lse_merge")
     return out if out is not None else o_acc
+
+
+def lse_merge_parts(parts: torch.Tensor, lses: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                    lse_out: Optional[torch.Tensor] = None, stream=None):
+    """Combine P partial results over disjoint key sets in one pass
+    (lc_bsa_lse_merge_parts): parts [P, B, n, heads, 64], lses [P, B, heads, n].
+    Returns (out [B, n, heads, 64] of parts' dtype, lse [B, heads, n])."""
+    P, B, n, heads, hd = parts.shape
+    _check_bmhk("parts", parts, parts.shape, parts.dtype)
+    _check_bmhk("lses", lses, (P, B, heads, n), torch.float32)
+    if out is None:
+        out = torch.empty(parts.shape[1:], dtype=parts.dtype, device=parts.device)
+    if lse_out is None:
+        lse_out = torch.empty(B, heads, n, dtype=torch.float32, device=parts.device)
+    _check_bmhk("out", out, parts.shape[1:], parts.dtype)
+    _check_bmhk("lse_out", lse_out, (B, heads, n), torch.float32)
+    _check(lib.lc_bsa_lse_merge_parts(parts.data_ptr(), lses.data_ptr(), P, out.data_ptr(),
+                                      lse_out.data_ptr(), B, n, heads, hd, _dtype_code(parts),
+                                      _stream(stream)), "lc_bsa_lse_merge_parts")
+    return out, lse_out
 
 
 def last_device_status(stream=None) -> int:

@@ -274,7 +274,8 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   if (s != LC_OK) return s;
   unsigned flags;
   lc_qk_norm norm;
-  if (!parse_opts(opts, 0u, &flags, &norm)) return LC_ERR_INVALID_ARGUMENT;
+  if (!parse_opts(opts, LC_FLAG_Q_ROTATED | LC_FLAG_K_ROTATED, &flags, &norm))
+    return LC_ERR_INVALID_ARGUMENT;
   if (!q || !k || !v || !out || !lse) return LC_ERR_INVALID_ARGUMENT;
   if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -287,6 +288,8 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   sv.q_n = lc_block_token(plan, plan->qhi) - sv.q_lo;
   sv.k_lo = lc_block_token(plan, plan->klo);
   sv.k_n = lc_block_token(plan, plan->khi) - sv.k_lo;
+  sv.q_rotated = (flags & LC_FLAG_Q_ROTATED) != 0;
+  sv.k_rotated = (flags & LC_FLAG_K_ROTATED) != 0;
   if (sv.q_n == 0) return LC_OK;
   int *dev_status = lc_device_status_ptr(&s);
   if (s != LC_OK) return s;
@@ -316,6 +319,22 @@ extern "C" lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *
   if ((long long)batch * n_tokens * heads >= (1LL << 40)) return LC_ERR_UNSUPPORTED;
   return lc_launch_lse_merge(o_acc, lse_acc, o_part, lse_part, out, batch, n_tokens, heads, dtype,
                              init, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" lc_status lc_bsa_lse_merge_parts(const void *parts, const float *lses, int n_parts,
+                                            void *out, float *lse_out, int batch,
+                                            long long n_tokens, int heads, int head_dim,
+                                            lc_dtype dtype, void *stream) {
+  if (batch <= 0 || heads <= 0 || head_dim <= 0 || n_tokens < 0 || n_parts <= 0)
+    return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
+  if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
+  if (!parts || !lses || !out || misaligned(parts) || misaligned(out) ||
+      ((reinterpret_cast<uintptr_t>(lses) | reinterpret_cast<uintptr_t>(lse_out)) & 3u))
+    return LC_ERR_INVALID_ARGUMENT;
+  if ((long long)batch * n_tokens * heads * n_parts >= (1LL << 40)) return LC_ERR_UNSUPPORTED;
+  return lc_launch_lse_merge_parts(parts, lses, n_parts, out, lse_out, batch, n_tokens, heads,
+                                   dtype, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" lc_status lc_last_device_status(void *stream) {

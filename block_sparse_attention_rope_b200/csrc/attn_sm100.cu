@@ -118,6 +118,7 @@ struct __align__(64) Sm100Params {
   int k_row_off[2];        // same for the k/v maps
   int tab_floats;
   int k_prerotated;        // K tensors already hold R(k): skip the K rotation
+  int q_prerotated;        // Q tensors already hold R(q): skip the Q rotation (shards)
   float scale_log2;
   const float *q_norm_w;   // RMSNorm weights [64] applied ahead of the rotation, or NULL
   const float *k_norm_w;
@@ -587,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         ok = wait_warp(ctx, ctx.bar(B_QFULL + qi), qph);
         if (!ok) break;
         const int r0 = it.row0 + 128 * i;
-        const int nrows = min(128, it.seg_len - r0);
+        const int nrows = p.q_prerotated ? 0 : min(128, it.seg_len - r0);
 #pragma unroll 1
         for (int r = rt; r < nrows; r += kRopeThreads)
           rope_row(sQ + qi * kTileBytes, r, seg_base + r0 + r, tab, p, q_nw);
@@ -1186,7 +1187,10 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   // K is rotated once per call into scratch (one pass over K) and the kernel
   // loads it rotated; rotating every loaded K tile in the kernel instead (as
   // the allocation-free entry point does, having no scratch) measured slower.
-  const bool k_prepass = true;
+  // (A shard whose K arrives rotated needs no prepass.)
+  const bool k_prepass = !(sharded && shard->k_rotated);
+  if (sharded && shard->k_rotated) prm.k_prerotated = 1;
+  if (sharded && shard->q_rotated) prm.q_prerotated = 1;
   int *counter = nullptr;
   void *k_rot = nullptr, *ck_rot = nullptr;
   cudaMemPool_t pool = lc_scratch_pool(&s);

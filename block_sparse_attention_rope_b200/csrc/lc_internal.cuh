@@ -29,6 +29,7 @@ struct lc_bsa_plan_s {
   int gc, gn, G;            // groups in the condition / noisy segment, total
   int qlo, qhi, klo, khi;   // block ranges the plan covers (a shard plan: part of the pattern)
   int G_active;             // groups with at least one entry (the first G_active of grp_order)
+  bool fill_needed;         // a group of the query range has no entry (shard plans)
   long long nnz;            // CSR entries (host closed form, checked on device)
   int device;
   cudaEvent_t ready;        // recorded after the planner kernels
@@ -174,6 +175,7 @@ __device__ __forceinline__ float lc_rms_apply(float x, float inv, float w) {
 enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2, LC_FWD_SHARD = 3 };
 struct lc_shard_view {
   long long q_lo, q_n, k_lo, k_n;
+  bool q_rotated, k_rotated;  // q / k already hold R(norm(x)) (rotated once per ring)
 };
 
 // RMSNorm of q and k ahead of the rotation: device fp32 weights [64] or NULL.
@@ -208,6 +210,9 @@ lc_status lc_launch_shard_fill(const lc_bsa_plan_s *plan, void *out, float *lse,
 lc_status lc_launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
                               const float *lse_part, void *out, int batch, long long n, int heads,
                               lc_dtype dtype, bool init, cudaStream_t stream);
+lc_status lc_launch_lse_merge_parts(const void *parts, const float *lses, int n_parts, void *out,
+                                    float *lse_out, int batch, long long n, int heads,
+                                    lc_dtype dtype, cudaStream_t stream);
 // Gradients dq, dk, dv of the whole-sequence attention (attn_bwd.cu).
 lc_status lc_launch_backward(const void *q, const void *k, const void *v, const void *out,
                              const float *lse, const void *dout, void *dq, void *dk, void *dv,

@@ -423,6 +423,7 @@ static lc_status plan_create(lc_bsa_plan *out, int T, int H, int W, int block, i
              p->kgc, p->kgn, p->KG, qlo, qhi, klo, khi};
   long long nnz = 0;
   p->G_active = p->G;
+  p->fill_needed = false;
   if (qlo == 0 && qhi == p->nq && klo == 0 && khi == p->nq) {  // closed form
     nnz = (long long)p->Cb * p->Cb + (long long)p->Nb * p->Cb;
     for (long long i = 0; i < p->Nb; ++i) nnz += noisy_row_count(i, p->Nb, local, stride);
@@ -441,6 +442,7 @@ static lc_status plan_create(lc_bsa_plan *out, int T, int H, int W, int block, i
           }
       }
       p->G_active += any ? 1 : 0;
+      if (!any && first >= qlo && first < qhi) p->fill_needed = true;
     }
   }
   p->nnz = nnz;

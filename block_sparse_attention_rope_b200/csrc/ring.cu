@@ -11,7 +11,9 @@
 //                m = max(lse, lse_p), w = e^(lse - m), w_p = e^(lse_p - m):
 //                o = (w o + w_p o_p) / (w + w_p), lse = m + log(w + w_p).
 //                Both -inf: the row stays (0, -inf).
-// Both are HBM-bound elementwise passes; eight lanes per (batch, token, head)
+//   lse_merge_parts  the same over P parts at once (one pass: a ring's
+//                partial results kept until the last step, then combined).
+// All are HBM-bound elementwise passes; eight lanes per (batch, token, head)
 // row, each on 8 channels with 16- / 32-byte vector accesses.
 #include <cuda_bf16.h>
 #include <math.h>
@@ -107,11 +109,51 @@ __global__ void lse_merge_kernel(float *o_acc, float *lse_acc, const T *o_part,
   if (ch == 0) lse_acc[li] = l;
 }
 
+// P partial results of the same rows over disjoint key sets -> the result
+// over all of them: m = max_i lse_i, w_i = e^(lse_i - m),
+// o = sum_i w_i o_i / sum_i w_i, lse = m + log sum_i w_i (all -inf: 0, -inf).
+// One pass over the parts' outputs (parts whose weight is 0 are not read).
+template <typename T>
+__global__ void lse_merge_parts_kernel(const T *parts, const float *lses, int n_parts, T *out,
+                                       float *lse_out, long long rows, long long n, int heads) {
+  const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  const long long i = gid >> 3;  // (b * n + t) * heads + h
+  const int ch = (int)(gid & 7);
+  if (i >= rows) return;
+  const int h = (int)(i % heads);
+  const long long bt = i / heads;
+  const long long b = bt / n, t = bt - b * n;
+  const long long li = (b * heads + h) * n + t;
+  const long long oi = i * LC_HEAD_DIM + 8 * ch;
+  const long long o_stride = rows * LC_HEAD_DIM, l_stride = rows;  // per part
+  float m = -INFINITY;
+  for (int k = 0; k < n_parts; ++k) m = fmaxf(m, lses[k * l_stride + li]);
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float wsum = 0.f;
+  if (m != -INFINITY) {
+    for (int k = 0; k < n_parts; ++k) {
+      const float w = expf(lses[k * l_stride + li] - m);
+      if (w > 0.f) {
+        float v[8];
+        ld8(parts + k * o_stride + oi, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w, v[e], acc[e]);
+        wsum += w;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] *= inv;
+  st8(out + oi, acc);
+  if (ch == 0 && lse_out) lse_out[li] = m == -INFINITY ? -INFINITY : m + logf(wsum);
+}
+
 }  // namespace
 
 lc_status lc_launch_shard_fill(const lc_bsa_plan_s *plan, void *out, float *lse, int batch,
                                int heads, lc_dtype dtype, cudaStream_t stream) {
-  if (plan->G_active == plan->G) return LC_OK;  // every group has entries
+  if (!plan->fill_needed) return LC_OK;  // every group of the query range has entries
   FillArgs a;
   a.grp_ptr = plan->grp_ptr;
   a.G = plan->G; a.gc = plan->gc; a.Cb = plan->Cb; a.Nc = plan->Nc; a.Nn = plan->Nn;
@@ -146,6 +188,24 @@ lc_status lc_launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
     lse_merge_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
         o_acc, lse_acc, static_cast<const __nv_bfloat16 *>(o_part), lse_part,
         static_cast<__nv_bfloat16 *>(out), rows, n, heads, init ? 1 : 0);
+  LC_CUDA_TRY(cudaGetLastError());
+  return LC_OK;
+}
+
+lc_status lc_launch_lse_merge_parts(const void *parts, const float *lses, int n_parts, void *out,
+                                    float *lse_out, int batch, long long n, int heads,
+                                    lc_dtype dtype, cudaStream_t stream) {
+  const long long rows = (long long)batch * n * heads;
+  if (rows == 0) return LC_OK;
+  const unsigned grid = (unsigned)((rows * 8 + 255) / 256);
+  if (dtype == LC_DTYPE_F32)
+    lse_merge_parts_kernel<float><<<grid, 256, 0, stream>>>(
+        static_cast<const float *>(parts), lses, n_parts, static_cast<float *>(out), lse_out,
+        rows, n, heads);
+  else
+    lse_merge_parts_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(parts), lses, n_parts,
+        static_cast<__nv_bfloat16 *>(out), lse_out, rows, n, heads);
   LC_CUDA_TRY(cudaGetLastError());
   return LC_OK;
 }

@@ -167,6 +167,27 @@ lc_status lc_rotate_rows(const void *x, void *out, int batch, long long ntok, in
   return LC_OK;
 }
 
+extern "C" lc_status lc_rope3d_apply_ex(const void *x, void *out, int batch, long long ntok,
+                                        int heads, int head_dim, long long tok_offset,
+                                        lc_dtype dtype, const float *norm_weight, float norm_eps,
+                                        lc_rope3d rope, void *stream) {
+  if (!x || !out || !rope || batch <= 0 || ntok <= 0 || heads <= 0 || tok_offset < 0)
+    return LC_ERR_INVALID_ARGUMENT;
+  if (dtype != LC_DTYPE_BF16 && dtype != LC_DTYPE_F32) return LC_ERR_INVALID_ARGUMENT;
+  if (head_dim != LC_HEAD_DIM) return LC_ERR_UNSUPPORTED;
+  if (tok_offset + ntok > (long long)rope->T * rope->H * rope->W) return LC_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return LC_ERR_INVALID_ARGUMENT;
+  if (norm_weight && ((reinterpret_cast<uintptr_t>(norm_weight) & 3) ||
+                      !(norm_eps >= 0.f && norm_eps <= 3.0e38f)))
+    return LC_ERR_INVALID_ARGUMENT;
+  int dev = -1;
+  LC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev != rope->device) return LC_ERR_INVALID_ARGUMENT;
+  return lc_rotate_rows(x, out, batch, ntok, heads, tok_offset, dtype, rope, norm_weight,
+                        norm_weight ? norm_eps : 0.f, static_cast<cudaStream_t>(stream));
+}
+
 extern "C" lc_status lc_rope3d_apply(const void *x, void *out, int batch, long long ntok, int heads,
                                      int head_dim, long long tok_offset, lc_dtype dtype,
                                      lc_rope3d rope, void *stream) {

@@ -9,12 +9,13 @@ and at step s holds the K/V shard of rank (r - s) mod world, which it passes
 on to rank r + 1 while it computes (NCCL send/recv over NVLink, one
 batched group per step, on the communicator's own stream so the transfer
 overlaps the attention).  Each step's partial result (lc_bsa_forward_shard)
-is folded into the rank's running result by log-sum-exp (lc_bsa_lse_merge);
-a step whose K/V shard holds no block the rank's queries attend is skipped
-(its K/V still travels on).
+is kept, and after the last step the rank's partial results are combined by
+log-sum-exp in one pass (lc_bsa_lse_merge_parts); a step whose K/V shard
+holds no block the rank's queries attend is skipped (its K/V still travels
+on).
 
 The schedule and the exchange are plain host logic; the compute steps are
-passed in, so the same ring runs on the GPU library (``gpu_steps``) or, in
+passed in, so the same ring runs on the GPU library (``GpuRingRank``) or, in
 tests, on anything with the same shape contract.
 """
 from __future__ import annotations
@@ -92,20 +93,20 @@ def _exchange(send: Sequence[torch.Tensor], recv: Sequence[torch.Tensor], dst: i
 
 
 def ring_forward(sched: RingSchedule, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                 partial: Callable, merge: Callable, group=None, fetch: Optional[Callable] = None):
+                 partial: Callable, combine: Callable, group=None,
+                 fetch: Optional[Callable] = None):
     """Run the ring for one rank.
 
     q, k, v: this rank's shard [B, n_rank, heads, hd].
-    partial(src, q, k_src, v_src) -> (o, lse): attention over shard src's keys.
-    merge(acc, part, first, last) -> acc: fold a part in; the value returned
-      after the last computing step is the result.
+    partial(src, q, k_src, v_src, slot): the attention over shard src's keys
+      (slot counts the computing steps from 0); its results are collected.
+    combine(results): the rank's result from the collected partial results.
     fetch(src) -> (k_src, v_src): instead of the NCCL exchange, take shard src
       directly (one process standing in for every rank).
     """
     world, rank = sched.world, sched.rank
     cur_k, cur_v = k, v
-    acc = None
-    first = True
+    parts = []
     for s in range(world):
         src = sched.sources[s]
         reqs = []
@@ -121,51 +122,65 @@ def ring_forward(sched: RingSchedule, q: torch.Tensor, k: torch.Tensor, v: torch
                 reqs = _exchange((cur_k, cur_v), (nxt_k, nxt_v), (rank + 1) % world,
                                  (rank - 1) % world, group)
         if sched.computes[s]:
-            part = partial(src, q, cur_k, cur_v)
-            acc = merge(acc, part, first, s == sched.last)
-            first = False
+            parts.append(partial(src, q, cur_k, cur_v, len(parts)))
         for r in reqs:
             r.wait()
         cur_k, cur_v = nxt_k, nxt_v
-    return acc
+    return combine(parts)
 
 
-def gpu_steps(api, T: int, H: int, W: int, *, local: int, stride: int, n_cond: int,
-              shards: Sequence[Tuple[int, int]], rank: int, rope, softmax_scale: float = 0.0,
-              q_norm=None, k_norm=None, norm_eps: float = 1e-6):
-    """Shard plans of one rank (one per K/V shard it attends) and the partial
-    / merge steps on the GPU library.  Returns (schedule, partial, merge)."""
-    full = api.Plan(T, H, W, local=local, stride=stride, n_cond=n_cond)
-    inf = full.info()
-    Cb, N, Nc = inf.num_cond_blocks, full.n_tokens, full.n_cond_tokens
-    plans = {}
-    for src in range(len(shards)):
-        p = api.Plan(T, H, W, local=local, stride=stride, n_cond=n_cond, q_blocks=shards[rank],
-                     k_blocks=shards[src])
-        if p.info().nnz > 0:
-            plans[src] = p
-    sched = RingSchedule(shards, Nc, Cb, N, rank, lambda r, src: src in plans)
-    kw = dict(softmax_scale=softmax_scale, q_norm=q_norm, k_norm=k_norm, norm_eps=norm_eps)
+class GpuRingRank:
+    """One rank of the ring on the GPU library: its shard plans (one per K/V
+    shard its queries attend), the buffers of its partial results, and the
+    steps.  The rank rotates its own q and k once (lc_rope3d_apply_ex, with
+    the RMSNorm if given); the rotated K shard is what travels, so no step
+    rotates again.  Partial results stay in one buffer until the last step
+    and are combined in one pass (lc_bsa_lse_merge_parts)."""
 
-    def partial(src, q, k_src, v_src):
-        return api.forward_shard(q, k_src, v_src, plans[src], rope, **kw)
+    def __init__(self, api, T: int, H: int, W: int, *, local: int, stride: int, n_cond: int,
+                 shards: Sequence[Tuple[int, int]], rank: int, rope, batch: int, heads: int,
+                 dtype=torch.bfloat16, device="cuda", softmax_scale: float = 0.0,
+                 q_norm=None, k_norm=None, norm_eps: float = 1e-6):
+        self.api, self.rope = api, rope
+        self.q_norm, self.k_norm, self.norm_eps = q_norm, k_norm, norm_eps
+        self.softmax_scale = softmax_scale
+        full = api.Plan(T, H, W, local=local, stride=stride, n_cond=n_cond)
+        Cb, N, Nc = full.info().num_cond_blocks, full.n_tokens, full.n_cond_tokens
+        self.plans = {}
+        for src in range(len(shards)):
+            p = api.Plan(T, H, W, local=local, stride=stride, n_cond=n_cond,
+                         q_blocks=shards[rank], k_blocks=shards[src])
+            if p.info().nnz > 0:
+                self.plans[src] = p
+        self.sched = RingSchedule(shards, Nc, Cb, N, rank, lambda r, src: src in self.plans)
+        nq = self.sched.n_tokens(rank)
+        n_parts = sum(self.sched.computes)
+        self.parts = torch.empty(n_parts, batch, nq, heads, 64, dtype=dtype, device=device)
+        self.lses = torch.empty(n_parts, batch, heads, nq, dtype=torch.float32, device=device)
 
-    def merge(acc, part, first, last):
-        o_p, l_p = part
-        if first and last:
-            return o_p, l_p
-        if first:
-            o_acc = torch.empty(o_p.shape, dtype=torch.float32, device=o_p.device)
-            l_acc = torch.empty_like(l_p)
-            api.lse_merge(o_acc, l_acc, o_p, l_p, init=True)
-            return o_acc, l_acc
-        o_acc, l_acc = acc
-        if last:
-            out = torch.empty_like(o_p)
-            api.lse_merge(o_acc, l_acc, o_p, l_p, out=out)
-            return out, l_acc
-        api.lse_merge(o_acc, l_acc, o_p, l_p)
-        return o_acc, l_acc
+    def rotate(self, x: torch.Tensor, shard: int, norm) -> torch.Tensor:
+        """R(norm(x)) of shard `shard`'s tokens at their sequence positions."""
+        return self.rope.apply(x, tok_offset=self.sched.tokens[shard][0], norm=norm,
+                               norm_eps=self.norm_eps)
 
-    sched.plans = plans
-    return sched, partial, merge
+    def partial(self, src, q_rot, k_rot, v, slot):
+        self.api.forward_shard(q_rot, k_rot, v, self.plans[src], self.rope, out=self.parts[slot],
+                               lse=self.lses[slot], softmax_scale=self.softmax_scale,
+                               q_rotated=True, k_rotated=True)
+        return slot
+
+    def combine(self, slots):
+        n = len(slots)
+        if n == 1:
+            return self.parts[0], self.lses[0]
+        return self.api.lse_merge_parts(self.parts[:n], self.lses[:n])
+
+    def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,
+                fetch: Optional[Callable] = None):
+        """This rank's attention output and lse over the whole sequence.  q, k,
+        v: the rank's own shard, pre-RoPE.  With `fetch(src) -> (R(norm(k_src)),
+        v_src)` the K/V shards are taken from it instead of the ring exchange."""
+        r = self.sched.rank
+        q_rot = self.rotate(q, r, self.q_norm)
+        k_rot = self.rotate(k, r, self.k_norm)
+        return ring_forward(self.sched, q_rot, k_rot, v, self.partial, self.combine, group, fetch)

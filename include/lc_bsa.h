@@ -154,6 +154,17 @@ lc_status lc_rope3d_apply(const void *x, void *out, int batch, long long ntok, i
                           int head_dim, long long tok_offset, lc_dtype dtype,
                           lc_rope3d rope, void *stream);
 
+/* lc_rope3d_apply with the RMSNorm of the attention modules ahead of the
+ * rotation: out = R(norm(x)), norm(x) = x / sqrt(mean(x^2) + norm_eps) * w
+ * per token and head (norm_weight: device fp32 [head_dim], or NULL for the
+ * plain rotation).  The same arithmetic as every rotation inside the
+ * attention entry points, so a tensor prepared here gives those calls the
+ * same bits (LC_FLAG_Q_ROTATED / LC_FLAG_K_ROTATED). */
+lc_status lc_rope3d_apply_ex(const void *x, void *out, int batch, long long ntok, int heads,
+                             int head_dim, long long tok_offset, lc_dtype dtype,
+                             const float *norm_weight, float norm_eps, lc_rope3d rope,
+                             void *stream);
+
 /*
  * lc_bsa_forward -- out = softmax(mask(scale * R(q) R(k)^T)) v over the whole
  * sequence of N = T*H*W tokens, with R the 3D-RoPE of `rope` and the mask of
@@ -185,6 +196,8 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
 
 /* Flags of lc_bsa_opts. */
 #define LC_FLAG_COND_K_ROTATED 1u  /* cond_k already holds R(k) (lc_bsa_cond_cache) */
+#define LC_FLAG_Q_ROTATED 2u       /* q already holds R(norm_q(q)) (lc_bsa_forward_shard) */
+#define LC_FLAG_K_ROTATED 4u       /* k already holds R(norm_k(k)) (lc_bsa_forward_shard) */
 
 /*
  * Options of the _ex entry points and of lc_bsa_cond_cache.  A NULL options
@@ -342,8 +355,12 @@ lc_status lc_bsa_plan_token_range(lc_bsa_plan plan, long long *q_lo, long long *
  * they are rotated at their whole-sequence positions), lse (required) is
  * [batch, heads, q_hi - q_lo].  Rows that attend no key of the shard get
  * out = 0 and lse = -inf, so lc_bsa_lse_merge can take every shard's result
- * as it is.  opts: the RMSNorm weights of lc_bsa_forward_ex, flags 0.
- * bf16 only (LC_DTYPE_F32: LC_ERR_UNSUPPORTED).  Errors as lc_bsa_forward.
+ * as it is.  opts: the RMSNorm weights of lc_bsa_forward_ex; flags
+ * LC_FLAG_Q_ROTATED / LC_FLAG_K_ROTATED when q / k already hold the
+ * normalised, rotated values (lc_rope3d_apply_ex at their whole-sequence
+ * positions): a ring rotates each shard once and reuses it at every step.
+ * The result is the same bits either way.  bf16 only (LC_DTYPE_F32:
+ * LC_ERR_UNSUPPORTED).  Errors as lc_bsa_forward.
  */
 lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void *out, float *lse,
                                int batch, int heads, int head_dim, lc_dtype dtype,
@@ -370,6 +387,22 @@ lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void
 lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
                            const float *lse_part, void *out, int batch, long long n_tokens,
                            int heads, int head_dim, lc_dtype dtype, unsigned flags, void *stream);
+
+/*
+ * lc_bsa_lse_merge_parts -- the merge of lc_bsa_lse_merge over n_parts
+ * partial results at once: parts [n_parts, batch, n_tokens, heads, 64] of
+ * dtype and lses [n_parts, batch, heads, n_tokens] fp32 (contiguous, part
+ * after part) -> out [batch, n_tokens, heads, 64] of dtype and, if lse_out is
+ * not NULL, lse_out [batch, heads, n_tokens]:  m = max_i lse_i,
+ * w_i = e^(lse_i - m);  out = sum_i w_i o_i / sum_i w_i,
+ * lse = m + log sum_i w_i (a row whose lse are all -inf: 0 and -inf).  One
+ * pass, fp32 arithmetic, one rounding to dtype.  Errors: LC_ERR_INVALID_ARGUMENT
+ * (NULL or misaligned pointer, n_parts <= 0, bad sizes), LC_ERR_UNSUPPORTED
+ * (head_dim != 64).
+ */
+lc_status lc_bsa_lse_merge_parts(const void *parts, const float *lses, int n_parts, void *out,
+                                 float *lse_out, int batch, long long n_tokens, int heads,
+                                 int head_dim, lc_dtype dtype, void *stream);
 
 /*
  * lc_last_device_status -- synchronise `stream`, then report and clear the

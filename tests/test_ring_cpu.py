@@ -57,18 +57,17 @@ def _schedule(shards, rank):
 def _oracle_steps(sched):
     geo = {k: GEOM[k] for k in ("T", "H", "W", "n_cond", "local", "stride")}
 
-    def partial(src, q, k, v):
-        o, l = orng.partial_attention(q.numpy(), k.numpy(), v.numpy(),
+    def partial(src, q, k, v, slot):
+        return orng.partial_attention(q.numpy(), k.numpy(), v.numpy(),
                                       q_tokens=sched.tokens[sched.rank],
                                       k_tokens=sched.tokens[src], **geo)
-        return torch.from_numpy(o), torch.from_numpy(l)
 
-    def merge(acc, part, first, last):
-        if first:
-            return part
-        o, l = orng.lse_merge(acc[0].numpy(), acc[1].numpy(), part[0].numpy(), part[1].numpy())
+    def combine(parts):
+        o, l = parts[0]
+        for po, pl in parts[1:]:
+            o, l = orng.lse_merge(o, l, po, pl)
         return torch.from_numpy(o), torch.from_numpy(l)
-    return partial, merge
+    return partial, combine
 
 
 def _worker(rank, world, port, shards, qout):
@@ -79,9 +78,9 @@ def _worker(rank, world, port, shards, qout):
         q, k, v = (torch.from_numpy(a) for a in _inputs())
         sched = _schedule(shards, rank)
         a, b = sched.tokens[rank]
-        partial, merge = _oracle_steps(sched)
+        partial, combine = _oracle_steps(sched)
         o, l = ring.ring_forward(sched, q[:, a:b].contiguous(), k[:, a:b].contiguous(),
-                                 v[:, a:b].contiguous(), partial, merge)
+                                 v[:, a:b].contiguous(), partial, combine)
         qout.put((rank, a, b, o.numpy(), l.numpy(), sched.computes))
     finally:
         dist.destroy_process_group()
@@ -123,7 +122,7 @@ def test_balanced_shards_cut_on_group_edges():
     with pytest.raises(ValueError):
         ring.balanced_shards(work, Cb, len(edges))
     # balance: the I2V 480p pattern over 8 ranks is within one group's work of even
-    rp, _ = oracle.block_csr(16, 30, 52, 64, 2, 4, 1)
+    rp, _ = oracle.block_csr(24, 30, 52, 64, 2, 4, 1)
     w = np.diff(rp)
     sh = ring.balanced_shards(w, 25, 8)
     per = [int(w[a:b].sum()) for a, b in sh]

@@ -160,28 +160,81 @@ def test_lse_merge_kernel(api):
         np.abs(out.double().cpu().numpy() - ref_o).max() <= 2 ** -8 * np.abs(ref_o).max()
 
 
-def run_ring(api, w, x, shards, rope, dev):
+def run_ring(api, w, x, shards, rope, dev, q_norm=None, k_norm=None):
     """Every rank of the ring in this process; returns out [B, N, heads, 64], lse."""
     d = {n: x[n].to(dev) for n in ("q", "k", "v")}
     out = torch.empty_like(d["q"])
     lse = torch.empty(w.batch, w.heads, w.n_tokens, device=dev)
-    for rank in range(len(shards)):
-        sched, partial, merge = ring.gpu_steps(api, w.T, w.H, w.W, local=w.local,
-                                               stride=w.stride, n_cond=w.n_cond, shards=shards,
-                                               rank=rank, rope=rope)
-        a, b = sched.tokens[rank]
-
-        def fetch(src):
-            ka, kb = sched.tokens[src]
-            return d["k"][:, ka:kb].contiguous(), d["v"][:, ka:kb].contiguous()
-        k0, v0 = fetch(rank)
-        o, l = ring.ring_forward(sched, d["q"][:, a:b].contiguous(), k0, v0, partial, merge,
-                                 fetch=fetch)
+    ranks = [ring.GpuRingRank(api, w.T, w.H, w.W, local=w.local, stride=w.stride,
+                              n_cond=w.n_cond, shards=shards, rank=r, rope=rope, batch=w.batch,
+                              heads=w.heads, device=dev, q_norm=q_norm, k_norm=k_norm)
+             for r in range(len(shards))]
+    toks = ranks[0].sched.tokens
+    # what each rank sends around the ring: its K shard normalised and rotated once
+    k_rot = {s: ranks[s].rotate(d["k"][:, a:b].contiguous(), s, k_norm)
+             for s, (a, b) in enumerate(toks)}
+    v_sh = {s: d["v"][:, a:b].contiguous() for s, (a, b) in enumerate(toks)}
+    for rank, rr in enumerate(ranks):
+        a, b = toks[rank]
+        o, l = rr.forward(d["q"][:, a:b].contiguous(), d["k"][:, a:b].contiguous(), v_sh[rank],
+                          fetch=lambda src: (k_rot[src], v_sh[src]))
         out[:, a:b] = o
         lse[:, :, a:b] = l
     torch.cuda.synchronize()
     assert api.last_device_status() == 0
     return out, lse
+
+
+def test_prerotated_shards_are_bit_exact(api):
+    """q / k rotated (and normalised) once by lc_rope3d_apply_ex and flagged
+    give the same bits as the shard kernel's own rotations."""
+    w = SMALL
+    x = synthetic.make_inputs(w, device="cuda")
+    rope = api.Rope3D(w.T, w.H, w.W)
+    g = torch.Generator().manual_seed(4)
+    for norm in (False, True):
+        qn = (1 + 0.3 * torch.randn(64, generator=g)).cuda() if norm else None
+        kn = (1 + 0.3 * torch.randn(64, generator=g)).cuda() if norm else None
+        for qs, ks in (((4, 10), (0, 25)), ((10, 18), (3, 11))):
+            p = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                         q_blocks=qs, k_blocks=ks)
+            (qa, qb), (ka, kb) = p.q_tokens, p.k_tokens
+            q, k, v = (x[n][:, a:b].contiguous() for n, a, b in
+                       (("q", qa, qb), ("k", ka, kb), ("v", ka, kb)))
+            o1, l1 = api.forward_shard(q, k, v, p, rope, q_norm=qn, k_norm=kn)
+            qr = rope.apply(q, tok_offset=qa, norm=qn)
+            kr = rope.apply(k, tok_offset=ka, norm=kn)
+            o2, l2 = api.forward_shard(qr, kr, v, p, rope, q_rotated=True, k_rotated=True)
+            o3, l3 = api.forward_shard(q, kr, v, p, rope, q_norm=qn, k_rotated=True)
+            torch.cuda.synchronize()
+            assert torch.equal(o1, o2) and torch.equal(l1, l2)
+            assert torch.equal(o1, o3) and torch.equal(l1, l3)
+
+
+@pytest.mark.parametrize("n_parts", [1, 3, 8])
+def test_lse_merge_parts_kernel(api, n_parts):
+    g = torch.Generator().manual_seed(n_parts)
+    B, n, heads = 2, 257, 3
+    parts = torch.randn(n_parts, B, n, heads, 64, generator=g).bfloat16()
+    lses = 4 * torch.randn(n_parts, B, heads, n, generator=g)
+    lses[:, 0, 1, :5] = -float("inf")          # rows empty in every part
+    parts[:, 0, :5, 1] = 0
+    lses[0, 1, 2, 7:40] = -float("inf")        # rows empty in one part
+    parts[0, 1, 7:40, 2] = 0
+    ref_o, ref_l = parts[0].double().numpy(), lses[0].double().numpy()
+    for i in range(1, n_parts):
+        ref_o, ref_l = orng.lse_merge(ref_o, ref_l, parts[i].double().numpy(),
+                                      lses[i].double().numpy())
+    out, lse = api.lse_merge_parts(parts.cuda(), lses.cuda())
+    torch.cuda.synchronize()
+    o = out.double().cpu().numpy()
+    # one rounding to bf16 of an fp32 combination
+    assert np.all(np.abs(o - ref_o) <= 2 ** -8 * np.abs(ref_o) + 1e-6 * np.abs(ref_o).max())
+    gl = lse.double().cpu().numpy()
+    assert np.array_equal(gl == -np.inf, ref_l == -np.inf)
+    fin = np.isfinite(ref_l)
+    assert np.abs(gl[fin] - ref_l[fin]).max() <= 1e-6 * np.abs(ref_l[fin]).max()
+    assert np.all(o.transpose(0, 2, 1, 3)[~fin] == 0)
 
 
 @pytest.mark.parametrize("w,world", [(SMALL, 2), (SMALL, 4), (RAGGED, 3)])
@@ -203,6 +256,21 @@ def test_ring_matches_oracle_and_full_forward(api, w, world):
                                  return_lse=True)
     assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
     assert (lse - full_l).abs().max().item() <= 1e-2
+
+
+def test_ring_with_rms_norm(api):
+    w = SMALL
+    x = synthetic.make_inputs(w)
+    g = torch.Generator().manual_seed(8)
+    qn, kn = 1 + 0.3 * torch.randn(64, generator=g), 1 + 0.3 * torch.randn(64, generator=g)
+    shards = [(0, 4), (4, 10), (10, 18), (18, 25)]
+    rope = api.Rope3D(w.T, w.H, w.W)
+    out, lse = run_ring(api, w, x, shards, rope, "cuda", qn.cuda(), kn.cuda())
+    ref_o, ref_l, _ = orng.ring_forward(x["q"], x["k"], x["v"], shards, q_norm=qn.double().numpy(),
+                                        k_norm=kn.double().numpy(), norm_eps=1e-6, **geo(w))
+    err = np.abs(out.double().cpu().numpy() - ref_o)
+    assert err.max() <= 1.5e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
+    assert np.abs(lse.double().cpu().numpy() - ref_l).max() <= 5e-2
 
 
 def test_ring_full_size_sampled(api):

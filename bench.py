@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward pass of --workload (one JSON line; for profiling)")
+    ap.add_argument("--ring-only", type=int, default=0, metavar="RANKS",
+                    help="time only the ring over RANKS ranks (all in this process) on "
+                         "--workload (one JSON line; for profiling)")
     return ap.parse_args()
 
 
@@ -562,6 +565,14 @@ def main():
                           torch.cuda.current_stream())
         print(json.dumps(dict(metric="backward ms per layer", value=r["ms_per_layer"], unit="ms",
                               higher_is_better=False, **r)), flush=True)
+    elif a.ring_only:
+        import torch
+        torch.cuda.set_device(0)
+        from block_sparse_attention_rope_b200 import api, synthetic
+        r = time_ring(api, synthetic, torch, a.workload, a.ring_only, torch.cuda.current_stream(),
+                      reps=max(1, a.steps))
+        print(json.dumps(dict(metric="ring ms per rank (slowest)", value=r["ms_per_rank_max"],
+                              unit="ms", higher_is_better=False, **r)), flush=True)
     else:
         run_ours(a)
 

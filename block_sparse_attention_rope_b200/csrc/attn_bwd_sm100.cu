@@ -68,7 +68,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // hold two 32-column TMEM loads and their results; producer / MMA / RoPE need
 // few; the dQ warpgroup holds one 64-column row.  The host refuses to launch
 // unless the block's registers cover the split.
-constexpr int kRegsEw = 152, kRegsCtl = 80, kRegsDq = 112;
+constexpr int kRegsEw = 160, kRegsCtl = 80, kRegsDq = 112;
 constexpr int kRegsTotal = 256 * kRegsEw + 128 * (kRegsCtl + kRegsDq);
 constexpr int kRegsAtLaunchMin = (kRegsTotal + kThreads - 1) / kThreads;
 static_assert(kRegsTotal <= 65536, "register split");
@@ -625,6 +625,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         // this one is computed (double buffer)
         uint8_t *ptile = sP + half * kTileBytes;  // P^T, this query block's tile
         uint32_t sr[2][16], dr[2][16];
+        // the whole row's P^T and dS^T, packed, before the wait for the tiles
+        uint32_t pk[4][8], dk[4][8];
         lcptx::tmem_ld16(tST + 64 * half, sr[0]);
         lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
         lcptx::tmem_wait_ld();
@@ -642,7 +644,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t(&scur)[16] = sr[k & 1];
           const uint32_t(&dcur)[16] = dr[k & 1];
           const int jb = k * 16;  // first query of the chunk within its block
-          uint32_t pp[8], dd[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
@@ -654,28 +655,27 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
               pv[u] = pe;
               dv2[u] = pe * (__uint_as_float(dcur[2 * i + u]) - dl[j]) * p.scale;
             }
-            pp[i] = pack_bf16(pv[0], pv[1]);
-            dd[i] = pack_bf16(dv2[0], dv2[1]);
-          }
-          if (k == 0 && q_it > 0) {  // the previous step's MMAs are done with the tiles
-            ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
-            if (!ok) {
-              lcptx::tmem_wait_ld();  // nothing of this warp stays in flight
-              break;
-            }
-          }
-          // row kr of the P^T and dS^T tiles: 64 queries of this block, 128-byte
-          // swizzled; K-major for dV / dK, MN-major (dS) for dQ
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            *reinterpret_cast<uint4 *>(ptile + swz(kr, k * 2 + i)) =
-                make_uint4(pp[4 * i], pp[4 * i + 1], pp[4 * i + 2], pp[4 * i + 3]);
-            *reinterpret_cast<uint4 *>(tile + swz(kr, k * 2 + i)) =
-                make_uint4(dd[4 * i], dd[4 * i + 1], dd[4 * i + 2], dd[4 * i + 3]);
+            pk[k][i] = pack_bf16(pv[0], pv[1]);
+            dk[k][i] = pack_bf16(dv2[0], dv2[1]);
           }
           if (k < 3) lcptx::tmem_wait_ld();
         }
-        if (!ok) break;
+        if (q_it > 0) {  // the previous step's MMAs are done with the tiles
+          ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
+          if (!ok) break;
+        }
+        // row kr of the P^T and dS^T tiles: 64 queries of this block, 128-byte
+        // swizzled; K-major for dV / dK, MN-major (dS) for dQ
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            *reinterpret_cast<uint4 *>(ptile + swz(kr, k * 2 + i)) =
+                make_uint4(pk[k][4 * i], pk[k][4 * i + 1], pk[k][4 * i + 2], pk[k][4 * i + 3]);
+            *reinterpret_cast<uint4 *>(tile + swz(kr, k * 2 + i)) =
+                make_uint4(dk[k][4 * i], dk[k][4 * i + 1], dk[k][4 * i + 2], dk[k][4 * i + 3]);
+          }
+        }
         lcptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));

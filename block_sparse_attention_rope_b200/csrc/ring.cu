@@ -34,7 +34,8 @@ struct FillArgs {
   int batch, heads;
 };
 
-// One CTA per group; groups outside the query range or with entries return.
+// Grid (group, slice): each CTA clears one of gridDim.y slices of a group's
+// rows; groups outside the query range or with entries return at once.
 template <typename T>
 __global__ void shard_fill_kernel(FillArgs a, T *out, float *lse) {
   const int g = blockIdx.x;
@@ -47,17 +48,21 @@ __global__ void shard_fill_kernel(FillArgs a, T *out, float *lse) {
   long long r0 = t0 - a.q_lo, r1 = t1 - a.q_lo;  // rows of the shard buffers
   r0 = r0 < 0 ? 0 : r0;
   r1 = r1 > a.q_n ? a.q_n : r1;
-  if (r0 >= r1) return;
-  // out[b, r0:r1] is one contiguous span per batch entry.
-  const long long span = (r1 - r0) * a.heads * LC_HEAD_DIM;  // elements
-  const long long vec = span * (long long)sizeof(T) / 16;
+  // this CTA's slice of the rows
+  const long long nr = r1 - r0, per = (nr + gridDim.y - 1) / gridDim.y;
+  const long long s0 = r0 + per * blockIdx.y;
+  const long long s1 = s0 + per < r1 ? s0 + per : r1;
+  if (s0 >= s1) return;
+  // out[b, s0:s1] is one contiguous span per batch entry (whole rows: a
+  // multiple of 16 bytes).
+  const long long vec = (s1 - s0) * a.heads * LC_HEAD_DIM * (long long)sizeof(T) / 16;
+  const long long nl = (s1 - s0) * a.heads;
   for (int b = 0; b < a.batch; ++b) {
-    uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)b * a.q_n + r0) * a.heads * LC_HEAD_DIM);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + ((long long)b * a.q_n + s0) * a.heads * LC_HEAD_DIM);
     for (long long i = threadIdx.x; i < vec; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
-    const long long nl = (r1 - r0) * a.heads;
     for (long long i = threadIdx.x; i < nl; i += blockDim.x) {
-      const int h = (int)(i / (r1 - r0));
-      const long long r = r0 + i % (r1 - r0);
+      const int h = (int)(i / (s1 - s0));
+      const long long r = s0 + i % (s1 - s0);
       lse[((long long)b * a.heads + h) * a.q_n + r] = -INFINITY;
     }
   }
@@ -163,10 +168,11 @@ lc_status lc_launch_shard_fill(const lc_bsa_plan_s *plan, void *out, float *lse,
   a.batch = batch; a.heads = heads;
   if (a.q_n <= 0) return LC_OK;
   LC_CUDA_TRY(cudaStreamWaitEvent(stream, plan->ready, 0));
+  const dim3 grid(plan->G, 16);  // 16 slices of up to 16 rows per group
   if (dtype == LC_DTYPE_F32)
-    shard_fill_kernel<float><<<plan->G, 256, 0, stream>>>(a, static_cast<float *>(out), lse);
+    shard_fill_kernel<float><<<grid, 256, 0, stream>>>(a, static_cast<float *>(out), lse);
   else
-    shard_fill_kernel<__nv_bfloat16><<<plan->G, 256, 0, stream>>>(
+    shard_fill_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
         a, static_cast<__nv_bfloat16 *>(out), lse);
   LC_CUDA_TRY(cudaGetLastError());
   return LC_OK;

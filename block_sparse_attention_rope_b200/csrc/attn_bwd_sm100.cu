@@ -60,6 +60,7 @@ constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kBoxBytes = 64 * 128;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256, kColDK = 320, kColDQ = 384;
+constexpr uint32_t kColPT = 448;  // P^T as bf16 pairs (the A operand of dV)
 constexpr uint32_t kIdescKQ = lcptx::idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
 constexpr uint32_t kIdescAcc = lcptx::idesc_bf16_f32(128, 64, 0, 1);  // dV, dK (A K-major)
 constexpr uint32_t kIdescDQ = lcptx::idesc_bf16_f32(128, 64, 1, 1);   // dQ (A = dS, MN-major)
@@ -100,8 +101,7 @@ struct SmemOffsets {
   static constexpr int v = k + kTileBytes;                     // value tile
   static constexpr int q = v + kTileBytes;                     // [kQStages] query tiles Q'
   static constexpr int g = q + kQStages * kTileBytes;          // [kQStages] dO tiles
-  static constexpr int pt = g + kQStages * kTileBytes;         // P^T, two 64-query tiles
-  static constexpr int ds = pt + 2 * kTileBytes;               // dS^T, two 64-query tiles
+  static constexpr int ds = g + kQStages * kTileBytes;         // dS^T, two 64-query tiles
   static constexpr int dq = ds + 2 * kTileBytes;               // dQ' staging: [block][half] 64 x 32 fp32
   static constexpr int lse = dq + 2 * kTileBytes;              // [kQStages][128] lse * log2e
   static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] D
@@ -121,8 +121,8 @@ enum {
   B_QG_READY = B_QG_FULL + kQStages,   // lse / D staged
   B_QG_EMPTY = B_QG_READY + kQStages,  // step's MMAs done with Q, dO
   B_SDP = B_QG_EMPTY + kQStages,    // S^T and dP^T in TMEM
-  B_PDS = B_SDP + 1,                // P^T, dS^T written to shared memory (8 warps)
-  B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete (P^T, dS^T tiles free)
+  B_PDS = B_SDP + 1,                // P^T in TMEM, dS^T in shared memory (8 warps)
+  B_STEP = B_PDS + 1,               // step's dV, dK, dQ MMAs complete (dS^T tiles free)
   B_DQ_FULL = B_STEP + 1,           // dQ of a step in TMEM
   B_DQ_EMPTY = B_DQ_FULL + 1,       // dQ read out (4 warps)
   B_ACC = B_DQ_EMPTY + 1,           // item's dK, dV complete
@@ -130,7 +130,8 @@ enum {
   B_DQ_STAGED = B_EPI_FREE + 1,     // dQ' tile staged in shared memory (4 warps)
   B_DQ_SMEM_FREE = B_DQ_STAGED + 1, // its reduce-add has read the staging tile
   B_DRAIN = B_DQ_SMEM_FREE + 1,
-  B_COUNT = B_DRAIN + 1
+  B_PT_FREE = B_DRAIN + 1,          // step's dV MMAs complete (P^T columns free)
+  B_COUNT = B_PT_FREE + 1
 };
 static_assert(B_COUNT <= SmemOffsets::n_bars, "barrier space");
 constexpr int kSchedConsumers = kEwWarps + 1 + 2 + 4;  // elementwise, MMA, RoPE, dQ warps
@@ -224,7 +225,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   uint8_t *sV = smem + SmemOffsets::v;
   uint8_t *sQ = smem + SmemOffsets::q;
   uint8_t *sG = smem + SmemOffsets::g;
-  uint8_t *sP = smem + SmemOffsets::pt;
   uint8_t *sDS = smem + SmemOffsets::ds;
   float *sLse = reinterpret_cast<float *>(smem + SmemOffsets::lse);
   float *sDel = reinterpret_cast<float *>(smem + SmemOffsets::del);
@@ -256,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     lcptx::mbar_init(ctx.bar(B_SDP), 1);
     lcptx::mbar_init(ctx.bar(B_PDS), kEwWarps);
     lcptx::mbar_init(ctx.bar(B_STEP), 1);
+    lcptx::mbar_init(ctx.bar(B_PT_FREE), 1);
     lcptx::mbar_init(ctx.bar(B_DQ_FULL), 1);
     lcptx::mbar_init(ctx.bar(B_DQ_EMPTY), 4);
     lcptx::mbar_init(ctx.bar(B_ACC), 1);
@@ -369,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const uint32_t q_mn = (lcptx::smem_addr(sQ) >> 4) | (512u << 16);
       const uint32_t g_mn = (lcptx::smem_addr(sG) >> 4) | (512u << 16);
       const uint32_t ds_mn = (lcptx::smem_addr(sDS) >> 4) | ((uint32_t)(kTileBytes >> 4) << 16);
-      const uint32_t pt_km = (lcptx::smem_addr(sP) >> 4) | (1u << 16);
       const uint32_t ds_km = (lcptx::smem_addr(sDS) >> 4) | (1u << 16);
       uint32_t st_free_ph = 0;
       // S^T = K' Q'^T and dP^T = V dO^T of step q (stage s) into TMEM, once the
@@ -417,11 +417,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             if (!ok) break;
           }
           lcptx::tc_fence_after();
-          // dV += P^T dO, dK' += dS^T Q': A = the 64-query tiles in shared memory
+          // dV += P^T dO with P^T in TMEM (only dO is read from shared memory);
+          // dK' += dS^T Q' with dS^T from the 64-query tiles in shared memory
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            lcptx::mma_ss(tmem + kColDV, desc(pt_km + (kk >> 2) * kTileLo + 2 * (kk & 3)),
+            lcptx::mma_ts(tmem + kColDV, tmem + kColPT + 8 * kk,
                           desc(g_mn + s * kTileLo + 128 * kk), kIdescAcc, (t > 0 || kk > 0) ? 1u : 0u);
+          lcptx::mma_commit(ctx.bar(B_PT_FREE));
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             lcptx::mma_ss(tmem + kColDK, desc(ds_km + (kk >> 2) * kTileLo + 2 * (kk & 3)),
@@ -623,10 +625,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         uint8_t *tile = sDS + half * kTileBytes;  // dS^T, this query block's MN-major chunk
         // 16 queries at a time; the next chunk's TMEM loads are in flight while
         // this one is computed (double buffer)
-        uint8_t *ptile = sP + half * kTileBytes;  // P^T, this query block's tile
         uint32_t sr[2][16], dr[2][16];
-        // the whole row's P^T and dS^T, packed, before the wait for the tiles
-        uint32_t pk[4][8], dk[4][8];
+        // P^T goes to TMEM chunk by chunk (the previous step's dV has read it
+        // by now); the whole row's dS^T is held, packed, until the previous
+        // step's dK / dQ are done with the shared-memory tiles
+        if (q_it > 0) {
+          ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
+          if (!ok) break;
+          lcptx::tc_fence_after();
+        }
+        uint32_t dk[4][8];
         lcptx::tmem_ld16(tST + 64 * half, sr[0]);
         lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
         lcptx::tmem_wait_ld();
@@ -644,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t(&scur)[16] = sr[k & 1];
           const uint32_t(&dcur)[16] = dr[k & 1];
           const int jb = k * 16;  // first query of the chunk within its block
+          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
@@ -655,27 +664,31 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
               pv[u] = pe;
               dv2[u] = pe * (__uint_as_float(dcur[2 * i + u]) - dl[j]) * p.scale;
             }
-            pk[k][i] = pack_bf16(pv[0], pv[1]);
+            pk[i] = pack_bf16(pv[0], pv[1]);
             dk[k][i] = pack_bf16(dv2[0], dv2[1]);
           }
+          // P^T row kr, queries 16k .. 16k + 15 of this block: 8 columns
+          lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk);
           if (k < 3) lcptx::tmem_wait_ld();
         }
-        if (q_it > 0) {  // the previous step's MMAs are done with the tiles
+        if (q_it > 0) {  // the previous step's dK / dQ are done with the dS^T tiles
           ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
-          if (!ok) break;
+          if (!ok) {
+            lcptx::tmem_wait_st();
+            break;
+          }
         }
-        // row kr of the P^T and dS^T tiles: 64 queries of this block, 128-byte
-        // swizzled; K-major for dV / dK, MN-major (dS) for dQ
+        // row kr of the dS^T tile: 64 queries of this block, 128-byte swizzled;
+        // K-major for dK, MN-major (dS) for dQ
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            *reinterpret_cast<uint4 *>(ptile + swz(kr, k * 2 + i)) =
-                make_uint4(pk[k][4 * i], pk[k][4 * i + 1], pk[k][4 * i + 2], pk[k][4 * i + 3]);
+          for (int i = 0; i < 2; ++i)
             *reinterpret_cast<uint4 *>(tile + swz(kr, k * 2 + i)) =
                 make_uint4(dk[k][4 * i], dk[k][4 * i + 1], dk[k][4 * i + 2], dk[k][4 * i + 3]);
-          }
         }
+        lcptx::tmem_wait_st();
+        lcptx::tc_fence_before();
         lcptx::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PDS));

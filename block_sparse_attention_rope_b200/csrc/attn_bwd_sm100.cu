@@ -626,15 +626,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         // 16 queries at a time; the next chunk's TMEM loads are in flight while
         // this one is computed (double buffer)
         uint32_t sr[2][16], dr[2][16];
-        // P^T goes to TMEM chunk by chunk (the previous step's dV has read it
-        // by now); the whole row's dS^T is held, packed, until the previous
-        // step's dK / dQ are done with the shared-memory tiles
-        if (q_it > 0) {
-          ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
-          if (!ok) break;
-          lcptx::tc_fence_after();
-        }
-        uint32_t dk[4][8];
+        // the whole row's P^T and dS^T, packed, before the waits for their
+        // space (the previous step's dV, then its dK / dQ)
+        uint32_t pk[4][8], dk[4][8];
         lcptx::tmem_ld16(tST + 64 * half, sr[0]);
         lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
         lcptx::tmem_wait_ld();
@@ -652,7 +646,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t(&scur)[16] = sr[k & 1];
           const uint32_t(&dcur)[16] = dr[k & 1];
           const int jb = k * 16;  // first query of the chunk within its block
-          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
@@ -664,13 +657,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
               pv[u] = pe;
               dv2[u] = pe * (__uint_as_float(dcur[2 * i + u]) - dl[j]) * p.scale;
             }
-            pk[i] = pack_bf16(pv[0], pv[1]);
+            pk[k][i] = pack_bf16(pv[0], pv[1]);
             dk[k][i] = pack_bf16(dv2[0], dv2[1]);
           }
-          // P^T row kr, queries 16k .. 16k + 15 of this block: 8 columns
-          lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk);
           if (k < 3) lcptx::tmem_wait_ld();
         }
+        // P^T row kr, this block's 64 queries: TMEM columns 32 * half .. + 31
+        if (q_it > 0) {
+          ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
+          if (!ok) break;
+          lcptx::tc_fence_after();
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk[k]);
         if (q_it > 0) {  // the previous step's dK / dQ are done with the dS^T tiles
           ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
           if (!ok) {

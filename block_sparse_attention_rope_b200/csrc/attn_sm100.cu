@@ -44,6 +44,7 @@
 #include "sm100_ptx.cuh"
 #include "sm100_sync.cuh"
 #include "sm100_rope.cuh"
+#include "sm100_math.cuh"
 
 namespace {
 
@@ -244,28 +245,6 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// 2^x on the FMA pipe, two lanes at once: x = n + f with n = rint(x) (by the
-// 1.5*2^23 rounding constant) and f in [-1/2, 1/2]; 2^f by a degree-3
-// polynomial fitted here by the Remez exchange for least maximum relative
-// error (7.5e-5, far below bf16's 2^-9); 2^n by adding n to the exponent
-// field.  Inputs below -126 are clamped (the result is then < 2^-125).
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 rnd = make_float2(12582912.f, 12582912.f);
-  const float2 t = __fadd2_rn(x, rnd);
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(0.0551716685f, 0.0551716685f), f,
-                        make_float2(0.242611125f, 0.242611125f));
-  p = __ffma2_rn(p, f, make_float2(0.693260968f, 0.693260968f));
-  p = __ffma2_rn(p, f, make_float2(0.999928057f, 0.999928057f));
-  float2 r;
-  r.x = __uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23));
-  r.y = __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23));
   return r;
 }
 
@@ -734,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
                 s[2 * j + 1] = x.y;
               }
               if (kPolyMask & (1u << (j & 7))) {
-                const float2 y = exp2_poly2(x);
+                const float2 y = lcsm100::exp2_poly2(x);
                 e[2 * (j & (kRing - 1))] = y.x;
                 e[2 * (j & (kRing - 1)) + 1] = y.y;
               } else {

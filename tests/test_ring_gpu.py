@@ -237,7 +237,7 @@ def test_lse_merge_parts_kernel(api, n_parts):
     assert np.all(o.transpose(0, 2, 1, 3)[~fin] == 0)
 
 
-@pytest.mark.parametrize("w,world", [(SMALL, 2), (SMALL, 4), (RAGGED, 3)])
+@pytest.mark.parametrize("w,world", [(SMALL, 1), (SMALL, 2), (SMALL, 4), (RAGGED, 3), (RAGGED, 5)])
 def test_ring_matches_oracle_and_full_forward(api, w, world):
     x = synthetic.make_inputs(w)
     Cb, Nb = blocks(w)

@@ -48,7 +48,7 @@ def parse():
     ap.add_argument("--sweep", action="store_true", help="also time the sparsity sweep")
     ap.add_argument("--no-extra", action="store_true", help="skip the 86,400-token line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward pass of --workload (one JSON line; for profiling)")
     ap.add_argument("--ring-only", type=int, default=0, metavar="RANKS",
@@ -287,33 +287,76 @@ def time_ring(api, synthetic, torch, name, world, stream, reps=3):
 
 
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):
-    """End to end through the public API: pinned host inputs -> device ->
-    forward -> result back to pinned host memory, every step."""
-    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
-    out_h = torch.empty_like(host["q"]).pin_memory()
+    """End to end through the public API: every step copies its inputs from
+    pinned host memory to the device, runs the forward, and reads the result
+    back into pinned host memory.  Timed two ways: serial (copy in, compute,
+    copy out, one after another on one stream) and pipelined as a serving loop
+    runs it (two device buffer sets; the host-to-device copy of step i+1 and
+    the device-to-host copy of step i-1 run on their own streams while step i
+    computes).  Returns (pipelined ms / step, serial ms / step, bytes in,
+    bytes out)."""
+    names = list(host.keys())
+    dev = [{k: torch.empty_like(host[k], device="cuda") for k in names} for _ in range(2)]
+    out_d = [torch.empty_like(dev[0]["q"]) for _ in range(2)]
+    out_h = [torch.empty_like(host["q"]).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_h[0].numel() * out_h[0].element_size()
 
-    def step():
-        for k, v in host.items():
-            dev[k].copy_(v, non_blocking=True)
+    def forward(b):
+        d = dev[b]
         if w.cached:
-            o = api.forward_cached(dev["q"], dev["k"], dev["v"], dev["cond_k"], dev["cond_v"],
-                                   plan, rope, stream=stream)
+            api.forward_cached(d["q"], d["k"], d["v"], d["cond_k"], d["cond_v"], plan, rope,
+                               out=out_d[b], stream=stream)
         else:
-            o = api.forward(dev["q"], dev["k"], dev["v"], plan, rope, stream=stream)
-        out_h.copy_(o, non_blocking=True)
+            api.forward(d["q"], d["k"], d["v"], plan, rope, out=out_d[b], stream=stream)
 
-    with torch.cuda.stream(stream):
-        step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(steps):
-            step()
-        e1.record(stream)
+    def serial_step():
+        with torch.cuda.stream(stream):
+            for k in names:
+                dev[0][k].copy_(host[k], non_blocking=True)
+            forward(0)
+            out_h[0].copy_(out_d[0], non_blocking=True)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    serial_step()
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps, h2d, d2h
+    e0, e1 = ev(), ev()
+    e0.record(stream)
+    for _ in range(steps):
+        serial_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    serial_ms = e0.elapsed_time(e1) / steps
+
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    out_done = [torch.cuda.Event() for _ in range(2)]
+    t0, t1 = ev(), ev()
+    t0.record(s_in)
+    for i in range(steps + 1):  # one extra step: the first fills the pipeline untimed
+        b = i % 2
+        if i == 1:
+            torch.cuda.synchronize()
+            t0.record(s_in)
+        if i >= 2:
+            s_in.wait_event(comp_done[b])      # step i-2 has read dev[b]
+        with torch.cuda.stream(s_in):
+            for k in names:
+                dev[b][k].copy_(host[k], non_blocking=True)
+            in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        if i >= 2:
+            stream.wait_event(out_done[b])     # step i-2's result has left out_d[b]
+        forward(b)
+        comp_done[b].record(stream)
+        s_out.wait_event(comp_done[b])
+        with torch.cuda.stream(s_out):
+            out_h[b].copy_(out_d[b], non_blocking=True)
+            out_done[b].record(s_out)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return t0.elapsed_time(t1) / steps, serial_ms, h2d, d2h
 
 
 def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, stream, e2e_steps=0):
@@ -335,8 +378,8 @@ def measure_workload(api, synthetic, torch, name, steps, warmup, dist, rank, str
     if e2e_steps:
         del d, out
         torch.cuda.empty_cache()
-        res["e2e_ms"], res["h2d"], res["d2h"] = time_e2e(api, torch, w, host, plan, rope,
-                                                         e2e_steps, stream)
+        res["e2e_ms"], res["e2e_serial_ms"], res["h2d"], res["d2h"] = time_e2e(
+            api, torch, w, host, plan, rope, e2e_steps, stream)
     return res
 
 
@@ -453,10 +496,16 @@ def run_ours(a):
                                e2e_steps=a.e2e_steps)
         e2e_ms = res["e2e_ms"]
         e2e_ms = max_over_ranks(e2e_ms, dist)
+        serial_ms = max_over_ranks(res["e2e_serial_ms"], dist)
         e2e = {"value": round(world * res["flops"] / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": res["h2d"],
                "d2h_bytes_per_step": res["d2h"],
-               "path": "pinned host q/k/v -> device, lc_bsa_forward, out -> pinned host"}
+               "path": "pinned host q/k/v -> device, lc_bsa_forward, out -> pinned host; "
+                       "pipelined: the copy in of step i+1 and the copy out of step i-1 run "
+                       "on their own streams while step i computes",
+               "serial": {"value": round(world * res["flops"] / (serial_ms * 1e-3) / 1e12, 3),
+                          "ms_per_step": round(serial_ms, 3),
+                          "path": "copy in, forward, copy out one after another"}}
     extra = {}
     names = [] if a.no_extra else ["refine_720p"]
     if a.sweep:

@@ -88,3 +88,44 @@ def test_python_binding_imports_only_the_library():
     for f in os.listdir(os.path.join(ROOT, "block_sparse_attention_rope_b200", "csrc")):
         assert "oracle" not in open(os.path.join(ROOT, "block_sparse_attention_rope_b200",
                                                  "csrc", f)).read().lower()
+
+
+def test_ring_entry_points_reject_bad_arguments(lib):
+    vp, I, LL, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float
+    h = ctypes.c_void_p()
+    f = lib.lc_bsa_plan_create_shard
+    f.argtypes = [ctypes.POINTER(vp)] + [I] * 11 + [vp]
+    # T=5, H=8, W=40, 2 condition frames: Cb = 10, Nb = 15 (25 blocks)
+    assert f(None, 5, 8, 40, 64, 1, 2, 2, 0, 4, 0, 25, None) == 1
+    assert f(ctypes.byref(h), 5, 8, 40, 64, 1, 2, 2, 0, 6, 0, 25, None) == 1   # inside a group
+    assert f(ctypes.byref(h), 5, 8, 40, 64, 1, 2, 2, 10, 13, 0, 25, None) == 1  # inside a group
+    assert f(ctypes.byref(h), 5, 8, 40, 64, 1, 2, 2, 0, 4, 0, 26, None) == 1   # past the end
+    assert f(ctypes.byref(h), 5, 8, 40, 64, 1, 2, 2, 4, 0, 0, 25, None) == 1   # lo > hi
+    assert f(ctypes.byref(h), 5, 8, 40, 64, 1, 2, 2, 0, -1, 0, 25, None) == 1
+    assert h.value is None
+    g = lib.lc_bsa_forward_shard
+    g.argtypes = [vp] * 5 + [I] * 4 + [F] + [vp] * 4
+    assert g(None, None, None, None, None, 1, 2, 64, 0, 0.0, None, None, None, None) == 1
+    m = lib.lc_bsa_lse_merge
+    m.argtypes = [vp] * 5 + [I, LL, I, I, I, ctypes.c_uint, vp]
+    buf = ctypes.create_string_buffer(4096 + 16)
+    a = (ctypes.addressof(buf) + 15) & ~15
+    assert m(None, a, a, a, None, 1, 4, 2, 64, 0, 0, None) == 1       # o_acc needed
+    assert m(a, a, a, a, None, 1, 4, 2, 64, 0, 8, None) == 1          # unknown flag
+    assert m(a, a, a, a, None, 1, 4, 2, 32, 0, 0, None) == 2          # head_dim
+    assert m(a, a, a + 4, a, None, 1, 4, 2, 64, 0, 0, None) == 1      # misaligned part
+    p = lib.lc_bsa_lse_merge_parts
+    p.argtypes = [vp, vp, I, vp, vp, I, LL, I, I, I, vp]
+    assert p(a, a, 0, a, None, 1, 4, 2, 64, 0, None) == 1             # no parts
+    assert p(None, a, 2, a, None, 1, 4, 2, 64, 0, None) == 1
+    assert p(a, a, 2, a, None, 1, 4, 2, 32, 0, None) == 2
+    r = lib.lc_rope3d_apply_ex
+    r.argtypes = [vp, vp, I, LL, I, I, LL, I, vp, F, vp, vp]
+    assert r(None, None, 1, 4, 2, 64, 0, 0, None, 0.0, None, None) == 1
+
+
+def test_package_never_reaches_the_oracle():
+    pkg = os.path.join(ROOT, "block_sparse_attention_rope_b200")
+    for f in ("api.py", "ring.py", "build.py", "__init__.py"):
+        src = open(os.path.join(pkg, f)).read()
+        assert "import oracle" not in src and "from oracle" not in src, f

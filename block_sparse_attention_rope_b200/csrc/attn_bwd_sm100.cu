@@ -15,18 +15,23 @@
 //     S^T  = K' Q'^T        dP^T = V dO^T          (tcgen05, into TMEM)
 //     P^T  = exp(scale S^T - lse),  dS^T = P^T (dP^T - D) scale
 //                           (warps 0-7, one key row and query block per
-//                            thread; P^T and dS^T written as bf16 tiles to
+//                            thread, the whole row formed before the waits
+//                            for the previous step's MMAs; P^T written as
+//                            bf16 pairs into TMEM, dS^T as bf16 tiles into
 //                            shared memory, so the next step's S^T, dP^T can
 //                            be computed while they are formed)
-//     dV  += P^T dO         dK' += dS^T Q'         (A from shared memory)
+//     dV  += P^T dO         (A = P^T from TMEM, only dO read from shared memory)
+//     dK' += dS^T Q'        (A from shared memory)
 //     dQ'  = dS K'          (A = dS from shared memory, MN-major; queries as
-//                            TMEM lanes), added to the fp32 buffer by warps
-//                            12-15 with vector reductions
+//                            TMEM lanes), staged in shared memory by warps
+//                            12-15 and added to the fp32 buffer by TMA
+//                            reduce-adds
 //   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
 //   warp 8: TMA producer (K', V per item; Q', dO per step, 2 stages); warp 9: MMA issuer; warps 10-11: stage lse / D per step.
 //   Q' = R(norm(q)) and K' = R(norm(k)) are formed once, before the kernel,
 //   by the one-pass rotation the forward uses for K (same arithmetic).
-//   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448).
+//   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448)
+//         P^T [448,512).
 // Every mbarrier wait is bounded; on expiry the CTA stops, drains and frees
 // TMEM, and LC_DEVSTAT_TIMEOUT is set.
 #include <cuda.h>

@@ -29,6 +29,11 @@
 //               O / l through shared memory to a TMA store, plus the LSE.
 //   TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384)
 //               P0 [384,448) P1 [448,512).
+// Launch modes (lc_fwd_mode): the whole sequence; the noisy queries with the
+// condition K/V from separate tensors (cache consumer); the condition queries
+// alone (cache producer); one shard pair of ring context parallelism (q / out
+// and k / v hold token ranges of the sequence, addressed through per-segment
+// tensor maps and row offsets; q and k may arrive rotated).
 // Every wait on an mbarrier is bounded (globaltimer); on expiry the kernel
 // flags LC_DEVSTAT_TIMEOUT in the device status word, stops all roles of the
 // CTA, drains its own copies and MMAs, frees TMEM and returns.

@@ -29,6 +29,10 @@ CASES = {
                            dtype="f32"),
     "local_f32": Workload("local_f32", T=2, H=10, W=30, n_cond=0, heads=3, local=0, stride=0,
                           dtype="f32"),
+    "short_noisy": Workload("short_noisy", T=4, H=6, W=10, n_cond=3, heads=2, local=1, stride=2,
+                            dtype="bf16"),
+    "tiny_tokens": Workload("tiny_tokens", T=5, H=1, W=7, n_cond=2, heads=2, local=0, stride=3,
+                            dtype="bf16"),
 }
 
 

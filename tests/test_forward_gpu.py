@@ -33,6 +33,19 @@ SMALL = {
                               stride=4, dtype="bf16", cached=True),
     "ragged_f32": Workload("ragged_f32", T=6, H=13, W=21, n_cond=1, heads=3, local=1, stride=3,
                            dtype="f32"),
+    # degenerate shapes: a noisy segment shorter than one block after three
+    # condition frames; one token row per frame (both segments one partial
+    # block); a stride past the last block (block 0 is the only global one)
+    "short_noisy": Workload("short_noisy", T=4, H=6, W=10, n_cond=3, heads=2, local=1, stride=2,
+                            dtype="bf16"),
+    "short_noisy_cached": Workload("short_noisy_cached", T=4, H=6, W=10, n_cond=3, heads=2,
+                                   local=1, stride=2, dtype="bf16", cached=True),
+    "tiny_tokens": Workload("tiny_tokens", T=5, H=1, W=7, n_cond=2, heads=2, local=0, stride=3,
+                            dtype="bf16"),
+    "tiny_tokens_f32": Workload("tiny_tokens_f32", T=5, H=1, W=7, n_cond=2, heads=2, local=0,
+                                stride=3, dtype="f32"),
+    "stride_past_end": Workload("stride_past_end", T=3, H=8, W=16, n_cond=0, heads=2, local=0,
+                                stride=100, dtype="bf16"),
     "cached_f32": Workload("cached_f32", T=5, H=8, W=20, n_cond=2, heads=2, local=1, stride=3,
                            dtype="f32", cached=True),
 }

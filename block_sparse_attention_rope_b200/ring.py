@@ -86,7 +86,11 @@ class RingSchedule:
 
 def _exchange(send: Sequence[torch.Tensor], recv: Sequence[torch.Tensor], dst: int, src: int,
               group) -> list:
+    """Send to ring neighbour `dst`, receive from `src` (ranks within `group`,
+    None = the default group), as one batched group of point-to-point ops."""
     import torch.distributed as dist
+    if group is not None:
+        dst, src = dist.get_global_rank(group, dst), dist.get_global_rank(group, src)
     ops = [dist.P2POp(dist.isend, t, dst, group) for t in send]
     ops += [dist.P2POp(dist.irecv, t, src, group) for t in recv]
     return dist.batch_isend_irecv(ops)

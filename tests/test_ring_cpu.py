@@ -138,3 +138,48 @@ def test_schedule_sources_and_skips():
     s2 = _schedule(shards, 2)
     assert s2.sources == [2, 1, 0, 3] and all(s2.computes)
     assert s0.tokens[1] == (256, 640) and s0.tokens[2] == (640, 1152)
+
+
+def _worker_subgroup(rank, world, port, shards, qout):
+    """Ranks 0 and 2 of three form the ring (a process subgroup); rank 1 only
+    takes part in creating the group."""
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        group = dist.new_group([0, 2])
+        if rank == 1:
+            qout.put(None)
+            return
+        grank = dist.get_rank(group)
+        q, k, v = (torch.from_numpy(a) for a in _inputs())
+        sched = _schedule(shards, grank)
+        a, b = sched.tokens[grank]
+        partial, combine = _oracle_steps(sched)
+        o, l = ring.ring_forward(sched, q[:, a:b].contiguous(), k[:, a:b].contiguous(),
+                                 v[:, a:b].contiguous(), partial, combine, group=group)
+        qout.put((grank, a, b, o.numpy(), l.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_over_a_process_subgroup():
+    shards = ring.balanced_shards(_work(), 10, 2)
+    ctx = mp.get_context("spawn")
+    qout = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_subgroup, args=(r, 3, port, shards, qout))
+             for r in range(3)]
+    for p in procs:
+        p.start()
+    res = [qout.get(timeout=300) for _ in range(3)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    res = sorted((r for r in res if r is not None), key=lambda r: r[0])
+    assert len(res) == 2
+    q, k, v = _inputs()
+    ref_o, ref_l = oracle.forward(q, k, v, **GEOM)
+    for grank, a, b, o, l in res:
+        assert np.abs(o - ref_o[:, a:b]).max() <= 1e-12 * np.abs(ref_o).max()
+        assert np.abs(l - ref_l[:, :, a:b]).max() <= 1e-12 * np.abs(ref_l).max()

@@ -52,6 +52,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward pass of --workload (one JSON line; for profiling)")
+    ap.add_argument("--plan-only", action="store_true",
+                    help="time only the planner and the RoPE tables of --workload (one JSON "
+                         "line; for profiling)")
     ap.add_argument("--ring-only", type=int, default=0, metavar="RANKS",
                     help="time only the ring over RANKS ranks (all in this process) on "
                          "--workload (one JSON line; for profiling)")
@@ -621,6 +624,30 @@ def main():
                           torch.cuda.current_stream())
         print(json.dumps(dict(metric="backward ms per layer", value=r["ms_per_layer"], unit="ms",
                               higher_is_better=False, **r)), flush=True)
+    elif a.plan_only:
+        import torch
+        torch.cuda.set_device(0)
+        from block_sparse_attention_rope_b200 import api, synthetic
+        w = synthetic.get(a.workload)
+        st = torch.cuda.current_stream()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        for _ in range(2):  # warm-up (first-call setup outside the timed pass)
+            api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond).close()
+            api.Rope3D(w.T, w.H, w.W).close()
+        torch.cuda.synchronize()
+        n = max(1, a.steps)
+        ev[0].record(st)
+        plans = [api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+                 for _ in range(n)]
+        ev[1].record(st)
+        ropes = [api.Rope3D(w.T, w.H, w.W) for _ in range(n)]
+        ev[2].record(st)
+        torch.cuda.synchronize()
+        inf = plans[0].info()
+        print(json.dumps(dict(metric="plan build ms", value=round(ev[0].elapsed_time(ev[1]) / n, 4),
+                              unit="ms", higher_is_better=False, workload=w.name,
+                              rope_tables_ms=round(ev[1].elapsed_time(ev[2]) / n, 4),
+                              nnz=inf.nnz, num_q_blocks=inf.num_q_blocks)), flush=True)
     elif a.ring_only:
         import torch
         torch.cuda.set_device(0)

@@ -227,6 +227,27 @@ def test_full_size_sampled_rows(api, name):
                                                                   mean, lerr))
 
 
+@pytest.mark.parametrize("name", ["i2v_480p", "refine_720p"])
+def test_full_size_all_rows_of_two_heads(api, name):
+    """Every query row of heads 0 and 31 at full size (the benchmark's launch),
+    element by element against the oracle."""
+    w = synthetic.get(name)
+    inputs = synthetic.make_inputs(w)
+    out, lse = run_gpu(api, w, inputs)
+    heads = [0, w.heads - 1]
+    sub = {k: v[:, :, heads].contiguous() for k, v in inputs.items()}
+    ref_out, ref_lse = oracle.attention_rows(
+        sub["q"], sub["k"], sub["v"], H=w.H, W=w.W, Nc=w.n_cond_tokens, block=w.block,
+        local=w.local, stride=w.stride, rows=oracle.all_rows(1, w.n_tokens, 2))
+    g = out[0][:, heads].float().numpy().astype(np.float64).transpose(1, 0, 2).reshape(-1, 64)
+    err = np.abs(g - ref_out)
+    assert err.max() <= parity.BF16_MAX_ABS and err.mean() <= parity.BF16_MEAN_ABS, \
+        (err.max(), err.mean())
+    gl = lse[0][heads].numpy().astype(np.float64).reshape(-1)
+    assert np.abs(gl - ref_lse).max() <= parity.BF16_LSE_ABS
+    print("%s all rows of heads %s: max %.3g mean %.3g" % (name, heads, err.max(), err.mean()))
+
+
 def test_argument_errors_on_gpu(api):
     w = SMALL["small_i2v"]
     plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)

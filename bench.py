@@ -250,8 +250,10 @@ def time_ring(api, synthetic, torch, name, world, stream, reps=3):
     x = synthetic.make_inputs(w, device="cuda")
     plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
     rope = api.Rope3D(w.T, w.H, w.W)
-    rp, _ = plan.csr()
-    shards = ring.balanced_shards(np.diff(rp.numpy()), plan.info().num_cond_blocks, world)
+    rp, ci = plan.csr()
+    cb = plan.info().num_cond_blocks
+    shards = ring.planned_shards(rp.tolist(), ci.tolist(), cb, world, heads=w.heads,
+                                 batch=w.batch)
     ranks = [ring.GpuRingRank(api, w.T, w.H, w.W, local=w.local, stride=w.stride,
                               n_cond=w.n_cond, shards=shards, rank=r, rope=rope, batch=w.batch,
                               heads=w.heads) for r in range(world)]

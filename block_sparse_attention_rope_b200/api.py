@@ -90,6 +90,7 @@ lib = _load()
 COND_K_ROTATED = 1  # LC_FLAG_COND_K_ROTATED
 Q_ROTATED = 2       # LC_FLAG_Q_ROTATED
 K_ROTATED = 4       # LC_FLAG_K_ROTATED
+KEEP_EMPTY_ROWS = 8  # LC_FLAG_KEEP_EMPTY_ROWS
 
 
 def status_string(s: int) -> str:
@@ -433,7 +434,8 @@ def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
                   *, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                   softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
                   k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
-                  q_rotated: bool = False, k_rotated: bool = False, stream=None):
+                  q_rotated: bool = False, k_rotated: bool = False,
+                  keep_empty_rows: bool = False, stream=None):
     """Partial attention of one shard pair (lc_bsa_forward_shard): q holds the
     shard plan's query tokens [B, nq, heads, 64], k / v its key tokens
     [B, nk, heads, 64] (pre-RoPE, bf16, or already normalised and rotated with
@@ -450,7 +452,8 @@ def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
         lse = torch.empty(B, heads, nq, dtype=torch.float32, device=q.device)
     _check_bmhk("out", out, q.shape, q.dtype)
     _check_bmhk("lse", lse, (B, heads, nq), torch.float32)
-    flags = (Q_ROTATED if q_rotated else 0) | (K_ROTATED if k_rotated else 0)
+    flags = ((Q_ROTATED if q_rotated else 0) | (K_ROTATED if k_rotated else 0) |
+             (KEEP_EMPTY_ROWS if keep_empty_rows else 0))
     opts = _opts(flags, q_norm, k_norm, norm_eps, hd)
     _check(lib.lc_bsa_forward_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     lse.data_ptr(), B, heads, hd, _dtype_code(q),

@@ -274,7 +274,8 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   if (s != LC_OK) return s;
   unsigned flags;
   lc_qk_norm norm;
-  if (!parse_opts(opts, LC_FLAG_Q_ROTATED | LC_FLAG_K_ROTATED, &flags, &norm))
+  if (!parse_opts(opts, LC_FLAG_Q_ROTATED | LC_FLAG_K_ROTATED | LC_FLAG_KEEP_EMPTY_ROWS, &flags,
+                  &norm))
     return LC_ERR_INVALID_ARGUMENT;
   if (!q || !k || !v || !out || !lse) return LC_ERR_INVALID_ARGUMENT;
   if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
@@ -295,7 +296,8 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   if (s != LC_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Rows of groups without entries (out = 0, lse = -inf); the kernel writes the rest.
-  s = lc_launch_shard_fill(plan, out, lse, batch, heads, dtype, st);
+  if (!(flags & LC_FLAG_KEEP_EMPTY_ROWS))
+    s = lc_launch_shard_fill(plan, out, lse, batch, heads, dtype, st);
   if (s != LC_OK || plan->G_active == 0) return s;
   return lc_launch_forward_sm100(q, k, v, nullptr, nullptr, out, lse, batch, heads, scale,
                                  LC_FWD_SHARD, false, norm, plan, rope, dev_status, st, nullptr,

@@ -4,7 +4,8 @@ myzaker / QbitAI "美团视频生成模型来了！一出手就是开源 SOTA", 
 "背后技术原理": the high-resolution pass pairs block-sparse attention with
 context-parallel ring block-sparse attention.  Here: the sequence's blocks are
 cut into contiguous shards, one per rank (query bounds on 4-block group
-edges, balanced by the plan's per-block work); a rank keeps its query shard,
+edges; `planned_shards` picks the cuts with a model of the kernel's work
+items, which fill the SMs in whole waves); a rank keeps its query shard,
 and at step s holds the K/V shard of rank (r - s) mod world, which it passes
 on to rank r + 1 while it computes (NCCL send/recv over NVLink, one
 batched group per step, on the communicator's own stream so the transfer
@@ -42,9 +43,9 @@ def balanced_shards(work: Sequence[int], Cb: int, world: int) -> List[Tuple[int,
     edges = group_edges(Cb, nq - Cb)
     if len(edges) - 1 < world:
         raise ValueError("%d query groups cannot be split over %d ranks" % (len(edges) - 1, world))
-    pre = [0]
+    pre = [0.0]
     for w in work:
-        pre.append(pre[-1] + int(w))
+        pre.append(pre[-1] + float(w))
     total = pre[-1]
     cuts = [0]
     for i in range(1, world):
@@ -57,9 +58,138 @@ def balanced_shards(work: Sequence[int], Cb: int, world: int) -> List[Tuple[int,
     return [(cuts[i], cuts[i + 1]) for i in range(world)]
 
 
+# Cost of a query block in the tensor-core kernel, in units of its CSR
+# entries: a work item (4 query blocks) costs about 8,500 cycles beyond its
+# key tiles (3,070 cycles per 2-block tile for both query tiles), i.e. about
+# 5.5 entries per block (least-squares fit over the sparsity sweep on B200).
+ITEM_OVERHEAD_ENTRIES = 5.5
+
+
+def block_work(row_counts: Sequence[int], num_cond_blocks: int = 0) -> List[float]:
+    """Per query block: its CSR entries plus its share of the per-item cost,
+    the work measure `balanced_shards` splits evenly."""
+    return [float(c) + ITEM_OVERHEAD_ENTRIES for c in row_counts]
+
+
 def block_token(r: int, Nc: int, Cb: int, N: int, block: int = 64) -> int:
     """First token of block r in the whole sequence (r == block count: N)."""
     return min(block * r if r < Cb else Nc + block * (r - Cb), N)
+
+
+# Cycles of one work item of the tensor-core kernel beyond its key tiles, and
+# of one 2-block key tile (both query tiles), from a least-squares fit over
+# the sparsity sweep on B200; used only to compare shard layouts.
+ITEM_CYCLES = 8500.0
+TILE_CYCLES = 3070.0
+STEP_CYCLES = 30000.0  # per computing step: launch and kernel ramp (ring measurements)
+
+
+def _group_unions(row_ptr: Sequence[int], col_idx: Sequence[int], Cb: int):
+    """Per work item group (4 query blocks of one segment): first block and
+    the sorted union of its members' key blocks."""
+    nq = len(row_ptr) - 1
+    out = []
+    for seg_lo, seg_hi in ((0, Cb), (Cb, nq)):
+        for g0 in range(seg_lo, seg_hi, 4):
+            u = set()
+            for r in range(g0, min(g0 + 4, seg_hi)):
+                u.update(int(c) for c in col_idx[row_ptr[r]:row_ptr[r + 1]])
+            out.append((g0, sorted(u)))
+    return out
+
+
+def _makespan(costs: List[float], n_sm: int) -> float:
+    """Finish time of items taken in order by n_sm persistent CTAs, each CTA
+    taking the next item as soon as it is free (the kernel's atomic queue)."""
+    import heapq
+    if not costs:
+        return 0.0
+    free = [0.0] * min(n_sm, len(costs))
+    heapq.heapify(free)
+    end = 0.0
+    for c in costs:
+        t = heapq.heappop(free) + c
+        end = max(end, t)
+        heapq.heappush(free, t)
+    return end
+
+
+def modeled_rank_cycles(shards: Sequence[Tuple[int, int]], row_ptr: Sequence[int],
+                        col_idx: Sequence[int], Cb: int, heads: int, batch: int = 1,
+                        n_sm: int = 148, unions=None, cache=None) -> List[float]:
+    """Modeled device cycles of each rank's ring: per step, the makespan of
+    the step's work items (one per batch entry, head and active group; cost =
+    ITEM_CYCLES + TILE_CYCLES x key tiles in the source shard, longest first,
+    head-major, as the kernel orders them) on n_sm CTAs."""
+    import bisect
+    import math
+    unions = unions if unions is not None else _group_unions(row_ptr, col_idx, Cb)
+    out = []
+    cache = {} if cache is None else cache
+    for r, (qa, qb) in enumerate(shards):
+        groups = None
+        total = 0.0
+        for ka, kb in shards:
+            key = (qa, qb, ka, kb)
+            if key not in cache:
+                if groups is None:
+                    groups = [u for g0, u in unions if qa <= g0 < qb]
+                tiles = [math.ceil((bisect.bisect_left(u, kb) - bisect.bisect_left(u, ka)) / 2)
+                         for u in groups]
+                lens = sorted((t for t in tiles if t > 0), reverse=True)
+                costs = [ITEM_CYCLES + TILE_CYCLES * t for t in lens] * (heads * batch)
+                cache[key] = _makespan(costs, n_sm) + STEP_CYCLES if lens else 0.0
+            total += cache[key]
+        out.append(total)
+    return out
+
+
+def planned_shards(row_ptr: Sequence[int], col_idx: Sequence[int], Cb: int, world: int,
+                   heads: int, batch: int = 1, n_sm: int = 148,
+                   max_rounds: int = 8) -> List[Tuple[int, int]]:
+    """Shard layout for the ring that minimises the slowest rank's modeled
+    time (modeled_rank_cycles): start from the layout even in work, then take
+    the best move of a run of consecutive cuts by one or two group edges,
+    while the slowest rank (then the total) improves.  The model captures what an even
+    split of work misses: each step's items fill the SMs in whole waves."""
+    nq = len(row_ptr) - 1
+    counts = [row_ptr[r + 1] - row_ptr[r] for r in range(nq)]
+    shards = balanced_shards(block_work(counts, Cb), Cb, world)
+    if world == 1:
+        return shards
+    unions = _group_unions(row_ptr, col_idx, Cb)
+    edges = group_edges(Cb, nq - Cb)
+    pos = {e: k for k, e in enumerate(edges)}
+    cuts = [pos[a] for a, _ in shards[1:]]  # as edge indices
+
+    def layout(c):
+        b = [0] + [edges[k] for k in c] + [nq]
+        return [(b[i], b[i + 1]) for i in range(len(b) - 1)]
+
+    cache = {}
+
+    def cost(c):
+        t = modeled_rank_cycles(layout(c), row_ptr, col_idx, Cb, heads, batch, n_sm, unions,
+                                cache)
+        return max(t), sum(t)
+
+    best = cost(cuts)
+    for _ in range(max_rounds):
+        cand_best, cand = best, None
+        for i in range(len(cuts)):
+            for j in range(i, len(cuts)):
+                for d in (-2, -1, 1, 2):
+                    c = cuts[:i] + [k + d for k in cuts[i:j + 1]] + cuts[j + 1:]
+                    if c[0] < 1 or c[-1] > len(edges) - 2 or any(
+                            c[m] >= c[m + 1] for m in range(len(c) - 1)):
+                        continue
+                    cc = cost(c)
+                    if cc < cand_best:
+                        cand_best, cand = cc, c
+        if cand is None:
+            break
+        best, cuts = cand_best, cand
+    return layout(cuts)
 
 
 class RingSchedule:
@@ -159,8 +289,11 @@ class GpuRingRank:
         self.sched = RingSchedule(shards, Nc, Cb, N, rank, lambda r, src: src in self.plans)
         nq = self.sched.n_tokens(rank)
         n_parts = sum(self.sched.computes)
-        self.parts = torch.empty(n_parts, batch, nq, heads, 64, dtype=dtype, device=device)
-        self.lses = torch.empty(n_parts, batch, heads, nq, dtype=torch.float32, device=device)
+        # Rows that a step's shard gives no key stay (0, -inf) from here on:
+        # each slot always holds the same step, so the launches skip them.
+        self.parts = torch.zeros(n_parts, batch, nq, heads, 64, dtype=dtype, device=device)
+        self.lses = torch.full((n_parts, batch, heads, nq), -float("inf"), dtype=torch.float32,
+                               device=device)
 
     def rotate(self, x: torch.Tensor, shard: int, norm) -> torch.Tensor:
         """R(norm(x)) of shard `shard`'s tokens at their sequence positions."""
@@ -170,7 +303,7 @@ class GpuRingRank:
     def partial(self, src, q_rot, k_rot, v, slot):
         self.api.forward_shard(q_rot, k_rot, v, self.plans[src], self.rope, out=self.parts[slot],
                                lse=self.lses[slot], softmax_scale=self.softmax_scale,
-                               q_rotated=True, k_rotated=True)
+                               q_rotated=True, k_rotated=True, keep_empty_rows=True)
         return slot
 
     def combine(self, slots):

@@ -198,6 +198,8 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
 #define LC_FLAG_COND_K_ROTATED 1u  /* cond_k already holds R(k) (lc_bsa_cond_cache) */
 #define LC_FLAG_Q_ROTATED 2u       /* q already holds R(norm_q(q)) (lc_bsa_forward_shard) */
 #define LC_FLAG_K_ROTATED 4u       /* k already holds R(norm_k(k)) (lc_bsa_forward_shard) */
+#define LC_FLAG_KEEP_EMPTY_ROWS 8u /* lc_bsa_forward_shard: rows of work groups without keys
+                                      in the shard are left as they are (not set to 0, -inf) */
 
 /*
  * Options of the _ex entry points and of lc_bsa_cond_cache.  A NULL options
@@ -359,7 +361,11 @@ lc_status lc_bsa_plan_token_range(lc_bsa_plan plan, long long *q_lo, long long *
  * LC_FLAG_Q_ROTATED / LC_FLAG_K_ROTATED when q / k already hold the
  * normalised, rotated values (lc_rope3d_apply_ex at their whole-sequence
  * positions): a ring rotates each shard once and reuses it at every step.
- * The result is the same bits either way.  bf16 only (LC_DTYPE_F32:
+ * The result is the same bits either way.  LC_FLAG_KEEP_EMPTY_ROWS: rows of
+ * the plan's work groups (4 query blocks) that have no key in the shard are
+ * not written, for a caller whose buffers already hold (0, -inf) there (the
+ * set of such rows is fixed by the plan); rows of groups with keys are always
+ * written, (0, -inf) included.  bf16 only (LC_DTYPE_F32:
  * LC_ERR_UNSUPPORTED).  Errors as lc_bsa_forward.
  */
 lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void *out, float *lse,

@@ -183,3 +183,25 @@ def test_ring_over_a_process_subgroup():
     for grank, a, b, o, l in res:
         assert np.abs(o - ref_o[:, a:b]).max() <= 1e-12 * np.abs(ref_o).max()
         assert np.abs(l - ref_l[:, :, a:b]).max() <= 1e-12 * np.abs(ref_l).max()
+
+
+def test_planned_shards_model():
+    """The shard planner: a valid layout on group edges whose modeled slowest
+    rank is no worse than the even-work layout's; the model sees the wave
+    step when a shard's items per step pass a multiple of the SM count."""
+    rp, ci = oracle.block_csr(24, 30, 52, 64, 2, 4, 1)     # I2V 480p: Cb 25, Nb 561
+    edges = set(ring.group_edges(25, 561))
+    even = ring.balanced_shards(ring.block_work(np.diff(rp), 25), 25, 8)
+    planned = ring.planned_shards(rp, ci, 25, 8, heads=32)
+    assert planned[0][0] == 0 and planned[-1][1] == 586
+    assert all(a < b and a in edges and b in edges for a, b in planned)
+    assert all(planned[i][1] == planned[i + 1][0] for i in range(7))
+    t_even = ring.modeled_rank_cycles(even, rp, ci, 25, 32)
+    t_plan = ring.modeled_rank_cycles(planned, rp, ci, 25, 32)
+    assert max(t_plan) <= max(t_even)
+    # 18 noisy groups x 32 heads = 576 items fill 148 SMs in 4 waves, 19 need 5
+    lay18 = [(0, 25), (25, 97), (97, 586)]
+    lay19 = [(0, 25), (25, 101), (101, 586)]
+    t18 = ring.modeled_rank_cycles(lay18, rp, ci, 25, 32)[1]
+    t19 = ring.modeled_rank_cycles(lay19, rp, ci, 25, 32)[1]
+    assert t19 > t18 * 1.1

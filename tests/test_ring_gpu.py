@@ -211,6 +211,28 @@ def test_prerotated_shards_are_bit_exact(api):
             assert torch.equal(o1, o3) and torch.equal(l1, l3)
 
 
+def test_keep_empty_rows_leaves_groups_without_keys(api):
+    """With LC_FLAG_KEEP_EMPTY_ROWS the rows of work groups that have no key in
+    the shard are not written; every other row is the same as without it."""
+    w = SMALL
+    x = synthetic.make_inputs(w, device="cuda")
+    rope = api.Rope3D(w.T, w.H, w.W)
+    p = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                 q_blocks=(0, 18), k_blocks=(18, 25))   # condition groups see no key here
+    (qa, qb), (ka, kb) = p.q_tokens, p.k_tokens
+    q, k, v = (x[n][:, a:b].contiguous() for n, a, b in
+               (("q", qa, qb), ("k", ka, kb), ("v", ka, kb)))
+    o1, l1 = api.forward_shard(q, k, v, p, rope)
+    o2 = torch.full_like(o1, float("nan"))
+    l2 = torch.full_like(l1, float("nan"))
+    api.forward_shard(q, k, v, p, rope, out=o2, lse=l2, keep_empty_rows=True)
+    torch.cuda.synchronize()
+    Nc = w.n_cond_tokens                                  # 640: the condition rows
+    assert torch.isnan(o2[:, :Nc]).all() and torch.isnan(l2[:, :, :Nc]).all()
+    assert torch.equal(o2[:, Nc:], o1[:, Nc:]) and torch.equal(l2[:, :, Nc:], l1[:, :, Nc:])
+    assert (o1[:, :Nc] == 0).all() and (l1[:, :, :Nc] == -float("inf")).all()
+
+
 @pytest.mark.parametrize("n_parts", [1, 3, 8])
 def test_lse_merge_parts_kernel(api, n_parts):
     g = torch.Generator().manual_seed(n_parts)

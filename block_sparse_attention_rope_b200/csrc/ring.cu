@@ -117,7 +117,7 @@ __global__ void lse_merge_kernel(float *o_acc, float *lse_acc, const T *o_part,
 // P partial results of the same rows over disjoint key sets -> the result
 // over all of them: m = max_i lse_i, w_i = e^(lse_i - m),
 // o = sum_i w_i o_i / sum_i w_i, lse = m + log sum_i w_i (all -inf: 0, -inf).
-// One pass over the parts' outputs (parts whose weight is 0 are not read).
+// One pass over the parts' outputs (a part of weight 0 is not added).
 template <typename T>
 __global__ void lse_merge_parts_kernel(const T *parts, const float *lses, int n_parts, T *out,
                                        float *lse_out, long long rows, long long n, int heads) {
@@ -136,7 +136,26 @@ __global__ void lse_merge_parts_kernel(const T *parts, const float *lses, int n_
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float wsum = 0.f;
   if (m != -INFINITY) {
-    for (int k = 0; k < n_parts; ++k) {
+    // four parts at a time, their loads issued together; a part of weight 0
+    // is read but not added (its values may be anything)
+    int k = 0;
+    for (; k + 4 <= n_parts; k += 4) {
+      float w[4], v[4][8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        w[u] = expf(lses[(k + u) * l_stride + li] - m);
+        ld8(parts + (k + u) * o_stride + oi, v[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (w[u] > 0.f) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[u], v[u][e], acc[e]);
+          wsum += w[u];
+        }
+      }
+    }
+    for (; k < n_parts; ++k) {
       const float w = expf(lses[k * l_stride + li] - m);
       if (w > 0.f) {
         float v[8];

@@ -172,3 +172,33 @@ def test_norm_option_errors(api):
     torch.cuda.synchronize()
     with pytest.raises(ValueError):
         api.forward(t, t, t, plan, rope, q_norm=torch.ones(64))  # host tensor
+
+
+def test_norm_full_size_sampled(api):
+    """I2V 480p with RMSNorm weights (the <true> instantiation of the kernel at
+    full size): every row of the sample of parity.sample_rows, heads 0 and 31."""
+    w = synthetic.get("i2v_480p")
+    x = synthetic.make_inputs(w)
+    qn, kn = weights(31), weights(32)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    d = {k: v.cuda() for k, v in x.items()}
+    out, lse = api.forward(d["q"], d["k"], d["v"], plan, rope, return_lse=True,
+                           q_norm=qn.cuda(), k_norm=kn.cuda(), norm_eps=EPS)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    rows = parity.sample_rows(w, n_random_blocks=16)
+    heads = [0, w.heads - 1]
+    sub = {k: v[:, :, heads].contiguous() for k, v in x.items()}
+    trip = np.array([(0, h, r) for h in range(2) for r in rows], dtype=np.int64)
+    ref_o, ref_l = oracle.attention_rows(
+        sub["q"], sub["k"], sub["v"], H=w.H, W=w.W, Nc=w.n_cond_tokens, block=w.block,
+        local=w.local, stride=w.stride, rows=trip, q_norm=qn.double().numpy(),
+        k_norm=kn.double().numpy(), norm_eps=EPS)
+    g = out[0][:, heads].float().cpu().numpy().astype(np.float64)   # [N, 2, 64]
+    g = np.transpose(g[rows], (1, 0, 2)).reshape(-1, 64)
+    err = np.abs(g - ref_o)
+    assert err.max() <= parity.BF16_MAX_ABS and err.mean() <= parity.BF16_MEAN_ABS, \
+        (err.max(), err.mean())
+    gl = lse[0][heads][:, rows].cpu().numpy().astype(np.float64).reshape(-1)
+    assert np.abs(gl - ref_l).max() <= parity.BF16_LSE_ABS

@@ -115,7 +115,8 @@ def backward(q, k, v, dout, *, T: int, H: int, W: int, n_cond: int, block: int =
 
 
 def backward_dq_rows(q, k, v, dout, *, H: int, W: int, Nc: int, block: int, local: int,
-                     stride: int, rows, scale: Optional[float] = None):
+                     stride: int, rows, scale: Optional[float] = None, q_norm=None,
+                     k_norm=None, norm_eps: float = 1e-6):
     """dq of the selected query rows (b, head, n) of the whole-sequence
     forward, row by row: a row's gradient needs only its own keys.  Returns
     [R, hd]."""
@@ -124,25 +125,32 @@ def backward_dq_rows(q, k, v, dout, *, H: int, W: int, Nc: int, block: int, loca
     sc = 1.0 / np.sqrt(hd) if scale is None else scale
     rows = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
     o, lse = attention_rows(qf, kf, vf, H=H, W=W, Nc=Nc, block=block, local=local,
-                            stride=stride, rows=rows, scale=sc)
+                            stride=stride, rows=rows, scale=sc, q_norm=q_norm, k_norm=k_norm,
+                            norm_eps=norm_eps)
+    qnf = rms_norm(qf, q_norm, norm_eps) if q_norm is not None else qf
+    knf = rms_norm(kf, k_norm, norm_eps) if k_norm is not None else kf
     cos, sin = rope_angles(N, H, W, hd)
     out = np.zeros((len(rows), hd))
     krot = {}
     for idx, (b, h, n) in enumerate(rows):
         if (b, h) not in krot:
-            krot[(b, h)] = rope3d_apply(kf[b:b + 1, :, h:h + 1], H, W)[0, :, 0]
+            krot[(b, h)] = rope3d_apply(knf[b:b + 1, :, h:h + 1], H, W)[0, :, 0]
         K = krot[(b, h)]
-        qn = rope3d_apply(qf[b:b + 1, n:n + 1, h:h + 1], H, W, tok_offset=int(n))[0, 0, 0]
+        qn = rope3d_apply(qnf[b:b + 1, n:n + 1, h:h + 1], H, W, tok_offset=int(n))[0, 0, 0]
         keys = np.nonzero(token_mask(N, Nc, block, local, stride, rows=[n])[0])[0]
         p = np.exp(sc * (K[keys] @ qn) - lse[idx])
         dp = vf[b, keys, h] @ gf[b, n, h]
         ds = p * (dp - gf[b, n, h] @ o[idx])
-        out[idx] = rope_transpose((sc * (ds @ K[keys]))[None], cos[n:n + 1], sin[n:n + 1])[0]
+        g = rope_transpose((sc * (ds @ K[keys]))[None], cos[n:n + 1], sin[n:n + 1])[0]
+        if q_norm is not None:
+            g = rms_norm_transpose(qf[b, n, h], g, q_norm, norm_eps)
+        out[idx] = g
     return out
 
 
 def backward_dkdv_keys(q, k, v, dout, *, H: int, W: int, Nc: int, block: int, local: int,
-                       stride: int, b: int, h: int, keys, scale: Optional[float] = None):
+                       stride: int, b: int, h: int, keys, scale: Optional[float] = None,
+                       q_norm=None, k_norm=None, norm_eps: float = 1e-6):
     """dk and dv of the selected key tokens of one (batch, head), gathered over
     every query that attends them (their softmax statistics come from
     attention_rows).  Returns (dk [K, hd], dv [K, hd])."""
@@ -154,9 +162,14 @@ def backward_dkdv_keys(q, k, v, dout, *, H: int, W: int, Nc: int, block: int, lo
     qrows = np.nonzero(att.any(axis=1))[0]
     trip = np.stack([np.full_like(qrows, b), np.full_like(qrows, h), qrows], axis=1)
     o, lse = attention_rows(qf, kf, vf, H=H, W=W, Nc=Nc, block=block, local=local,
-                            stride=stride, rows=trip, scale=sc)
-    Q = rope3d_apply(qf[b:b + 1, :, h:h + 1], H, W)[0, qrows, 0]
-    Kr = rope3d_apply(kf[b:b + 1, :, h:h + 1], H, W)[0, keys, 0]
+                            stride=stride, rows=trip, scale=sc, q_norm=q_norm, k_norm=k_norm,
+                            norm_eps=norm_eps)
+    qnf = rms_norm(qf[b:b + 1, :, h:h + 1], q_norm, norm_eps) if q_norm is not None \
+        else qf[b:b + 1, :, h:h + 1]
+    knf = rms_norm(kf[b:b + 1, :, h:h + 1], k_norm, norm_eps) if k_norm is not None \
+        else kf[b:b + 1, :, h:h + 1]
+    Q = rope3d_apply(qnf, H, W)[0, qrows, 0]
+    Kr = rope3d_apply(knf, H, W)[0, keys, 0]
     G = gf[b, qrows, h]
     A = att[qrows]
     P = np.where(A, np.exp(sc * (Q @ Kr.T) - lse[:, None]), 0.0)  # [Rq, K]
@@ -166,4 +179,6 @@ def backward_dkdv_keys(q, k, v, dout, *, H: int, W: int, Nc: int, block: int, lo
     dS = P * (dP - Dn)
     cos, sin = rope_angles(N, H, W, hd)
     dk = rope_transpose(sc * (dS.T @ Q), cos[keys], sin[keys])
+    if k_norm is not None:
+        dk = rms_norm_transpose(kf[b, keys, h], dk, k_norm, norm_eps)
     return dk, dv

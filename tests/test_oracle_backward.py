@@ -126,3 +126,22 @@ def test_sampled_forms_match_dense():
     gk, gv = ob.backward_dkdv_keys(q, k, v, g, b=0, h=1, keys=keys, **kw)
     np.testing.assert_allclose(gk, dk[0, keys, 1], rtol=0, atol=1e-11)
     np.testing.assert_allclose(gv, dv[0, keys, 1], rtol=0, atol=1e-11)
+
+
+def test_sampled_forms_with_rms_norm_match_dense():
+    c = CASES[1]
+    q, k, v, g = _inputs(c, heads=2, seed=60)
+    rng = np.random.default_rng(61)
+    qn, kn = 1 + 0.3 * rng.standard_normal(64), 1 + 0.3 * rng.standard_normal(64)
+    nkw = dict(q_norm=qn, k_norm=kn, norm_eps=1e-6)
+    dq, dk, dv = ob.backward(q, k, v, g, **c, **nkw)
+    N = q.shape[1]
+    Nc = c["n_cond"] * c["H"] * c["W"]
+    kw = dict(H=c["H"], W=c["W"], Nc=Nc, block=64, local=c["local"], stride=c["stride"])
+    rows = np.array([(0, 0, n) for n in (0, 3, N // 3, N - 1)] + [(0, 1, 7)])
+    got = ob.backward_dq_rows(q, k, v, g, rows=rows, **kw, **nkw)
+    np.testing.assert_allclose(got, dq[0, rows[:, 2], rows[:, 1]], rtol=0, atol=1e-11)
+    keys = np.array([0, 1, 64, N - 1])
+    gk, gv = ob.backward_dkdv_keys(q, k, v, g, b=0, h=1, keys=keys, **kw, **nkw)
+    np.testing.assert_allclose(gk, dk[0, keys, 1], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(gv, dv[0, keys, 1], rtol=0, atol=1e-11)

@@ -163,3 +163,32 @@ def test_backward_argument_errors(api):
     assert lib.lc_bsa_backward(*args, 1, w.heads, 32, 0, 0.0, None, plan.handle, rope.handle,
                                None) == 2  # head_dim 32 unsupported
     torch.cuda.synchronize()
+
+
+def test_backward_full_size_with_rms_norm_sampled(api):
+    """I2V 480p backward with RMSNorm weights (dq and dk through the norm
+    transpose, the finalize pass): dq on sampled rows and dk / dv on two key
+    blocks of head 0, against the oracle."""
+    w = synthetic.get("i2v_480p")
+    x = synthetic.make_inputs(w)
+    dout = synthetic.make_dout(w)
+    g = torch.Generator().manual_seed(78)
+    qn = 1.0 + 0.3 * torch.randn(64, generator=g)
+    kn = 1.0 + 0.3 * torch.randn(64, generator=g)
+    dq, dk, dv = run(api, w, x, dout, qn.cuda(), kn.cuda())
+    Nc, N = w.n_cond_tokens, w.n_tokens
+    kw = dict(H=w.H, W=w.W, Nc=Nc, block=64, local=w.local, stride=w.stride,
+              q_norm=qn.double().numpy(), k_norm=kn.double().numpy(), norm_eps=1e-6)
+    xh = {k: x[k][:, :, 0:1].contiguous() for k in ("q", "k", "v")}
+    gh = dout[:, :, 0:1].contiguous()
+    rng = np.random.default_rng(10)
+    rows_n = np.unique(np.concatenate([[0, Nc - 1, Nc, N - 1], rng.integers(0, N, 24)]))
+    trip = np.stack([np.zeros_like(rows_n), np.zeros_like(rows_n), rows_n], axis=1)
+    ref = ob.backward_dq_rows(xh["q"], xh["k"], xh["v"], gh, rows=trip, **kw)
+    assert_close(w, dq[0, torch.as_tensor(rows_n), 0], ref, "dq rows")
+    for j in (9, 8):
+        keys = np.arange(Nc + 64 * j, Nc + 64 * j + 64)
+        rk, rv = ob.backward_dkdv_keys(xh["q"], xh["k"], xh["v"], gh, b=0, h=0, keys=keys, **kw)
+        kt = torch.as_tensor(keys)
+        assert_close(w, dk[0, kt, 0], rk, "dk block %d" % j)
+        assert_close(w, dv[0, kt, 0], rv, "dv block %d" % j)

@@ -739,10 +739,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           const float mt = row_max(s) + m_use;  // s now holds logits minus m_use
           if (__any_sync(0xffffffffu, mt > m_ref + kRescaleThreshold)) {
             const float m_new = fmaxf(m_ref, mt);
-            alpha = (m_new == -INFINITY) ? 1.f : ex2(m_ref - m_new);
+            const float m_new_use = (m_new == -INFINITY) ? 0.f : m_new;
+            // O and l so far are relative to m_use, which is 0 while the row
+            // has met no attended key in an earlier tile (m_ref = -inf) -- a
+            // group's first tile can be fully masked for some member rows.
+            alpha = ex2(m_use - m_new_use);
             l_sum *= alpha;
             m_ref = m_new;
-            const float m_new_use = (m_ref == -INFINITY) ? 0.f : m_ref;
             ok = pass(1.f, m_use - m_new_use);
             if (!ok) break;
             m_use = m_new_use;

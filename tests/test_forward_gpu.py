@@ -46,6 +46,8 @@ SMALL = {
                                 stride=3, dtype="f32"),
     "stride_past_end": Workload("stride_past_end", T=3, H=8, W=16, n_cond=0, heads=2, local=0,
                                 stride=100, dtype="bf16"),
+    "local1": Workload("local1", T=4, H=12, W=32, n_cond=0, heads=2, local=1, stride=0,
+                       dtype="bf16"),
     "cached_f32": Workload("cached_f32", T=5, H=8, W=20, n_cond=2, heads=2, local=1, stride=3,
                            dtype="f32", cached=True),
 }
@@ -115,11 +117,15 @@ def test_small_all_rows(api, name):
     print("%s max %.3g mean %.3g lse %.3g" % (name, mx, mean, lerr))
 
 
-@pytest.mark.parametrize("name,qscale", [("small_i2v", 4.0), ("ragged", 8.0), ("dense_small", 6.0)])
+@pytest.mark.parametrize("name,qscale", [("small_i2v", 4.0), ("ragged", 8.0), ("dense_small", 6.0),
+                                         ("local_only", 6.0), ("local1", 6.0)])
 def test_large_logits_exercise_rescaling(api, name, qscale):
     """Scaled queries give logits with a wide range, so the running maximum
     moves often and the kernel's rescaling path (new reference max, O and l
-    rescaled, P recomputed) runs on many tiles."""
+    rescaled, P recomputed) runs on many tiles.  With no condition frame and
+    no global blocks (local_only, local1) the first key tile of a 4-block
+    group is fully masked for some member rows, which then meet their first
+    attended key -- and possibly a rescale -- in a later tile."""
     w = SMALL[name]
     inputs = synthetic.make_inputs(w)
     inputs["q"] = (inputs["q"].float() * qscale).to(inputs["q"].dtype)

@@ -319,3 +319,22 @@ def test_ring_full_size_sampled(api):
                                  return_lse=True)
     assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
     assert (lse - full_l).abs().max().item() <= 1e-2
+
+
+def test_ring_720p_equals_single_launch():
+    """720p refine (86,400 tokens, 1,350 blocks, no condition frames) over 8
+    ranks with the planned cuts: the same as the whole-sequence launch up to
+    one more bf16 rounding of the output, every element."""
+    from block_sparse_attention_rope_b200 import api as a
+    w = synthetic.get("refine_720p")
+    x = synthetic.make_inputs(w)
+    plan = a.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rp, ci = plan.csr()
+    shards = ring.planned_shards(rp.tolist(), ci.tolist(), 0, 8, heads=w.heads)
+    rope = a.Rope3D(w.T, w.H, w.W)
+    out, lse = run_ring(a, w, x, shards, rope, "cuda")
+    full_o, full_l = a.forward(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), plan, rope,
+                               return_lse=True)
+    torch.cuda.synchronize()
+    assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
+    assert (lse - full_l).abs().max().item() <= 1e-2

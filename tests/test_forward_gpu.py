@@ -48,6 +48,11 @@ SMALL = {
                                 stride=100, dtype="bf16"),
     "local1": Workload("local1", T=4, H=12, W=32, n_cond=0, heads=2, local=1, stride=0,
                        dtype="bf16"),
+    # the cached form with no condition frames (no cond_k / cond_v at all)
+    "cached_nocond": Workload("cached_nocond", T=3, H=8, W=24, n_cond=0, heads=2, local=1,
+                              stride=2, dtype="bf16", cached=True),
+    "cached_nocond_f32": Workload("cached_nocond_f32", T=3, H=8, W=24, n_cond=0, heads=2,
+                                  local=1, stride=2, dtype="f32", cached=True),
     "cached_f32": Workload("cached_f32", T=5, H=8, W=20, n_cond=2, heads=2, local=1, stride=3,
                            dtype="f32", cached=True),
 }

@@ -207,3 +207,23 @@ def test_backward_reproducibility():
     assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
     d = (g1[0].float() - g2[0].float()).abs().max().item()
     assert d <= 2 ** -7 * g1[0].float().abs().max().item()
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_custom_softmax_scale(dtype):
+    from block_sparse_attention_rope_b200 import api as a
+    w = Workload("sc", T=3, H=8, W=20, n_cond=1, heads=2, local=1, stride=2, dtype=dtype)
+    x = synthetic.make_inputs(w)
+    dout = synthetic.make_dout(w)
+    d = {k: v.cuda() for k, v in x.items()}
+    plan = a.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = a.Rope3D(w.T, w.H, w.W)
+    out, lse = a.forward(d["q"], d["k"], d["v"], plan, rope, return_lse=True, softmax_scale=0.3)
+    grads = a.backward(d["q"], d["k"], d["v"], out, lse, dout.cuda(), plan, rope,
+                       softmax_scale=0.3)
+    torch.cuda.synchronize()
+    assert a.last_device_status() == 0
+    ref = ob.backward(x["q"], x["k"], x["v"], dout, T=w.T, H=w.H, W=w.W, n_cond=w.n_cond,
+                      local=w.local, stride=w.stride, scale=0.3)
+    for got, r, what in zip(grads, ref, ("dq", "dk", "dv")):
+        assert_close(w, got, r, what)

@@ -287,3 +287,34 @@ def test_watchdog_gives_up_and_context_survives(api):
     out, lse = run_gpu(api, w, inputs)
     ref_out, ref_lse = full_oracle(w, inputs)
     check_all_rows(w, out, lse, ref_out, ref_lse)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_custom_softmax_scale(api, dtype):
+    """A softmax scale other than 1/sqrt(64), forward and cached forms."""
+    w = Workload("sc", T=4, H=8, W=24, n_cond=1, heads=2, local=1, stride=2, dtype=dtype)
+    x = synthetic.make_inputs(w)
+    plan = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    d = {k: v.cuda() for k, v in x.items()}
+    out, lse = api.forward(d["q"], d["k"], d["v"], plan, rope, return_lse=True,
+                           softmax_scale=0.3)
+    Nc = w.n_cond_tokens
+    oc, lc = api.forward_cached(d["q"][:, Nc:].contiguous(), d["k"][:, Nc:].contiguous(),
+                                d["v"][:, Nc:].contiguous(), d["k"][:, :Nc].contiguous(),
+                                d["v"][:, :Nc].contiguous(), plan, rope, return_lse=True,
+                                softmax_scale=0.3)
+    torch.cuda.synchronize()
+    assert api.last_device_status() == 0
+    ref_o, ref_l = oracle.forward(x["q"], x["k"], x["v"], T=w.T, H=w.H, W=w.W, n_cond=w.n_cond,
+                                  local=w.local, stride=w.stride, scale=0.3)
+    if dtype == "f32":
+        check_all_rows(w, out.cpu(), lse.cpu(), ref_o, ref_l)
+    else:
+        # logits 2.4x those of the default scale: the bf16 rounding of R(q),
+        # R(k) moves them 2.4x as far (as in the large-logit test)
+        err = np.abs(out.cpu().float().numpy().astype(np.float64) - ref_o)
+        k = 0.3 / 0.125
+        assert err.max() <= parity.BF16_MAX_ABS * k and err.mean() <= parity.BF16_MEAN_ABS * k
+        assert np.abs(lse.cpu().numpy() - ref_l).max() <= parity.BF16_LSE_ABS * k
+    assert torch.equal(oc, out[:, Nc:]) and torch.equal(lc, lse[:, :, Nc:])

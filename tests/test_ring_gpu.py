@@ -338,3 +338,26 @@ def test_ring_720p_equals_single_launch():
     torch.cuda.synchronize()
     assert (out.float() - full_o.float()).abs().max().item() <= 1.6e-2
     assert (lse - full_l).abs().max().item() <= 1e-2
+
+
+def test_forward_shard_custom_scale(api):
+    w = SMALL
+    x = synthetic.make_inputs(w)
+    rope = api.Rope3D(w.T, w.H, w.W)
+    p = api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                 q_blocks=(10, 18), k_blocks=(5, 20))
+    (qa, qb), (ka, kb) = p.q_tokens, p.k_tokens
+    o, l = api.forward_shard(x["q"][:, qa:qb].contiguous().cuda(),
+                             x["k"][:, ka:kb].contiguous().cuda(),
+                             x["v"][:, ka:kb].contiguous().cuda(), p, rope, softmax_scale=0.3)
+    torch.cuda.synchronize()
+    ref_o, ref_l = orng.partial_attention(x["q"][:, qa:qb], x["k"][:, ka:kb], x["v"][:, ka:kb],
+                                          q_tokens=(qa, qb), k_tokens=(ka, kb), scale=0.3,
+                                          **geo(w))
+    # logits 2.4x those of the default scale, so 2.4x the bf16 bounds (as in
+    # the forward's large-logit test)
+    k = 0.3 / 0.125
+    err = np.abs(o.double().cpu().numpy() - ref_o)
+    assert err.max() <= 1.5e-2 * k and err.mean() <= 1e-3 * k
+    fin = np.isfinite(ref_l)
+    assert np.abs(l.double().cpu().numpy()[fin] - ref_l[fin]).max() <= 5e-2 * k

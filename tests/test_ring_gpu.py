@@ -361,3 +361,25 @@ def test_forward_shard_custom_scale(api):
     assert err.max() <= 1.5e-2 * k and err.mean() <= 1e-3 * k
     fin = np.isfinite(ref_l)
     assert np.abs(l.double().cpu().numpy()[fin] - ref_l[fin]).max() <= 5e-2 * k
+
+
+def test_merges_with_fp32_parts(api):
+    """lc_bsa_lse_merge and lc_bsa_lse_merge_parts on fp32 partial outputs."""
+    g = torch.Generator().manual_seed(21)
+    P, B, n, heads = 3, 1, 130, 2
+    parts = torch.randn(P, B, n, heads, 64, generator=g)
+    lses = 2 * torch.randn(P, B, heads, n, generator=g)
+    lses[1, 0, 0, :9] = -float("inf")
+    parts[1, 0, :9, 0] = 0
+    ref_o, ref_l = parts[0].double().numpy(), lses[0].double().numpy()
+    for i in range(1, P):
+        ref_o, ref_l = orng.lse_merge(ref_o, ref_l, parts[i].double().numpy(),
+                                      lses[i].double().numpy())
+    out, lse = api.lse_merge_parts(parts.cuda(), lses.cuda())
+    acc_o, acc_l = parts[0].cuda().clone(), lses[0].cuda().clone()
+    for i in range(1, P):
+        api.lse_merge(acc_o, acc_l, parts[i].cuda(), lses[i].cuda())
+    torch.cuda.synchronize()
+    for o, l in ((out, lse), (acc_o, acc_l)):
+        assert np.abs(o.double().cpu().numpy() - ref_o).max() <= 1e-5 * np.abs(ref_o).max()
+        assert np.abs(l.double().cpu().numpy() - ref_l).max() <= 1e-5 * np.abs(ref_l).max()

@@ -10,6 +10,7 @@
 #include <new>
 
 #include "lc_internal.cuh"
+#include "lc_vec8.cuh"
 #include <cuda_bf16.h>
 
 namespace {
@@ -76,18 +77,14 @@ __global__ void rope_apply_kernel(const Tin *x, Tin *out, long long n_chunks, in
     int h = lc_div(rem, div_w);
     int w = rem - h * div_w.d;
     float v[8];
-    const Tin *src = x + i * 8;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = (float)src[e];
+    lcvec::ld8(x + i * 8, v);  // one 16- / 32-byte load (x is 16-byte aligned)
     if (nw) {  // uniform: every lane of a group is in the loop together
       const float inv = lc_rms_inv(lc_sumsq_lanes8(lc_sumsq8(v), group), eps);
 #pragma unroll
       for (int e = 0; e < 8; ++e) v[e] = lc_rms_apply(v[e], inv, __ldg(nw + 8 * ch + e));
     }
     rotate_chunk(v, ch, t, h, w, tab, T, H, W);
-    Tin *dst = out + i * 8;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = (Tin)v[e];
+    lcvec::st8(out + i * 8, v);
   }
 }
 

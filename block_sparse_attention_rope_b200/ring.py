@@ -207,7 +207,6 @@ class RingSchedule:
         self.computes = [bool(active(rank, src)) for src in self.sources]
         if not any(self.computes):
             raise ValueError("rank %d attends no key shard" % rank)
-        self.last = max(s for s, c in enumerate(self.computes) if c)
 
     def n_tokens(self, shard: int) -> int:
         a, b = self.tokens[shard]

@@ -126,3 +126,26 @@ def test_condition_tokens_never_see_noise_tokens():
                 assert not oracle.token_allowed(n, m, Nc, 64, 2, 4)
             if n >= Nc and m < Nc:
                 assert oracle.token_allowed(n, m, Nc, 64, 0, 0)
+
+
+def test_random_geometries_csr_against_token_mask():
+    """Seeded random small geometries: the brute-force block CSR, the closed
+    row counts and the token-level pair count agree (every attended block pair
+    contributes exactly its two blocks' token counts)."""
+    from oracle.backward import token_mask
+    rng = np.random.default_rng(2024)
+    for _ in range(25):
+        T = int(rng.integers(1, 6))
+        H, W = int(rng.integers(1, 9)), int(rng.integers(1, 40))
+        n_cond = int(rng.integers(0, T))
+        local, stride = int(rng.integers(0, 4)), int(rng.integers(-1, 7))
+        Nc, Nn, Cb, Nb = oracle.segment_sizes(T, H, W, n_cond)
+        N = Nc + Nn
+        rp, ci = oracle.block_csr(T, H, W, 64, local, stride, n_cond)
+        assert rp[-1] == len(ci)
+        for i in range(Nb):
+            assert rp[Cb + i + 1] - rp[Cb + i] == Cb + closed_form_row_count(i, Nb, local, stride)
+        def ntok(b):
+            return min(64, Nc - 64 * b) if b < Cb else min(64, Nn - 64 * (b - Cb))
+        pairs = sum(ntok(r) * ntok(int(c)) for r in range(Cb + Nb) for c in ci[rp[r]:rp[r + 1]])
+        assert pairs == int(token_mask(N, Nc, 64, local, stride).sum())

@@ -205,3 +205,30 @@ def test_planned_shards_model():
     t18 = ring.modeled_rank_cycles(lay18, rp, ci, 25, 32)[1]
     t19 = ring.modeled_rank_cycles(lay19, rp, ci, 25, 32)[1]
     assert t19 > t18 * 1.1
+
+
+def test_shard_layouts_on_random_geometries():
+    """Seeded random geometries and rank counts: the even-work and the planned
+    layouts both cover the blocks with contiguous ranges on group edges, and
+    the planned one is never worse under the model."""
+    rng = np.random.default_rng(7)
+    for _ in range(12):
+        T = int(rng.integers(2, 6))
+        H, W = int(rng.integers(4, 12)), int(rng.integers(16, 48))
+        n_cond = int(rng.integers(0, T - 1))
+        local, stride = int(rng.integers(0, 3)), int(rng.integers(0, 6))
+        Nc, Nn, Cb, Nb = oracle.segment_sizes(T, H, W, n_cond)
+        rp, ci = oracle.block_csr(T, H, W, 64, local, stride, n_cond)
+        edges = ring.group_edges(Cb, Nb)
+        for world in (1, 2, 3):
+            if len(edges) - 1 < world:
+                continue
+            even = ring.balanced_shards(ring.block_work(np.diff(rp), Cb), Cb, world)
+            plan = ring.planned_shards(rp, ci, Cb, world, heads=4, n_sm=8)
+            for sh in (even, plan):
+                assert sh[0][0] == 0 and sh[-1][1] == Cb + Nb and len(sh) == world
+                assert all(a < b and a in edges and b in edges for a, b in sh)
+                assert all(sh[i][1] == sh[i + 1][0] for i in range(world - 1))
+            te = ring.modeled_rank_cycles(even, rp, ci, Cb, 4, n_sm=8)
+            tp = ring.modeled_rank_cycles(plan, rp, ci, Cb, 4, n_sm=8)
+            assert max(tp) <= max(te) + 1e-6

@@ -2,7 +2,7 @@
 """Benchmark of block-sparse 3D-RoPE attention (one attention layer per step).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload i2v_480p] [--sweep] [--no-cpu-baseline]
+                    [--workload i2v_480p] [--no-extra] [--no-cpu-baseline]
 
 One step = one lc_bsa_forward call over one layer: B=1 per GPU, 32 heads x 64,
 the 480x832 93-frame image-to-video latent (24x30x52 = 37,440 tokens, first
@@ -46,8 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="i2v_480p")
-    ap.add_argument("--sweep", action="store_true", help="also time the sparsity sweep")
-    ap.add_argument("--no-extra", action="store_true", help="skip the 86,400-token line")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (skip the other workloads, backward and ring)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--backward-only", action="store_true",
@@ -480,6 +480,17 @@ def exp_roofline(res, clocks):
                     % res["scores"]}
 
 
+def workload_config(w, world: int) -> dict:
+    """The `config` object of a bench line (both arms name the workload the
+    same way)."""
+    return {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "n_cond_frames": w.n_cond,
+            "tokens": w.n_tokens, "heads": w.heads, "head_dim": w.head_dim, "block": w.block,
+            "local": w.local, "stride": w.stride, "batch_per_gpu": w.batch,
+            "global_batch": w.batch * world,
+            "parallelism": "replicas: one batch element per GPU, no data-path collective",
+            "l2": "inputs larger than L2 (q, k, v 153 MB each); no flush"}
+
+
 def run_ours(a):
     import torch
     world, rank, local = dist_env()
@@ -519,10 +530,11 @@ def run_ours(a):
                           "ms_per_step": round(serial_ms, 3),
                           "path": "copy in, forward, copy out one after another"}}
     extra = {}
-    names = [] if a.no_extra else ["refine_720p"]
-    if a.sweep:
-        names += ["continuation_cached"] + ["sweep_" + s for s in
-                                            ("dense", "l2s4", "l2s8", "l1s16", "l1s32")]
+    # every other named workload: the 86,400-token refine pass, the cached
+    # continuation and the five masks of the sparsity sweep at 37,440 tokens
+    names = [] if a.no_extra else (["refine_720p", "continuation_cached"] +
+                                   ["sweep_" + s for s in
+                                    ("dense", "l2s4", "l2s8", "l1s16", "l1s32")])
     for n in names:
         if n == a.workload:
             continue
@@ -549,12 +561,7 @@ def run_ours(a):
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) q/k/v, bf16)",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "n_cond_frames": w.n_cond,
-                   "tokens": w.n_tokens, "heads": w.heads, "head_dim": w.head_dim, "block": w.block,
-                   "local": w.local, "stride": w.stride, "batch_per_gpu": w.batch,
-                   "global_batch": w.batch * world,
-                   "parallelism": "replicas: one batch element per GPU, no data-path collective",
-                   "l2": "inputs larger than L2 (q, k, v 153 MB each); no flush"},
+        "config": workload_config(w, world),
         "pct_bf16_peak": round(100.0 * achieved / peak, 2),
         "launch_ms_min_median_max": main["spread"],
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
@@ -605,9 +612,7 @@ def run_reference(a):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) q/k/v, bf16 values upcast to f64)",
             "impl": "reference",
-            "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W,
-                       "n_cond_frames": w.n_cond, "tokens": w.n_tokens, "heads": w.heads,
-                       "head_dim": w.head_dim, "local": w.local, "stride": w.stride},
+            "config": workload_config(w, world),
             "cpu_baseline": {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tf, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -76,7 +76,9 @@ def _load():
         "lc_bsa_lse_merge_parts": (S, [vp, vp, I, vp, vp, I, LL, I, I, I, vp]),
         "lc_rope3d_apply_ex": (S, [vp, vp, I, LL, I, I, LL, I, vp, F, vp, vp]),
         "lc_last_device_status": (S, [vp]),
+        "lc_device_status_decode": (S, [I]),
         "lc_debug_watchdog_selftest": (S, [I, vp]),
+        "lc_debug_scratch_pool_used_high": (S, [ctypes.POINTER(ctypes.c_ulonglong), I]),
         "lc_status_string": (ctypes.c_char_p, [S]),
         "lc_version": (ctypes.c_char_p, []),
     }
@@ -515,3 +517,12 @@ def last_device_status(stream=None) -> int:
 
 def watchdog_selftest(timeout_us: int = 20000, stream=None) -> int:
     return int(lib.lc_debug_watchdog_selftest(int(timeout_us), _stream(stream)))
+
+
+def scratch_pool_used_high(reset: bool = False) -> int:
+    """High-water mark (bytes) of the library's scratch pool on the current
+    device; with reset, the mark is first reset to the bytes in use now."""
+    v = ctypes.c_ulonglong(0)
+    _check(lib.lc_debug_scratch_pool_used_high(ctypes.byref(v), 1 if reset else 0),
+           "lc_debug_scratch_pool_used_high")
+    return int(v.value)

@@ -343,16 +343,22 @@ extern "C" lc_status lc_last_device_status(void *stream) {
   lc_status s;
   int *p = lc_device_status_ptr(&s);
   if (s != LC_OK) return s;
-  int *na = lc_noalloc_scratch(&s);
-  if (s != LC_OK) return s;
+  // The allocation-free entry point's status word is read only on a device
+  // where that entry point has run (its address was looked up then).
+  int *na = lc_noalloc_scratch_if_ready();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   LC_CUDA_TRY(cudaStreamSynchronize(st));
   int word = 0, word_na = 0;
   LC_CUDA_TRY(cudaMemcpy(&word, p, sizeof(int), cudaMemcpyDeviceToHost));
-  LC_CUDA_TRY(cudaMemcpy(&word_na, na + 1, sizeof(int), cudaMemcpyDeviceToHost));
   LC_CUDA_TRY(cudaMemset(p, 0, sizeof(int)));
-  LC_CUDA_TRY(cudaMemset(na + 1, 0, sizeof(int)));
-  word |= word_na;
+  if (na) {
+    LC_CUDA_TRY(cudaMemcpy(&word_na, na + 1, sizeof(int), cudaMemcpyDeviceToHost));
+    LC_CUDA_TRY(cudaMemset(na + 1, 0, sizeof(int)));
+  }
+  return lc_device_status_decode(word | word_na);
+}
+
+extern "C" lc_status lc_device_status_decode(int word) {
   if (word & LC_DEVSTAT_TIMEOUT) return LC_ERR_TIMEOUT;
   if (word & LC_DEVSTAT_CHECK) return LC_ERR_DEVICE_CHECK;
   return LC_OK;
@@ -369,6 +375,21 @@ extern "C" lc_status lc_debug_watchdog_selftest(int timeout_us, void *stream) {
   s = lc_launch_watchdog_selftest(p, (long long)timeout_us * 1000LL, st);
   if (s != LC_OK) return s;
   return lc_last_device_status(stream);
+}
+
+extern "C" lc_status lc_debug_scratch_pool_used_high(unsigned long long *bytes, int reset) {
+  if (!bytes) return LC_ERR_INVALID_ARGUMENT;
+  lc_status s;
+  cudaMemPool_t pool = lc_scratch_pool(&s);
+  if (s != LC_OK) return s;
+  if (reset) {
+    uint64_t zero = 0;  // resets the mark to the bytes in use now
+    LC_CUDA_TRY(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero));
+  }
+  uint64_t v = 0;
+  LC_CUDA_TRY(cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &v));
+  *bytes = (unsigned long long)v;
+  return LC_OK;
 }
 
 extern "C" const char *lc_status_string(lc_status s) {

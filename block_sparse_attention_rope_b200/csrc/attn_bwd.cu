@@ -38,6 +38,9 @@ struct BwdArgs {
   float *delta;  // [B, heads, N] scratch
   void *dq, *dk, *dv;
   const int *row_ptr, *col_idx, *col_ptr, *row_idx;
+  int *status;     // device status word (plan checks)
+  long long nnz;   // CSR / CSC entries
+  int n_blocks;    // blocks of the pattern
   const float *tab;
   const float *q_nw, *k_nw;
   float norm_eps, scale;
@@ -215,7 +218,10 @@ __global__ void __launch_bounds__(64) bwd_dq_kernel(BwdArgs a) {
   for (int d = 0; d < LC_HEAD_DIM; ++d) dq[d] = 0.f;
   const Tin *K = static_cast<const Tin *>(a.k);
   const Tin *V = static_cast<const Tin *>(a.v);
-  for (int e = a.row_ptr[r]; e < a.row_ptr[r + 1]; ++e) {
+  int e_lo, e_hi;
+  lc_checked_row(a.row_ptr, r, a.nnz, a.status, e_lo, e_hi);
+  for (int e = e_lo; e < e_hi; ++e) {
+    if (!lc_checked_block(a.col_idx[e], a.n_blocks, a.status)) continue;
     int k_lo, k_hi;
     block_range(a, a.col_idx[e], k_lo, k_hi);
     const int kn = k_hi - k_lo;
@@ -284,7 +290,10 @@ __global__ void __launch_bounds__(64) bwd_dkdv_kernel(BwdArgs a) {
   for (int d = 0; d < LC_HEAD_DIM; ++d) dk[d] = dv[d] = 0.f;
   const Tin *Q = static_cast<const Tin *>(a.q);
   const Tin *G = static_cast<const Tin *>(a.dout);
-  for (int e = a.col_ptr[c]; e < a.col_ptr[c + 1]; ++e) {
+  int e_lo, e_hi;
+  lc_checked_row(a.col_ptr, c, a.nnz, a.status, e_lo, e_hi);
+  for (int e = e_lo; e < e_hi; ++e) {
+    if (!lc_checked_block(a.row_idx[e], a.n_blocks, a.status)) continue;
     int q_lo, q_hi;
     block_range(a, a.row_idx[e], q_lo, q_hi);
     const int qn = q_hi - q_lo;
@@ -439,6 +448,8 @@ lc_status lc_launch_backward(const void *q, const void *k, const void *v, const 
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.row_ptr = plan->row_ptr; a.col_idx = plan->col_idx;
   a.col_ptr = plan->col_ptr; a.row_idx = plan->row_idx;
+  a.nnz = plan->nnz;
+  a.n_blocks = plan->Cb + plan->Nb;
   a.tab = rope->tab;
   a.q_nw = norm.q_w; a.k_nw = norm.k_w; a.norm_eps = norm.eps;
   a.scale = scale;
@@ -448,6 +459,8 @@ lc_status lc_launch_backward(const void *q, const void *k, const void *v, const 
   a.Nc = plan->Nc; a.Nn = plan->Nn; a.Cb = plan->Cb; a.heads = heads;
   if (plan->nq == 0) return LC_OK;
   lc_status s = LC_OK;
+  a.status = lc_device_status_ptr(&s);
+  if (s != LC_OK) return s;
   cudaMemPool_t pool = lc_scratch_pool(&s);
   if (s != LC_OK) return s;
   const size_t dbytes = sizeof(float) * (size_t)batch * heads * (plan->Nc + plan->Nn);

@@ -98,6 +98,8 @@ struct __align__(64) BwdParams {
   lc_divmod div_hw, div_w;
   int T, H, W;
   int Nc, Nn, Cb, kgc, heads, KG, total_items, tab_floats;
+  int n_blocks;   // query / key blocks of the pattern (valid block ids: [0, n_blocks))
+  int ent_cap;    // entries kg_ent holds (valid list bounds: [0, ent_cap])
   float scale;
 };
 
@@ -148,24 +150,52 @@ struct KItem {
   const uint32_t *ent;
 };
 
-__device__ __forceinline__ KItem decode_kitem(const BwdParams &p, int item) {
+// Device-side plan checks: a key group id, key block, list bound or query
+// entry that a consistent plan never holds is replaced by a harmless one (a
+// group with no valid key row, so nothing is stored; a one-entry list; an
+// absent query block that loads as zeros, is masked and adds nothing to dq)
+// before it is used as an index, a TMA coordinate or a store address, and
+// LC_DEVSTAT_CHECK is raised by the role passed `status` (the producer).
+__device__ __forceinline__ KItem decode_kitem(const BwdParams &p, int item, int *status) {
   KItem it;
   const int per = p.KG;
   const int bh = item / per;
-  const int g = p.kg_order[item - bh * per];
+  int g = p.kg_order[item - bh * per];
+  bool bad = (unsigned)g >= (unsigned)p.KG;
+  if (bad) g = 0;
   it.b = bh / p.heads;
   it.h = bh - it.b * p.heads;
   it.seg = g < p.kgc ? 0 : 1;
-  const int2 kb = p.kg_blk[g];  // global key block ids
+  int2 kb = p.kg_blk[g];  // global key block ids
   const int base = it.seg ? p.Cb : 0;
+  const int nseg = it.seg ? p.n_blocks - p.Cb : p.Cb;  // key blocks of the segment
   it.seg_len = it.seg ? p.Nn : p.Nc;
-  it.cnt = kb.y >= 0 ? 2 : 1;
-  it.krow0 = 64 * (kb.x - base);
-  it.krow1 = kb.y >= 0 ? 64 * (kb.y - base) : it.seg_len;
-  const int lo = p.kg_ptr[g];
-  it.len = p.kg_ptr[g + 1] - lo;
+  const bool x_ok = (unsigned)(kb.x - base) < (unsigned)nseg;
+  const bool y_ok = kb.y < 0 || (unsigned)(kb.y - base) < (unsigned)nseg;
+  if (!x_ok || !y_ok) {
+    bad = true;
+    it.cnt = 0;  // no key row of the item is valid: nothing is loaded or stored
+    it.krow0 = it.krow1 = it.seg_len;
+  } else {
+    it.cnt = kb.y >= 0 ? 2 : 1;
+    it.krow0 = 64 * (kb.x - base);
+    it.krow1 = kb.y >= 0 ? 64 * (kb.y - base) : it.seg_len;
+  }
+  int lo = p.kg_ptr[g], hi = p.kg_ptr[g + 1];
+  if (lo < 0 || hi <= lo || hi > p.ent_cap) {
+    bad = true;
+    lo = 0;
+    hi = 1;
+  }
+  it.len = hi - lo;
   it.ent = p.kg_ent + lo;
+  if (bad && status) atomicOr(status, LC_DEVSTAT_CHECK);
   return it;
+}
+
+// A list entry names a query block of the pattern and at least one member.
+__device__ __forceinline__ bool qentry_ok(const BwdParams &p, uint32_t e) {
+  return (int)(e & 0xFFFFFFu) < p.n_blocks && ((e >> 24) - 1u) < 3u;
 }
 
 // Query block of a list entry -> segment, first row in the segment, tokens.
@@ -304,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         misc[1 + slot] = (uint32_t)item;
         lcptx::mbar_arrive(ctx.bar(B_SCHED_FULL + slot));
         if (item < 0) break;
-        const KItem it = decode_kitem(p, item);
+        const KItem it = decode_kitem(p, item, p.status);
         const uint32_t kph = item_it & 1;
         bool ok = wait_bar(ctx, ctx.bar(B_KV_EMPTY), kph ^ 1);
         if (!ok) break;
@@ -327,13 +357,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t ph = (q_it / kQStages) & 1;
           ok = wait_bar(ctx, ctx.bar(B_QG_EMPTY + s), ph ^ 1);
           if (!ok) break;
-          int sa, ra, na, sb, rb, nb;
-          qblock(p, __ldg(it.ent + 2 * t), sa, ra, na);
+          // no second query block, or an entry that fails the plan check: a
+          // box past the noisy segment's end reads zeros
+          int sa = 1, ra = p.Nn, na, sb = 1, rb = p.Nn, nb;
+          const uint32_t ea = __ldg(it.ent + 2 * t);
+          if (qentry_ok(p, ea)) qblock(p, ea, sa, ra, na);
+          else atomicOr(p.status, LC_DEVSTAT_CHECK);
           if (2 * t + 1 < it.len) {
-            qblock(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
-          } else {  // no second query block: a box past the noisy segment's end reads zeros
-            sb = 1;
-            rb = p.Nn;
+            const uint32_t eb = __ldg(it.ent + 2 * t + 1);
+            if (qentry_ok(p, eb)) qblock(p, eb, sb, rb, nb);
+            else atomicOr(p.status, LC_DEVSTAT_CHECK);
           }
           const uint32_t bar = ctx.bar(B_QG_FULL + s);
           lcptx::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
@@ -403,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         const int item = (int)misc[1 + slot];
         lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
         if (item < 0) break;
-        const KItem it = decode_kitem(p, item);
+        const KItem it = decode_kitem(p, item, nullptr);
         bool ok = wait_bar(ctx, ctx.bar(B_KV_FULL), item_it & 1);
         const int nsteps = (it.len + 1) >> 1;
         if (ok) ok = issue_sdp(q_it % kQStages, (q_it / kQStages) & 1, k_step > 0);
@@ -468,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
-      const KItem it = decode_kitem(p, item);
+      const KItem it = decode_kitem(p, item, nullptr);
       bool ok = true;
       const int nsteps = (it.len + 1) >> 1;
       const float *lse_bh = p.lse + ((long long)it.b * p.heads + it.h) * N;
@@ -482,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         for (int i = 0; i < 2; ++i) {
           l2r[i] = dlr[i] = 0.f;
           const int e = 2 * t + i;
-          if (e < it.len) {
+          if (e < it.len && qentry_ok(p, __ldg(it.ent + e))) {
             int qs, qr, qn;
             qblock(p, __ldg(it.ent + e), qs, qr, qn);
             if (rt < qn) {
@@ -526,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
-      const KItem it = decode_kitem(p, item);
+      const KItem it = decode_kitem(p, item, nullptr);
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
       for (int t = 0; t < nsteps; ++t, ++dq_step) {
@@ -561,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
               const int e = 2 * t + blk;
-              if (e >= it.len) continue;
+              if (e >= it.len || !qentry_ok(p, __ldg(it.ent + e))) continue;
               int qs, qr, qn;
               qblock(p, __ldg(it.ent + e), qs, qr, qn);
               const int tok0 = (qs ? p.Nc : 0) + qr;
@@ -603,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
-      const KItem it = decode_kitem(p, item);
+      const KItem it = decode_kitem(p, item, nullptr);
       const bool key_valid = (kr >> 6) < it.cnt && it.krow(kr >> 6) + (kr & 63) < it.seg_len;
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
@@ -614,7 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         const int e = 2 * t + half;
         if (key_valid && e < it.len) {
           const uint32_t ent = __ldg(it.ent + e);
-          if ((ent >> (24 + (kr >> 6))) & 1u) {
+          if (qentry_ok(p, ent) && ((ent >> (24 + (kr >> 6))) & 1u)) {
             int qs, qr, qn;
             qblock(p, ent, qs, qr, qn);
             lim = qn;
@@ -852,6 +885,8 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
     prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.kgc = plan->kgc;
     prm.heads = heads;
     prm.KG = plan->KG;
+    prm.n_blocks = plan->Cb + plan->Nb;
+    prm.ent_cap = (int)plan->nnz;
     prm.total_items = (int)total;
     prm.tab_floats = (int)rope->n_floats;
     prm.scale = scale;

@@ -16,6 +16,9 @@ struct F32Args {
   const float *q, *k, *v, *cond_k, *cond_v;
   float *out, *lse;
   const int *row_ptr, *col_idx;
+  int *status;     // device status word (plan checks)
+  long long nnz;   // CSR entries
+  int n_blocks;    // blocks of the pattern
   const float *tab;
   int T, H, W;
   lc_divmod div_hw, div_w;
@@ -99,8 +102,11 @@ __global__ void __launch_bounds__(64) attn_f32_kernel(F32Args a) {
   }
   float m_run = -INFINITY, l_run = 0.f;
 
-  for (int e = a.row_ptr[r]; e < a.row_ptr[r + 1]; ++e) {
+  int e_lo, e_hi;
+  lc_checked_row(a.row_ptr, r, a.nnz, a.status, e_lo, e_hi);
+  for (int e = e_lo; e < e_hi; ++e) {
     const int c = a.col_idx[e];
+    if (!lc_checked_block(c, a.n_blocks, a.status)) continue;
     int k_lo, k_hi;
     if (c < a.Cb) { k_lo = 64 * c; k_hi = min(a.Nc, k_lo + 64); }
     else { k_lo = a.Nc + 64 * (c - a.Cb); k_hi = min(a.Nc + a.Nn, k_lo + 64); }
@@ -154,11 +160,14 @@ lc_status lc_launch_forward_f32(const float *q, const float *k, const float *v,
                                 int batch, int heads, float scale, lc_fwd_mode mode,
                                 bool cond_k_rotated, const lc_qk_norm &norm,
                                 const lc_bsa_plan_s *plan, const lc_rope3d_s *rope,
-                                int * /*dev_status*/, cudaStream_t stream) {
+                                int *dev_status, cudaStream_t stream) {
   F32Args a;
   a.q = q; a.k = k; a.v = v; a.cond_k = cond_k; a.cond_v = cond_v;
   a.out = out; a.lse = lse;
   a.row_ptr = plan->row_ptr; a.col_idx = plan->col_idx;
+  a.status = dev_status;
+  a.nnz = plan->nnz;
+  a.n_blocks = plan->Cb + plan->Nb;
   a.tab = rope->tab;
   a.T = rope->T; a.H = rope->H; a.W = rope->W;
   a.div_hw = lc_make_divmod(rope->H * rope->W);

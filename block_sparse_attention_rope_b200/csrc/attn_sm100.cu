@@ -117,6 +117,9 @@ struct __align__(64) Sm100Params {
   int T, H, W;
   int Nc, Nn, Cb, gc;
   int heads, n_groups_active, total_items;
+  int n_groups;            // groups of the plan (valid group ids: [0, n_groups))
+  int n_blocks;            // key blocks of the pattern (valid key block ids: [0, n_blocks))
+  int ent_cap;             // entries grp_ent holds (valid list bounds: [0, ent_cap])
   int group_offset;        // first rank of grp_order this launch works on
   int lse_nq;              // rows of the lse tensor per (batch, head)
   int lse_base[2];         // lse row of segment row 0, per segment ([0] condition, [1] noisy)
@@ -175,21 +178,40 @@ struct Item {
   const uint32_t *ent;
 };
 
-__device__ __forceinline__ Item decode_item(const Sm100Params &p, int item) {
+// Device-side plan checks: a group id, list bound or entry that a consistent
+// plan never holds is replaced by a harmless one (group 0, a one-entry list,
+// an absent key block that loads as zeros and is fully masked) before it is
+// used as an index or a TMA coordinate, and LC_DEVSTAT_CHECK is raised by the
+// role passed `status` (the producer), so that every role of the CTA takes
+// the same decision and the host learns of it from lc_last_device_status.
+__device__ __forceinline__ Item decode_item(const Sm100Params &p, int item, int *status) {
   Item it;
   int per = p.n_groups_active;
   int bh = item / per;
   int g = p.grp_order[p.group_offset + item - bh * per];
+  bool bad = (unsigned)g >= (unsigned)p.n_groups;
+  if (bad) g = 0;
   it.b = bh / p.heads;
   it.h = bh - it.b * p.heads;
   it.seg = g < p.gc ? 0 : 1;
   int qb0 = it.seg ? 4 * (g - p.gc) : 4 * g;
   it.row0 = 64 * qb0;
   it.seg_len = it.seg ? p.Nn : p.Nc;
-  int lo = p.grp_ptr[g];
-  it.len = p.grp_ptr[g + 1] - lo;
+  int lo = p.grp_ptr[g], hi = p.grp_ptr[g + 1];
+  if (lo < 0 || hi <= lo || hi > p.ent_cap) {
+    bad = true;
+    lo = 0;
+    hi = 1;
+  }
+  it.len = hi - lo;
   it.ent = p.grp_ent + lo;
+  if (bad && status) atomicOr(status, LC_DEVSTAT_CHECK);
   return it;
+}
+
+// A plan entry names a key block of the pattern and at least one member.
+__device__ __forceinline__ bool entry_ok(const Sm100Params &p, uint32_t e) {
+  return (int)(e & 0xFFFFFFu) < p.n_blocks && ((e >> 24) - 1u) < 15u;
 }
 
 // Key block `e` (plan entry) -> segment, first token in the segment, token count.
@@ -277,13 +299,17 @@ __device__ __forceinline__ uint32_t tile_limits(const Sm100Params &p, const Item
                                                 int qsub) {
   if (2 * tt >= it.len) return 0u;
   const uint32_t ea = __ldg(it.ent + 2 * tt);
-  int sx, rx, na, nb = 0;
-  entry_block(p, ea, sx, rx, na);
-  if (!((ea >> (24 + qsub)) & 1u)) na = 0;
+  int sx, rx, na = 0, nb = 0;
+  if (entry_ok(p, ea)) {
+    entry_block(p, ea, sx, rx, na);
+    if (!((ea >> (24 + qsub)) & 1u)) na = 0;
+  }
   if (2 * tt + 1 < it.len) {
     const uint32_t eb = __ldg(it.ent + 2 * tt + 1);
-    entry_block(p, eb, sx, rx, nb);
-    if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
+    if (entry_ok(p, eb)) {
+      entry_block(p, eb, sx, rx, nb);
+      if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
+    }
   }
   return (uint32_t)na | ((uint32_t)nb << 8);
 }
@@ -379,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         misc[1 + slot] = (uint32_t)item;
         lcptx::mbar_arrive(ctx.bar(B_SCHED_FULL + slot));
         if (item < 0) break;
-        const Item it = decode_item(p, item);
+        const Item it = decode_item(p, item, p.status);
         const int buf = item_it & 1;
         const uint32_t qph = (item_it >> 1) & 1;
         bool ok = true;
@@ -401,15 +427,24 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         for (int t = 0; t < ntiles && ok; ++t, ++kv_it) {
           const int s = kv_it % kStages;
           const uint32_t ph = (kv_it / kStages) & 1;
-          int sa, ra, na, sb, rb, nb;
-          entry_block(p, __ldg(it.ent + 2 * t), sa, ra, na);
-          ra -= p.k_row_off[sa];
+          // a missing second block, or an entry that fails the plan check, is a
+          // box far past every map's end: it reads zeros (and is masked)
+          int sa = 1, ra = 1 << 24, na, sb = 1, rb = 1 << 24, nb;
+          const uint32_t ea = __ldg(it.ent + 2 * t);
+          if (entry_ok(p, ea)) {
+            entry_block(p, ea, sa, ra, na);
+            ra -= p.k_row_off[sa];
+          } else {
+            atomicOr(p.status, LC_DEVSTAT_CHECK);
+          }
           if (2 * t + 1 < it.len) {
-            entry_block(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
-            rb -= p.k_row_off[sb];
-          } else {  // no second block: a box far past every map's end reads zeros
-            sb = 1;
-            rb = 1 << 24;
+            const uint32_t eb = __ldg(it.ent + 2 * t + 1);
+            if (entry_ok(p, eb)) {
+              entry_block(p, eb, sb, rb, nb);
+              rb -= p.k_row_off[sb];
+            } else {
+              atomicOr(p.status, LC_DEVSTAT_CHECK);
+            }
           }
           ok = wait_bar(ctx, ctx.bar(B_KEMPTY + s), ph ^ 1);
           if (!ok) break;
@@ -478,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         const int item = (int)misc[1 + slot];
         lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
         if (item < 0) break;
-        const Item it = decode_item(p, item);
+        const Item it = decode_item(p, item, nullptr);
         const int ntiles = (it.len + 1) >> 1;
         const int buf = item_it & 1;
         const uint32_t qph = (item_it >> 1) & 1;
@@ -562,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
-      const Item it = decode_item(p, item);
+      const Item it = decode_item(p, item, nullptr);
       const int seg_base = it.seg ? p.Nc : 0;  // sequence index of the segment's token 0
       const int buf = item_it & 1;
       const uint32_t qph = (item_it >> 1) & 1;
@@ -594,8 +629,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
 #pragma unroll 1
           for (int half = 0; half < 2; ++half) {
             if (half == 1 && 2 * t + 1 >= it.len) break;
+            const uint32_t ex = half ? eb : ea;
+            if (!entry_ok(p, ex)) continue;
             int sx, rx, nx;
-            entry_block(p, half ? eb : ea, sx, rx, nx);
+            entry_block(p, ex, sx, rx, nx);
             if (rt < nx) rope_row(tile, 64 * half + rt, (sx ? p.Nc : 0) + rx + rt, tab, p, k_nw);
           }
           lcptx::fence_proxy_async_smem();
@@ -625,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       __syncwarp();
       if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SCHED_EMPTY + slot));
       if (item < 0) break;
-      const Item it = decode_item(p, item);
+      const Item it = decode_item(p, item, nullptr);
       const int ntiles = (it.len + 1) >> 1;
       // Mask limits of this warp's rows, one tile per lane, 32 tiles at a time.
       uint32_t lim_lane = 0;
@@ -1015,6 +1052,13 @@ int *lc_noalloc_scratch(lc_status *st) {
   return g_noalloc_ptr[dev];
 }
 
+int *lc_noalloc_scratch_if_ready() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  return g_noalloc_ptr[dev];
+}
+
 lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, const void *cond_k,
                                   const void *cond_v, void *out, float *lse, int batch, int heads,
                                   float scale, lc_fwd_mode mode, bool cond_k_rotated,
@@ -1127,6 +1171,9 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
   prm.T = rope->T; prm.H = rope->H; prm.W = rope->W;
   prm.Nc = (int)Nc; prm.Nn = (int)Nn; prm.Cb = plan->Cb; prm.gc = plan->gc;
   prm.heads = heads;
+  prm.n_groups = plan->G;
+  prm.n_blocks = plan->Cb + plan->Nb;
+  prm.ent_cap = (int)plan->nnz;
   prm.k_prerotated = 0;
   prm.q_norm_w = norm.q_w;
   prm.k_norm_w = norm.k_w;

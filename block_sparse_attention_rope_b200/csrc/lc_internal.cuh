@@ -11,6 +11,28 @@
 #define LC_DEVSTAT_TIMEOUT 0x1
 #define LC_DEVSTAT_CHECK 0x2
 
+#ifdef __CUDACC__
+// One row [lo, hi) of a plan's CSR (or CSC) lists with its bounds checked: a
+// row that a consistent plan never holds (negative, reversed, or past the
+// nnz entries) is walked as an empty row and LC_DEVSTAT_CHECK is raised.
+__device__ __forceinline__ void lc_checked_row(const int *ptr, int r, long long nnz, int *status,
+                                               int &lo, int &hi) {
+  lo = ptr[r];
+  hi = ptr[r + 1];
+  if (lo < 0 || hi < lo || (long long)hi > nnz) {
+    if (status && threadIdx.x == 0) atomicOr(status, LC_DEVSTAT_CHECK);
+    lo = hi = 0;
+  }
+}
+// A block id of a list entry, checked against the pattern's block count; the
+// caller skips the entry when this returns false (LC_DEVSTAT_CHECK raised).
+__device__ __forceinline__ bool lc_checked_block(int c, int n_blocks, int *status) {
+  if ((unsigned)c < (unsigned)n_blocks) return true;
+  if (status && threadIdx.x == 0) atomicOr(status, LC_DEVSTAT_CHECK);
+  return false;
+}
+#endif
+
 // Tokens of one block, head dimension and RoPE split supported by v1.
 #define LC_BLOCK 64
 #define LC_HEAD_DIM 64
@@ -249,4 +271,7 @@ lc_status lc_rotate_rows(const void *x, void *out, int batch, long long ntok, in
 // g_lc_noalloc_scratch on the current device, looked up once per device.
 #define LC_NOALLOC_SCRATCH_INTS 64
 int *lc_noalloc_scratch(lc_status *st);
+// The same address if it has been looked up on the current device already,
+// else NULL (no lookup, no CUDA call beyond cudaGetDevice).
+int *lc_noalloc_scratch_if_ready();
 lc_status lc_launch_watchdog_selftest(int *dev_status, long long timeout_ns, cudaStream_t stream);

@@ -203,7 +203,9 @@ lc_status lc_launch_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
   const long long rows = (long long)batch * n * heads;
   if (rows == 0) return LC_OK;
   const long long threads = rows * 8;
-  const unsigned grid = (unsigned)((threads + 255) / 256);
+  const long long blocks = (threads + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return LC_ERR_UNSUPPORTED;  // past the grid's x limit
+  const unsigned grid = (unsigned)blocks;
   if (dtype == LC_DTYPE_F32)
     lse_merge_kernel<float><<<grid, 256, 0, stream>>>(o_acc, lse_acc,
                                                       static_cast<const float *>(o_part), lse_part,
@@ -222,7 +224,9 @@ lc_status lc_launch_lse_merge_parts(const void *parts, const float *lses, int n_
                                     lc_dtype dtype, cudaStream_t stream) {
   const long long rows = (long long)batch * n * heads;
   if (rows == 0) return LC_OK;
-  const unsigned grid = (unsigned)((rows * 8 + 255) / 256);
+  const long long blocks = (rows * 8 + 255) / 256;
+  if (blocks > 0x7FFFFFFFLL) return LC_ERR_UNSUPPORTED;  // past the grid's x limit
+  const unsigned grid = (unsigned)blocks;
   if (dtype == LC_DTYPE_F32)
     lse_merge_parts_kernel<float><<<grid, 256, 0, stream>>>(
         static_cast<const float *>(parts), lses, n_parts, static_cast<float *>(out), lse_out,

@@ -306,9 +306,11 @@ class GpuRingRank:
         return slot
 
     def combine(self, slots):
+        """The rank's result, always in fresh tensors (the partial buffers are
+        reused by the next forward, so a one-step result is copied out)."""
         n = len(slots)
         if n == 1:
-            return self.parts[0], self.lses[0]
+            return self.parts[0].clone(), self.lses[0].clone()
         return self.api.lse_merge_parts(self.parts[:n], self.lses[:n])
 
     def forward(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, group=None,

@@ -94,7 +94,8 @@ typedef struct {
  * work lists.  Source: "longcat-video-rs" section 03-03 and the section 02
  * table row (local window + strided global blocks, block=64); myzaker / QbitAI
  * "背后技术原理" (condition frames first, isolated from noise).
- *   T: latent frames including condition frames (T > n_cond_frames >= 0);
+ *   T: latent frames including condition frames (T > n_cond_frames >= 0: the
+ *      frames to generate are never empty, so n_cond_frames == T is refused);
  *   block: 64; local >= 0; stride: <= 0 none, 1 dense, > 1 strided globals.
  * Errors: LC_ERR_INVALID_ARGUMENT (out NULL, T/H/W <= 0, local < 0,
  * n_cond_frames outside [0, T), token count >= 2^31), LC_ERR_UNSUPPORTED
@@ -388,7 +389,8 @@ lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void
  * flags: LC_MERGE_INIT (o_acc and lse_acc not read; o_acc may then be NULL
  * when out is given).  lse_acc always receives the merged lse.  Errors:
  * LC_ERR_INVALID_ARGUMENT (NULL or misaligned pointer, bad sizes or flags),
- * LC_ERR_UNSUPPORTED (head_dim != 64).
+ * LC_ERR_UNSUPPORTED (head_dim != 64, or more rows than one launch covers:
+ * batch x n_tokens x heads x 8 threads past 2^31 - 1 blocks of 256).
  */
 lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
                            const float *lse_part, void *out, int batch, long long n_tokens,
@@ -404,7 +406,7 @@ lc_status lc_bsa_lse_merge(float *o_acc, float *lse_acc, const void *o_part,
  * lse = m + log sum_i w_i (a row whose lse are all -inf: 0 and -inf).  One
  * pass, fp32 arithmetic, one rounding to dtype.  Errors: LC_ERR_INVALID_ARGUMENT
  * (NULL or misaligned pointer, n_parts <= 0, bad sizes), LC_ERR_UNSUPPORTED
- * (head_dim != 64).
+ * (head_dim != 64, or more rows than one launch covers, as lc_bsa_lse_merge).
  */
 lc_status lc_bsa_lse_merge_parts(const void *parts, const float *lses, int n_parts, void *out,
                                  float *lse_out, int batch, long long n_tokens, int heads,
@@ -419,6 +421,16 @@ lc_status lc_bsa_lse_merge_parts(const void *parts, const float *lses, int n_par
 lc_status lc_last_device_status(void *stream);
 
 /*
+ * lc_device_status_decode -- the status lc_last_device_status reports for a
+ * device status word: bit 0 (a bounded in-kernel wait gave up) gives
+ * LC_ERR_TIMEOUT, else bit 1 (an in-kernel check of the plan's lists failed:
+ * a block id past the pattern, an empty member mask, a list bound outside
+ * the plan's entries) gives LC_ERR_DEVICE_CHECK, else LC_OK.  Pure host
+ * function, no CUDA call.
+ */
+lc_status lc_device_status_decode(int word);
+
+/*
  * lc_debug_watchdog_selftest -- launch one CTA that waits, with the same
  * bounded wait the attention kernel uses, on a barrier that nothing ever
  * arrives on; the wait gives up after timeout_us microseconds and the kernel
@@ -426,6 +438,17 @@ lc_status lc_last_device_status(void *stream);
  * (LC_ERR_TIMEOUT when the watchdog works).  For tests of failure detection.
  */
 lc_status lc_debug_watchdog_selftest(int timeout_us, void *stream);
+
+/*
+ * lc_debug_scratch_pool_used_high -- the high-water mark, in bytes, of the
+ * memory in use from the library's own scratch pool on the current device
+ * (the stream-ordered pool the allocating entry points draw per-call scratch
+ * from).  With reset != 0 the mark is first reset to the bytes in use now.
+ * For tests that check which calls draw scratch (the allocation-free entry
+ * point must not).  Synchronous; no GPU work.  Errors: LC_ERR_INVALID_ARGUMENT
+ * when bytes is NULL, LC_ERR_CUDA when the pool cannot be reached.
+ */
+lc_status lc_debug_scratch_pool_used_high(unsigned long long *bytes, int reset);
 
 /* Static description of a status code. */
 const char *lc_status_string(lc_status s);

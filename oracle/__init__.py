@@ -93,10 +93,13 @@ def max_threads() -> int:
 def segment_sizes(T: int, H: int, W: int, n_cond: int, block: int = 64):
     """(Nc, Nn, Cb, Nb): condition / noisy token counts and block counts.
     Condition frames come first on the time axis (myzaker / QbitAI page,
-    section on the unified tasks)."""
-    if min(T, H, W, block) <= 0 or not 0 <= n_cond <= T:
+    section on the unified tasks: no condition frame for text-to-video, one
+    for image-to-video, several for continuation -- the frames after them are
+    the ones generated).  Reading taken: at least one frame is generated, so
+    0 <= n_cond < T."""
+    if min(T, H, W, block) <= 0 or not 0 <= n_cond < T:
         raise ValueError(f"bad sizes T={T} H={H} W={W} block={block} n_cond={n_cond} "
-                         "(n_cond counts latent frames, 0 <= n_cond <= T)")
+                         "(n_cond counts latent frames, 0 <= n_cond < T)")
     Nc = n_cond * H * W
     Nn = (T - n_cond) * H * W
     return Nc, Nn, -(-Nc // block), -(-Nn // block)

@@ -48,6 +48,19 @@ def test_status_strings(lib):
     assert lib.lc_status_string(99).decode() == "unknown status"
 
 
+def test_device_status_word_decoding(lib):
+    """The device status word's bits map to the codes lc_last_device_status
+    returns: bit 0 (a bounded wait gave up) before bit 1 (a failed in-kernel
+    check of the plan's lists)."""
+    f = lib.lc_device_status_decode
+    f.argtypes, f.restype = [ctypes.c_int], ctypes.c_int
+    assert f(0) == 0
+    assert f(1) == 5       # LC_ERR_TIMEOUT
+    assert f(2) == 6       # LC_ERR_DEVICE_CHECK
+    assert f(3) == 5
+    assert f(4) == 0       # bits the kernels never set
+
+
 def test_plan_argument_errors_before_any_gpu_work(lib):
     h = ctypes.c_void_p()
     f = lib.lc_bsa_plan_create

@@ -139,10 +139,19 @@ def test_large_logits_exercise_rescaling(api, name, qscale):
     g = out.float().numpy().astype(np.float64)
     err = np.abs(g - ref_out)
     # outputs are larger and sharper here; bf16 rounding of R(q), R(k) moves
-    # logits by up to ~|s| * 2^-8, so the bound scales with the query scale.
+    # logits by up to ~|s| * 2^-8, so the bound against the exact oracle
+    # scales with the query scale.
     assert err.max() <= parity.BF16_MAX_ABS * qscale, err.max()
     assert err.mean() <= parity.BF16_MEAN_ABS * qscale, err.mean()
     assert np.abs(lse.numpy() - ref_lse).max() <= parity.BF16_LSE_ABS * qscale
+    # Against the oracle on bf16-rounded R(q), R(k) the logit rounding is
+    # gone, so bounds that do not grow with the logits apply: a fault in the
+    # rescaling (a wrong correction factor, a lost or doubled P) shows here.
+    r_out, r_lse = parity.oracle_on_rounded_operands(w, inputs)
+    rmx, rmean, rl = parity.assert_rounded_operand_close(g, lse.numpy(), r_out, r_lse,
+                                                         inputs["v"])
+    print("%s x%g: exact max %.3g mean %.3g | rounded-operand max %.3g mean %.3g lse %.3g" %
+          (name, qscale, err.max(), err.mean(), rmx, rmean, rl))
 
 
 @pytest.mark.parametrize("name", ["small_i2v", "ragged", "many_heads", "batch2"])
@@ -218,8 +227,8 @@ def test_deterministic(api):
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
-FULL = ["i2v_480p", "refine_720p", "continuation_cached", "sweep_l2s8", "sweep_l1s32",
-        "sweep_dense"]
+FULL = ["i2v_480p", "refine_720p", "continuation_cached", "sweep_dense", "sweep_l2s4",
+        "sweep_l2s8", "sweep_l1s16", "sweep_l1s32"]
 
 
 @pytest.mark.parametrize("name", FULL)
@@ -238,25 +247,20 @@ def test_full_size_sampled_rows(api, name):
                                                                   mean, lerr))
 
 
-@pytest.mark.parametrize("name", ["i2v_480p", "refine_720p"])
+@pytest.mark.parametrize("name", ["i2v_480p", "refine_720p", "continuation_cached"])
 def test_full_size_all_rows_of_two_heads(api, name):
     """Every query row of heads 0 and 31 at full size (the benchmark's launch),
-    element by element against the oracle."""
+    element by element against the oracle; for the cached form the rows are
+    the noisy queries over the cached condition keys plus the noisy keys."""
     w = synthetic.get(name)
     inputs = synthetic.make_inputs(w)
     out, lse = run_gpu(api, w, inputs)
     heads = [0, w.heads - 1]
+    nq = w.n_noisy_tokens if w.cached else w.n_tokens
     sub = {k: v[:, :, heads].contiguous() for k, v in inputs.items()}
-    ref_out, ref_lse = oracle.attention_rows(
-        sub["q"], sub["k"], sub["v"], H=w.H, W=w.W, Nc=w.n_cond_tokens, block=w.block,
-        local=w.local, stride=w.stride, rows=oracle.all_rows(1, w.n_tokens, 2))
-    g = out[0][:, heads].float().numpy().astype(np.float64).transpose(1, 0, 2).reshape(-1, 64)
-    err = np.abs(g - ref_out)
-    assert err.max() <= parity.BF16_MAX_ABS and err.mean() <= parity.BF16_MEAN_ABS, \
-        (err.max(), err.mean())
-    gl = lse[0][heads].numpy().astype(np.float64).reshape(-1)
-    assert np.abs(gl - ref_lse).max() <= parity.BF16_LSE_ABS
-    print("%s all rows of heads %s: max %.3g mean %.3g" % (name, heads, err.max(), err.mean()))
+    ref_out, ref_lse = parity.oracle_rows(w, sub, np.arange(nq), heads=[0, 1])
+    mx, mean, lerr = parity.compare(w, out, lse, ref_out, ref_lse, np.arange(nq), heads=heads)
+    print("%s all rows of heads %s: max %.3g mean %.3g lse %.3g" % (name, heads, mx, mean, lerr))
 
 
 def test_argument_errors_on_gpu(api):
@@ -317,4 +321,10 @@ def test_custom_softmax_scale(api, dtype):
         k = 0.3 / 0.125
         assert err.max() <= parity.BF16_MAX_ABS * k and err.mean() <= parity.BF16_MEAN_ABS * k
         assert np.abs(lse.cpu().numpy() - ref_l).max() <= parity.BF16_LSE_ABS * k
+        # with the logit rounding modelled, the plain bf16 bounds
+        r_o, r_l = parity.oracle_on_rounded_operands(w, x, scale=0.3)
+        rmx, rmean, rl = parity.assert_rounded_operand_close(
+            out.cpu().float().numpy(), lse.cpu().numpy(), r_o, r_l, x["v"])
+        print("scale 0.3: exact max %.3g mean %.3g | rounded-operand max %.3g mean %.3g lse %.3g"
+              % (err.max(), err.mean(), rmx, rmean, rl))
     assert torch.equal(oc, out[:, Nc:]) and torch.equal(lc, lse[:, :, Nc:])

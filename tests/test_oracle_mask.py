@@ -149,3 +149,13 @@ def test_random_geometries_csr_against_token_mask():
             return min(64, Nc - 64 * b) if b < Cb else min(64, Nn - 64 * (b - Cb))
         pairs = sum(ntok(r) * ntok(int(c)) for r in range(Cb + Nb) for c in ci[rp[r]:rp[r + 1]])
         assert pairs == int(token_mask(N, Nc, 64, local, stride).sum())
+
+
+def test_every_frame_a_condition_frame_is_refused():
+    """At least one frame is generated: n_cond == T is outside the domain on
+    both sides of the boundary (lc_bsa_plan_create refuses it as well)."""
+    with pytest.raises(ValueError):
+        oracle.segment_sizes(4, 8, 16, 4)
+    with pytest.raises(ValueError):
+        oracle.block_csr(4, 8, 16, 64, 2, 4, 4)
+    assert oracle.segment_sizes(4, 8, 16, 3) == (384, 128, 6, 2)

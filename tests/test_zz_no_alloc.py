@@ -58,3 +58,26 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(api):
         lerr = (lse - ref_lse).abs().max().item()
         assert lerr <= parity.BF16_LSE_ABS, (call, lerr)
         assert np.isfinite(out.float().cpu().numpy()).all()
+
+
+def test_noalloc_draws_no_scratch_from_the_library_pool(api):
+    """The allocating entry point draws its per-call scratch (rotated K, the
+    scheduler counter) from the library's pool; the allocation-free one must
+    not touch it.  The pool's high-water mark, reset to what is in use when
+    no call is running, stays there across a noalloc call, while one
+    lc_bsa_forward call raises it."""
+    plan = api.Plan(W.T, W.H, W.W, local=W.local, stride=W.stride, n_cond=W.n_cond)
+    rope = api.Rope3D(W.T, W.H, W.W)
+    x = {k: v.cuda() for k, v in synthetic.make_inputs(W).items()}
+    out = torch.zeros_like(x["q"])
+    lse = torch.zeros(1, W.heads, W.n_tokens, dtype=torch.float32, device="cuda")
+    api.forward(x["q"], x["k"], x["v"], plan, rope)  # the pool exists and holds nothing now
+    torch.cuda.synchronize()
+    base = api.scratch_pool_used_high(reset=True)
+    assert _call_noalloc_c_abi(api, x["q"], x["k"], x["v"], out, lse, plan, rope) == api.LC_OK
+    torch.cuda.synchronize()
+    assert api.scratch_pool_used_high() == base
+    api.forward(x["q"], x["k"], x["v"], plan, rope)
+    torch.cuda.synchronize()
+    assert api.scratch_pool_used_high() > base
+    assert api.last_device_status() == api.LC_OK

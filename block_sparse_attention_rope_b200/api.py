@@ -93,6 +93,7 @@ COND_K_ROTATED = 1  # LC_FLAG_COND_K_ROTATED
 Q_ROTATED = 2       # LC_FLAG_Q_ROTATED
 K_ROTATED = 4       # LC_FLAG_K_ROTATED
 KEEP_EMPTY_ROWS = 8  # LC_FLAG_KEEP_EMPTY_ROWS
+OVERLAP_PREVIOUS = 16  # LC_FLAG_OVERLAP_PREVIOUS
 
 
 def status_string(s: int) -> str:
@@ -437,7 +438,7 @@ def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
                   softmax_scale: float = 0.0, q_norm: Optional[torch.Tensor] = None,
                   k_norm: Optional[torch.Tensor] = None, norm_eps: float = 1e-6,
                   q_rotated: bool = False, k_rotated: bool = False,
-                  keep_empty_rows: bool = False, stream=None):
+                  keep_empty_rows: bool = False, overlap_previous: bool = False, stream=None):
     """Partial attention of one shard pair (lc_bsa_forward_shard): q holds the
     shard plan's query tokens [B, nq, heads, 64], k / v its key tokens
     [B, nk, heads, 64] (pre-RoPE, bf16, or already normalised and rotated with
@@ -455,7 +456,8 @@ def forward_shard(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
     _check_bmhk("out", out, q.shape, q.dtype)
     _check_bmhk("lse", lse, (B, heads, nq), torch.float32)
     flags = ((Q_ROTATED if q_rotated else 0) | (K_ROTATED if k_rotated else 0) |
-             (KEEP_EMPTY_ROWS if keep_empty_rows else 0))
+             (KEEP_EMPTY_ROWS if keep_empty_rows else 0) |
+             (OVERLAP_PREVIOUS if overlap_previous else 0))
     opts = _opts(flags, q_norm, k_norm, norm_eps, hd)
     _check(lib.lc_bsa_forward_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     lse.data_ptr(), B, heads, hd, _dtype_code(q),

@@ -274,8 +274,13 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   if (s != LC_OK) return s;
   unsigned flags;
   lc_qk_norm norm;
-  if (!parse_opts(opts, LC_FLAG_Q_ROTATED | LC_FLAG_K_ROTATED | LC_FLAG_KEEP_EMPTY_ROWS, &flags,
-                  &norm))
+  if (!parse_opts(opts,
+                  LC_FLAG_Q_ROTATED | LC_FLAG_K_ROTATED | LC_FLAG_KEEP_EMPTY_ROWS |
+                      LC_FLAG_OVERLAP_PREVIOUS,
+                  &flags, &norm))
+    return LC_ERR_INVALID_ARGUMENT;
+  // An overlapping launch must not be preceded by a fill of the rows without keys.
+  if ((flags & LC_FLAG_OVERLAP_PREVIOUS) && !(flags & LC_FLAG_KEEP_EMPTY_ROWS))
     return LC_ERR_INVALID_ARGUMENT;
   if (!q || !k || !v || !out || !lse) return LC_ERR_INVALID_ARGUMENT;
   if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(out) ||
@@ -291,6 +296,7 @@ extern "C" lc_status lc_bsa_forward_shard(const void *q, const void *k, const vo
   sv.k_n = lc_block_token(plan, plan->khi) - sv.k_lo;
   sv.q_rotated = (flags & LC_FLAG_Q_ROTATED) != 0;
   sv.k_rotated = (flags & LC_FLAG_K_ROTATED) != 0;
+  sv.overlap_previous = (flags & LC_FLAG_OVERLAP_PREVIOUS) != 0;
   if (sv.q_n == 0) return LC_OK;
   int *dev_status = lc_device_status_ptr(&s);
   if (s != LC_OK) return s;

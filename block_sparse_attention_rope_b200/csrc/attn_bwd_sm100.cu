@@ -357,16 +357,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t ph = (q_it / kQStages) & 1;
           ok = wait_bar(ctx, ctx.bar(B_QG_EMPTY + s), ph ^ 1);
           if (!ok) break;
-          // no second query block, or an entry that fails the plan check: a
-          // box past the noisy segment's end reads zeros
-          int sa = 1, ra = p.Nn, na, sb = 1, rb = p.Nn, nb;
-          const uint32_t ea = __ldg(it.ent + 2 * t);
-          if (qentry_ok(p, ea)) qblock(p, ea, sa, ra, na);
-          else atomicOr(p.status, LC_DEVSTAT_CHECK);
+          // (TMA loads may start anywhere: an entry that fails the plan check
+          // reads zeros or other rows here; the dQ and lse / D paths, which
+          // address memory with it, check it and report it)
+          int sa, ra, na, sb, rb, nb;
+          qblock(p, __ldg(it.ent + 2 * t), sa, ra, na);
           if (2 * t + 1 < it.len) {
-            const uint32_t eb = __ldg(it.ent + 2 * t + 1);
-            if (qentry_ok(p, eb)) qblock(p, eb, sb, rb, nb);
-            else atomicOr(p.status, LC_DEVSTAT_CHECK);
+            qblock(p, __ldg(it.ent + 2 * t + 1), sb, rb, nb);
+          } else {  // no second query block: a box past the noisy segment's end reads zeros
+            sb = 1;
+            rb = p.Nn;
           }
           const uint32_t bar = ctx.bar(B_QG_FULL + s);
           lcptx::mbar_arrive_expect_tx(bar, 2 * kTileBytes);
@@ -594,9 +594,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk) {
               const int e = 2 * t + blk;
-              if (e >= it.len || !qentry_ok(p, __ldg(it.ent + e))) continue;
+              if (e >= it.len) continue;
+              const uint32_t ent = __ldg(it.ent + e);
+              if (!qentry_ok(p, ent)) {
+                atomicOr(p.status, LC_DEVSTAT_CHECK);
+                continue;
+              }
               int qs, qr, qn;
-              qblock(p, __ldg(it.ent + e), qs, qr, qn);
+              qblock(p, ent, qs, qr, qn);
               const int tok0 = (qs ? p.Nc : 0) + qr;
 #pragma unroll
               for (int hd = 0; hd < 2; ++hd)
@@ -645,9 +650,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         // attended query tokens of this warp's query block, for this key row
         int lim = 0;
         const int e = 2 * t + half;
-        if (key_valid && e < it.len) {
-          const uint32_t ent = __ldg(it.ent + e);
-          if (qentry_ok(p, ent) && ((ent >> (24 + (kr >> 6))) & 1u)) {
+        if (key_valid && e < it.len) {  // (an entry failing the plan check only
+          const uint32_t ent = __ldg(it.ent + e);  // yields a mask here; the producer flags it)
+          if ((ent >> (24 + (kr >> 6))) & 1u) {
             int qs, qr, qn;
             qblock(p, ent, qs, qr, qn);
             lim = qn;

@@ -132,6 +132,12 @@ struct __align__(64) Sm100Params {
   const float *q_norm_w;   // RMSNorm weights [64] applied ahead of the rotation, or NULL
   const float *k_norm_w;
   float norm_eps;
+  // Programmatic dependent launch (shard steps of a ring): the next kernel on
+  // the stream may launch once every CTA is set up, and this grid does not
+  // finish before the previous one.  exit_counter (with work_counter, the
+  // plan's own pair) counts finished CTAs; the last one resets both to 0.
+  int pdl;
+  int *exit_counter;
 };
 
 // Shared memory carve-up (offsets from a 1024-aligned base).
@@ -297,19 +303,17 @@ __device__ __forceinline__ float row_max(const float (&s)[128]) {
 // is not attended), bits 8-15 = same for the second block.
 __device__ __forceinline__ uint32_t tile_limits(const Sm100Params &p, const Item &it, int tt,
                                                 int qsub) {
+  // (an entry that fails the plan check only gives a mask here; the
+  // producer reports it and loads zeros for it)
   if (2 * tt >= it.len) return 0u;
   const uint32_t ea = __ldg(it.ent + 2 * tt);
-  int sx, rx, na = 0, nb = 0;
-  if (entry_ok(p, ea)) {
-    entry_block(p, ea, sx, rx, na);
-    if (!((ea >> (24 + qsub)) & 1u)) na = 0;
-  }
+  int sx, rx, na, nb = 0;
+  entry_block(p, ea, sx, rx, na);
+  if (!((ea >> (24 + qsub)) & 1u)) na = 0;
   if (2 * tt + 1 < it.len) {
     const uint32_t eb = __ldg(it.ent + 2 * tt + 1);
-    if (entry_ok(p, eb)) {
-      entry_block(p, eb, sx, rx, nb);
-      if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
-    }
+    entry_block(p, eb, sx, rx, nb);
+    if (!((eb >> (24 + qsub)) & 1u)) nb = 0;
   }
   return (uint32_t)na | ((uint32_t)nb << 8);
 }
@@ -383,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   lcptx::tc_fence_after();
   const uint32_t tmem = misc[0];
   const bool k_rot = p.k_prerotated != 0;
+  if (p.pdl) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Register split: the softmax warpgroups (warps 0-7) hold a 128-column row
   // of S in registers; the producer / MMA / RoPE warpgroup needs few.
@@ -877,6 +882,17 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
   __syncthreads();
   lcptx::tc_fence_after();
   if (warp == kWarpMma) lcptx::tmem_dealloc(tmem, kTmemCols);
+  if (tid == 0) {
+    // Every producer has taken its last item: the last CTA out resets the
+    // plan's scheduler for the next launch that uses it.
+    if (p.exit_counter && atomicAdd(p.exit_counter, 1) == (int)gridDim.x - 1) {
+      *p.work_counter = 0;
+      *p.exit_counter = 0;
+      __threadfence();
+    }
+    // Finish no earlier than the previous grid on the stream.
+    if (p.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -1265,14 +1281,34 @@ lc_status lc_launch_forward_sm100(const void *q, const void *k, const void *v, c
       prm.k_prerotated = 1;
     }
   }
-  if (e == cudaSuccess && s == LC_OK)
-    e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&counter), sizeof(int), pool, stream);
-  if (e == cudaSuccess && s == LC_OK) {
-    prm.work_counter = counter;
-    e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
-    if (e == cudaSuccess) {
-      kern<<<grid, kThreads, smem, stream>>>(prm);
-      e = cudaGetLastError();
+  const bool overlap = sharded && shard->overlap_previous;
+  if (overlap && e == cudaSuccess && s == LC_OK) {
+    // The plan's own scheduler (zero between launches) and a programmatic
+    // dependent launch: no stream operation separates it from the previous kernel.
+    prm.work_counter = plan->sched;
+    prm.exit_counter = plan->sched + 1;
+    prm.pdl = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+  } else {
+    if (e == cudaSuccess && s == LC_OK)
+      e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&counter), sizeof(int), pool, stream);
+    if (e == cudaSuccess && s == LC_OK) {
+      prm.work_counter = counter;
+      e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+      if (e == cudaSuccess) {
+        kern<<<grid, kThreads, smem, stream>>>(prm);
+        e = cudaGetLastError();
+      }
     }
   }
   if (counter) cudaFreeAsync(counter, stream);

@@ -79,6 +79,8 @@ struct lc_bsa_plan_s {
   int2 *kgrp_blk;           // [KG]      the group's key blocks (second -1 if none)
   unsigned long long *pairs;  // [2] attended token pairs: all rows, noisy rows
   int *err;                 // [1] planner consistency flag
+  int *sched;               // [2] work-item and finished-CTA counters of launches that use
+                            //     the plan's own scheduler (zero between launches)
   long long pairs_host[2];
   bool info_cached;
 };
@@ -198,6 +200,7 @@ enum lc_fwd_mode { LC_FWD_FULL = 0, LC_FWD_CACHED = 1, LC_FWD_COND = 2, LC_FWD_S
 struct lc_shard_view {
   long long q_lo, q_n, k_lo, k_n;
   bool q_rotated, k_rotated;  // q / k already hold R(norm(x)) (rotated once per ring)
+  bool overlap_previous;      // programmatic dependent launch, the plan's own scheduler
 };
 
 // RMSNorm of q and k ahead of the rotation: device fp32 weights [64] or NULL.

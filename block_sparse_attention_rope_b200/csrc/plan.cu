@@ -457,7 +457,7 @@ static lc_status plan_create(lc_bsa_plan *out, int T, int H, int W, int block, i
   carve<int>(probe, p->G); carve<unsigned long long>(probe, 2); carve<int>(probe, 1);
   carve<int>(probe, p->nq + 1); carve<int>(probe, nnz); carve<int>(probe, p->nq);
   carve<int>(probe, p->KG + 1); carve<int>(probe, p->KG); carve<uint32_t>(probe, nnz);
-  carve<int>(probe, p->KG); carve<int2>(probe, p->KG);
+  carve<int>(probe, p->KG); carve<int2>(probe, p->KG); carve<int>(probe, 2);
   size_t bytes = reinterpret_cast<size_t>(probe);
   cudaError_t e = cudaMallocAsync(&p->mem, bytes, st);
   if (e != cudaSuccess) { delete p; return lc_from_cuda(e); }
@@ -479,9 +479,11 @@ static lc_status plan_create(lc_bsa_plan *out, int T, int H, int W, int block, i
   p->kgrp_ent = carve<uint32_t>(q, nnz);
   p->kgrp_order = carve<int>(q, p->KG);
   p->kgrp_blk = carve<int2>(q, p->KG);
+  p->sched = carve<int>(q, 2);
 
   e = cudaMemsetAsync(p->pairs, 0, 2 * sizeof(unsigned long long), st);
   if (e == cudaSuccess) e = cudaMemsetAsync(p->err, 0, sizeof(int), st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(p->sched, 0, 2 * sizeof(int), st);
   const int tpb = 256;
   int row_blocks = (p->nq * 32 + tpb - 1) / tpb;
   int grp_blocks = (p->G * 32 + tpb - 1) / tpb;

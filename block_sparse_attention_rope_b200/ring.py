@@ -300,9 +300,13 @@ class GpuRingRank:
                                norm_eps=self.norm_eps)
 
     def partial(self, src, q_rot, k_rot, v, slot):
+        # Steps after the rank's first write their own slot and read inputs
+        # that were complete before the first step: each may start on the SMs
+        # the previous step's kernel frees while its last items finish.
         self.api.forward_shard(q_rot, k_rot, v, self.plans[src], self.rope, out=self.parts[slot],
                                lse=self.lses[slot], softmax_scale=self.softmax_scale,
-                               q_rotated=True, k_rotated=True, keep_empty_rows=True)
+                               q_rotated=True, k_rotated=True, keep_empty_rows=True,
+                               overlap_previous=slot > 0)
         return slot
 
     def combine(self, slots):

@@ -201,6 +201,8 @@ lc_status lc_bsa_forward_cached(const void *q, const void *k, const void *v,
 #define LC_FLAG_K_ROTATED 4u       /* k already holds R(norm_k(k)) (lc_bsa_forward_shard) */
 #define LC_FLAG_KEEP_EMPTY_ROWS 8u /* lc_bsa_forward_shard: rows of work groups without keys
                                       in the shard are left as they are (not set to 0, -inf) */
+#define LC_FLAG_OVERLAP_PREVIOUS 16u /* lc_bsa_forward_shard: the launch may start while the
+                                        previous kernel on the stream is still finishing */
 
 /*
  * Options of the _ex entry points and of lc_bsa_cond_cache.  A NULL options
@@ -366,7 +368,18 @@ lc_status lc_bsa_plan_token_range(lc_bsa_plan plan, long long *q_lo, long long *
  * the plan's work groups (4 query blocks) that have no key in the shard are
  * not written, for a caller whose buffers already hold (0, -inf) there (the
  * set of such rows is fixed by the plan); rows of groups with keys are always
- * written, (0, -inf) included.  bf16 only (LC_DTYPE_F32:
+ * written, (0, -inf) included.  LC_FLAG_OVERLAP_PREVIOUS (needs
+ * LC_FLAG_KEEP_EMPTY_ROWS): the launch is made with programmatic dependent
+ * launch, so that its CTAs take the SMs the previous kernel on the stream
+ * frees while that kernel's last work items finish, and its work-item
+ * counter is the plan's own (reset by the kernel's last CTA) instead of one
+ * set up by a memset between the launches.  The caller guarantees that this
+ * launch reads nothing the previous kernel on the stream writes (true of the
+ * steps of one ring rank: each writes its own out / lse, all read inputs
+ * that were complete before the first step, which is made without the
+ * flag), and that no other launch with the same plan is in flight.  The
+ * kernel does not finish before the previous one, so a launch after it
+ * without the flag sees every step's results.  bf16 only (LC_DTYPE_F32:
  * LC_ERR_UNSUPPORTED).  Errors as lc_bsa_forward.
  */
 lc_status lc_bsa_forward_shard(const void *q, const void *k, const void *v, void *out, float *lse,

@@ -233,6 +233,52 @@ def test_keep_empty_rows_leaves_groups_without_keys(api):
     assert (o1[:, :Nc] == 0).all() and (l1[:, :, :Nc] == -float("inf")).all()
 
 
+def test_overlapping_shard_launches_are_bit_exact(api):
+    """LC_FLAG_OVERLAP_PREVIOUS (programmatic dependent launch, the plan's
+    self-resetting scheduler): a rank's steps launched back to back, each
+    overlapping the previous one, give the same bits as separate launches;
+    launching the same plans again (their schedulers reset by the previous
+    launch's last CTA) gives them once more.  The flag needs keep_empty_rows."""
+    w = RAGGED
+    x = synthetic.make_inputs(w, device="cuda")
+    rope = api.Rope3D(w.T, w.H, w.W)
+    Cb, Nb = blocks(w)
+    qs = (4, 13)                     # group edges: condition block 4, noisy 5 + 8
+    steps = [(0, 6), (6, 14), (14, Cb + Nb), (3, 9)]
+    plans = [api.Plan(w.T, w.H, w.W, local=w.local, stride=w.stride, n_cond=w.n_cond,
+                      q_blocks=qs, k_blocks=ks) for ks in steps]
+    (qa, qb) = plans[0].q_tokens
+    q = rope.apply(x["q"][:, qa:qb].contiguous(), tok_offset=qa)
+    kv = []
+    for p in plans:
+        ka, kb = p.k_tokens
+        kv.append((rope.apply(x["k"][:, ka:kb].contiguous(), tok_offset=ka),
+                   x["v"][:, ka:kb].contiguous()))
+
+    def run(overlap):
+        outs = [torch.zeros(w.batch, qb - qa, w.heads, 64, dtype=torch.bfloat16, device="cuda")
+                for _ in plans]
+        lses = [torch.full((w.batch, w.heads, qb - qa), -float("inf"), device="cuda")
+                for _ in plans]
+        for i, (p, (k, v)) in enumerate(zip(plans, kv)):
+            api.forward_shard(q, k, v, p, rope, out=outs[i], lse=lses[i], q_rotated=True,
+                              k_rotated=True, keep_empty_rows=True,
+                              overlap_previous=overlap and i > 0)
+        torch.cuda.synchronize()
+        assert api.last_device_status() == 0
+        return outs, lses
+
+    ref = run(False)
+    for _ in range(2):
+        got = run(True)
+        for a, b in zip(ref[0] + ref[1], got[0] + got[1]):
+            assert torch.equal(a, b)
+    with pytest.raises(api.LcError) as e:
+        api.forward_shard(q, kv[0][0], kv[0][1], plans[0], rope, q_rotated=True,
+                          k_rotated=True, overlap_previous=True)
+    assert e.value.status == api.LC_ERR_INVALID_ARGUMENT
+
+
 @pytest.mark.parametrize("n_parts", [1, 3, 8])
 def test_lse_merge_parts_kernel(api, n_parts):
     g = torch.Generator().manual_seed(n_parts)

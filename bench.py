@@ -294,8 +294,8 @@ def time_ring(api, synthetic, torch, name, world, stream, reps=3):
             "ms_per_rank_max": round(max(per), 3), "ms_per_rank_mean": round(sum(per) / world, 3),
             "whole_sequence_ms": round(full, 3), "ideal_ms": round(full / world, 3),
             "compute_efficiency": round(full / world / max(per), 3),
-            "kernels": "per rank: rope_apply (q, k once); per step: bsa_sm100_kernel "
-                       "(shard_fill where a group has no entry); lse_merge_parts once"}
+            "kernels": "per rank: rope_apply (q, k once); per step: bsa_sm100_kernel (steps "
+                       "after the first by programmatic dependent launch); lse_merge_parts once"}
 
 
 def time_e2e(api, torch, w, host, plan, rope, steps, stream):

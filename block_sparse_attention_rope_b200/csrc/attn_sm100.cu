@@ -72,8 +72,19 @@ constexpr int kRopeThreads = 64;
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kBoxBytes = 64 * 128;    // one 64-row TMA box
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 320, kColP0 = 384,
-                   kColP1 = 448;
+// 1: three S buffers [0,128) [128,256) [256,384) taken in turn by the
+// (tile, warpgroup) sequence, each tile's P written as bf16 over the first 64
+// columns of its own S buffer, O0 [384,448) O1 [448,512): the next S never
+// waits for a warpgroup to load its current one, and P never waits for the
+// previous P*V (its buffer was last read by the P*V three positions back,
+// which the tensor pipe executed before this tile's S).  0: two S buffers
+// S0 [0,128) S1 [128,256), O0 [256,320) O1 [320,384), P0 [384,448) P1 [448,512).
+#ifndef LC_S3
+#define LC_S3 1
+#endif
+constexpr bool kS3 = LC_S3 != 0;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = kS3 ? 384 : 256, kColO1 = kS3 ? 448 : 320,
+                   kColP0 = 384, kColP1 = 448;
 constexpr uint32_t kIdescQK = lcptx::idesc_bf16_f32(128, 128, 0, 0);
 constexpr uint32_t kIdescPV = lcptx::idesc_bf16_f32(128, 64, 0, 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: p stays below 2^8 before a rescale
@@ -162,8 +173,8 @@ enum {
   B_KEMPTY = B_KFULL + 2 * kStages,
   B_VFULL = B_KFULL + 3 * kStages,
   B_VEMPTY = B_KFULL + 4 * kStages,
-  B_SFULL = B_KFULL + 5 * kStages,  // [2]
-  B_SFREE = B_SFULL + 2,            // [2]
+  B_SFULL = B_KFULL + 5 * kStages,  // [2] per warpgroup, or [3] per S buffer (kS3)
+  B_SFREE = B_SFULL + 3,            // [2] (not with kS3)
   B_PFULL = B_SFREE + 2,            // [2]
   B_ODONE = B_PFULL + 2,            // [2]
   B_EPI = B_ODONE + 2,              // [2] O rows staged in smem
@@ -351,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       lcptx::mbar_init(ctx.bar(B_QREADY + i), kRopeThreads);
       lcptx::mbar_init(ctx.bar(B_QEMPTY + i), 1);
     }
+    lcptx::mbar_init(ctx.bar(B_SFULL + 2), 1);
     for (int i = 0; i < 2; ++i) {
       lcptx::mbar_init(ctx.bar(B_SFULL + i), 1);
       lcptx::mbar_init(ctx.bar(B_SFREE + i), 4);
@@ -499,6 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
       int cs = 0;        // K/V stage of the current tile
       uint32_t cph = 0;  // and its phase parity
       uint32_t sfree_bits = 0, pfull_bits = 0;  // bit i: phase parity for tile i
+      uint32_t kpos = 0;  // (tile, warpgroup) position of the item's tile 0, warpgroup 0
       const int kbar = k_rot ? B_KFULL : B_KREADY;
       // Operand descriptors, built once: the high word (stride byte offset
       // 1024, version 1, 128-byte swizzle) is common; the low word holds the
@@ -526,25 +539,33 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
                   wait_bar(ctx, ctx.bar(B_QREADY + 2 * buf + 1), qph);
         if (!ok) break;
         const uint32_t q_lo = q_lo0 + 2 * buf * kTileLo;
-        auto issue_s = [&](int i, int s) -> bool {
-          if (!wait_bar(ctx, ctx.bar(B_SFREE + i), ((sfree_bits >> i) & 1u) ^ 1u)) return false;
-          sfree_bits ^= 1u << i;
+        // k: the (tile, warpgroup) position; with kS3 its S buffer is k % 3.
+        auto issue_s = [&](int i, int s, uint32_t k) -> bool {
+          uint32_t d, bar;
+          if (kS3) {
+            d = tmem + 128u * (k % 3u);
+            bar = ctx.bar(B_SFULL + (int)(k % 3u));
+          } else {
+            if (!wait_bar(ctx, ctx.bar(B_SFREE + i), ((sfree_bits >> i) & 1u) ^ 1u)) return false;
+            sfree_bits ^= 1u << i;
+            d = tmem + (i ? kColS1 : kColS0);
+            bar = ctx.bar(B_SFULL + i);
+          }
           lcptx::tc_fence_after();
           const uint32_t qa = q_lo + i * kTileLo, kb = k_lo0 + s * kTileLo;
-          const uint32_t d = tmem + (i ? kColS1 : kColS0);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             lcptx::mma_ss(d, desc(qa + 2 * kk), desc(kb + 2 * kk), kIdescQK, kk > 0);
-          lcptx::mma_commit(ctx.bar(B_SFULL + i));
+          lcptx::mma_commit(bar);
           return true;
         };
-        auto issue_pv = [&](int i, int s, bool accumulate) -> bool {
+        auto issue_pv = [&](int i, int s, bool accumulate, uint32_t k) -> bool {
           if (!wait_bar(ctx, ctx.bar(B_PFULL + i), (pfull_bits >> i) & 1u)) return false;
           pfull_bits ^= 1u << i;
           lcptx::tc_fence_after();
           const uint32_t vb = v_lo0 + s * kTileLo;
           const uint32_t d = tmem + (i ? kColO1 : kColO0);
-          const uint32_t a = tmem + (i ? kColP1 : kColP0);
+          const uint32_t a = kS3 ? tmem + 128u * (k % 3u) : tmem + (i ? kColP1 : kColP0);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             lcptx::mma_ts(d, a + 8 * kk, desc(vb + 128 * kk), kIdescPV,
@@ -553,31 +574,35 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           return true;
         };
         // tile 0: both S tiles
-        ok = wait_bar(ctx, ctx.bar(kbar + cs), cph) && issue_s(0, cs) && issue_s(1, cs);
+        const uint32_t k0 = kpos;
+        ok = wait_bar(ctx, ctx.bar(kbar + cs), cph) && issue_s(0, cs, k0) && issue_s(1, cs, k0 + 1);
         if (!ok) break;
         if (!kKVMerged) lcptx::mma_commit(ctx.bar(B_KEMPTY + cs));
         for (int t = 0; t < ntiles && ok; ++t) {
           const bool more = t + 1 < ntiles;
           const int ns = cs + 1 == kStages ? 0 : cs + 1;
           const uint32_t nph = ns == 0 ? cph ^ 1u : cph;
+          const uint32_t kt = k0 + 2u * (uint32_t)t;
           if (more) {
-            ok = wait_bar(ctx, ctx.bar(kbar + ns), nph) && issue_s(0, ns);
+            ok = wait_bar(ctx, ctx.bar(kbar + ns), nph) && issue_s(0, ns, kt + 2);
             if (!ok) break;
           }
-          ok = (kKVMerged || wait_bar(ctx, ctx.bar(B_VFULL + cs), cph)) && issue_pv(0, cs, t > 0);
+          ok = (kKVMerged || wait_bar(ctx, ctx.bar(B_VFULL + cs), cph)) &&
+               issue_pv(0, cs, t > 0, kt);
           if (!ok) break;
           if (more) {
-            ok = issue_s(1, ns);
+            ok = issue_s(1, ns, kt + 3);
             if (!ok) break;
             if (!kKVMerged) lcptx::mma_commit(ctx.bar(B_KEMPTY + ns));
           }
-          ok = issue_pv(1, cs, t > 0);
+          ok = issue_pv(1, cs, t > 0, kt + 1);
           if (!ok) break;
           lcptx::mma_commit(ctx.bar(kKVMerged ? B_KEMPTY + cs : B_VEMPTY + cs));
           cs = ns;
           cph = nph;
         }
         if (!ok) break;
+        kpos = k0 + 2u * (uint32_t)ntiles;
         ++item_it;
       }
       // Drain: wait until every MMA this thread issued has completed.
@@ -655,11 +680,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
     const int row = tid & 127;             // TMEM lane == tile row
     const int qsub = 2 * wg + (row >> 6);  // member index of this row's query block
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + (wg ? kColS1 : kColS0);
     const uint32_t tO = tmem + lane_base + (wg ? kColO1 : kColO0);
-    const uint32_t tP = tmem + lane_base + (wg ? kColP1 : kColP0);
     const float sl2 = p.scale_log2;
     uint32_t item_it = 0, sfull_ph = 0, odone_ph = 0;
+    // kS3: this warpgroup's next (tile, warpgroup) position and the P*V
+    // products issued for it so far (ODONE completes once per product; a
+    // wait for the latest one takes its parity from this count).
+    uint32_t kpos = (uint32_t)wg, n_pv = 0;
     for (;;) {
       const int slot = item_it & 1;
       if (!wait_warp(ctx, ctx.bar(B_SCHED_FULL + slot), (item_it >> 1) & 1)) break;
@@ -677,9 +704,17 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         if ((t & 31) == 0) lim_lane = tile_limits(p, it, t + lane, qsub);
         const uint32_t lim = __shfl_sync(0xffffffffu, lim_lane, t & 31);
         const int na = lim & 0xFF, nb = (lim >> 8) & 0xFF;
-        ok = wait_warp(ctx, ctx.bar(B_SFULL + wg), sfull_ph);
+        // This tile's S (and, with kS3, its P) columns.
+        const uint32_t buf = kS3 ? kpos % 3u : 0u;
+        const uint32_t tS = tmem + lane_base + (kS3 ? 128u * buf : (wg ? kColS1 : kColS0));
+        const uint32_t tP = kS3 ? tS : tmem + lane_base + (wg ? kColP1 : kColP0);
+        if (kS3) {
+          ok = wait_warp(ctx, ctx.bar(B_SFULL + (int)buf), (kpos / 3u) & 1u);
+        } else {
+          ok = wait_warp(ctx, ctx.bar(B_SFULL + wg), sfull_ph);
+          sfull_ph ^= 1;
+        }
         if (!ok) break;
-        sfull_ph ^= 1;
         lcptx::tc_fence_after();
         uint32_t r0[32], r1[32], r2[32], r3[32];
         lcptx::tmem_ld32(tS, r0);
@@ -689,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         lcptx::tmem_wait_ld();
         lcptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_SFREE + wg));
+        if (!kS3 && lane == 0) lcptx::mbar_arrive(ctx.bar(B_SFREE + wg));
         float s[128];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -716,7 +751,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         // rescaled and P is redone from the logits kept in s.
         if (t == 0) m_ref = row_max(s) * sl2;
         float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        bool o_ready = (t == 0);  // P / O of this warpgroup free (previous P*V done)
+        // P / O of this warpgroup free (previous P*V done); with kS3 P goes
+        // to a buffer no product reads any more, so only O needs the wait.
+        bool o_ready = kS3 || t == 0;
         float l_tile = 0.f;
         // One pass: s <- s * mul + add in place, P = 2^s pipelined (the ex2 of
         // pair j is issued after pair j-8 is packed and summed), P to TMEM in
@@ -801,6 +838,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
           lcptx::tc_fence_after();
         }
         l_sum += l_tile;
+        // kS3: the previous tile's P*V (issued about a pass ago) is waited for
+        // before this tile's P is handed over, so that at most one product is
+        // ever outstanding and a parity wait on ODONE is never two phases
+        // behind; O may then be rescaled.
+        if (kS3 && n_pv > 0) {
+          ok = wait_warp(ctx, ctx.bar(B_ODONE + wg), (n_pv - 1u) & 1u);
+          if (!ok) break;
+          lcptx::tc_fence_after();
+        }
         if (rescale_o) {
           uint32_t o0[32], o1[32];
           lcptx::tmem_ld32(tO, o0);
@@ -821,12 +867,18 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_sm100_kernel(const __grid_con
         lcptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_PFULL + wg));
+        ++n_pv;
+        kpos += 2;
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> smem (swizzled) -> TMA store; lse
-      ok = wait_warp(ctx, ctx.bar(B_ODONE + wg), odone_ph);
+      if (kS3) {
+        ok = wait_warp(ctx, ctx.bar(B_ODONE + wg), (n_pv - 1u) & 1u);
+      } else {
+        ok = wait_warp(ctx, ctx.bar(B_ODONE + wg), odone_ph);
+        odone_ph ^= 1;
+      }
       if (!ok) break;
-      odone_ph ^= 1;
       lcptx::tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
       const int buf = item_it & 1;

@@ -27,8 +27,10 @@
 //               exp2 (part on the MUFU unit, part as a polynomial on the FMA
 //               pipe), packed f32x2 sums, P as bf16 into TMEM; at the end
 //               O / l through shared memory to a TMA store, plus the LSE.
-//   TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,320) O1 [320,384)
-//               P0 [384,448) P1 [448,512).
+//   TMEM (512 columns): three S buffers [0,128) [128,256) [256,384) taken
+//               in turn by the (tile, warpgroup) sequence, each tile's P
+//               written as bf16 over the first 64 columns of its own S
+//               buffer; O0 [384,448) O1 [448,512).
 // Launch modes (lc_fwd_mode): the whole sequence; the noisy queries with the
 // condition K/V from separate tensors (cache consumer); the condition queries
 // alone (cache producer); one shard pair of ring context parallelism (q / out
@@ -105,7 +107,7 @@ constexpr uint32_t kPolyMask = LC_POLY_EXP2_MASK;
 // exp pass shape: pairs in flight between ex2 and their use (kLag <= kRing),
 // and whether all logits are formed before the ex2 stream starts.
 #ifndef LC_PASS_LAG
-#define LC_PASS_LAG 4
+#define LC_PASS_LAG 2
 #endif
 #ifndef LC_LOGITS_FIRST
 #define LC_LOGITS_FIRST 1

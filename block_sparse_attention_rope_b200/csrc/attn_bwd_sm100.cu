@@ -57,8 +57,11 @@ constexpr int kWarpMma = 9;
 constexpr int kWarpRope = 10;     // and 11
 constexpr int kRopeThreads = 64;
 constexpr int kWarpDq = 12;       // 12-15
+// Q' / dO stages: with three, a stage's reload is issued a whole step
+// before the S^T / dP^T MMAs that read it (with two, the MMA issuer waited
+// for the load after every step).
 #ifndef LC_BWD_Q_STAGES
-#define LC_BWD_Q_STAGES 2
+#define LC_BWD_Q_STAGES 3
 #endif
 constexpr int kQStages = LC_BWD_Q_STAGES;
 constexpr int kTileBytes = 128 * 128;  // 128 rows x 64 bf16
@@ -97,7 +100,8 @@ struct __align__(64) BwdParams {
   long long timeout_ns;
   lc_divmod div_hw, div_w;
   int T, H, W;
-  int Nc, Nn, Cb, kgc, heads, KG, total_items, tab_floats;
+  int Nc, Nn, Cb, kgc, heads, KG, total_items;
+  int tab_floats;  // RoPE table floats copied to shared memory (0: read from global memory)
   int n_blocks;   // query / key blocks of the pattern (valid block ids: [0, n_blocks))
   int ent_cap;    // entries kg_ent holds (valid list bounds: [0, ent_cap])
   float scale;
@@ -111,11 +115,11 @@ struct SmemOffsets {
   static constexpr int ds = g + kQStages * kTileBytes;         // dS^T, two 64-query tiles
   static constexpr int dq = ds + 2 * kTileBytes;               // dQ' staging: [block][half] 64 x 32 fp32
   static constexpr int lse = dq + 2 * kTileBytes;              // [kQStages][128] lse * log2e
-  static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] D
+  static constexpr int del = lse + kQStages * 128 * 4;         // [kQStages][128] scale * D
   static constexpr int bars = del + kQStages * 128 * 4;
   static constexpr int n_bars = 48;
   static constexpr int misc = bars + n_bars * 8;
-  static constexpr int tab = misc + 64;
+  static constexpr int tab = misc + 64;  // the RoPE table, when it fits
 };
 
 enum {
@@ -228,7 +232,7 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-// cos / sin of pair p (0..31) at token n.
+// cos / sin of pair p (0..31) at token n (the table in shared or global memory).
 __device__ __forceinline__ void pair_angle(const BwdParams &a, const float *tab, int n, int p,
                                            float &c, float &s) {
   const int t = lc_div(n, a.div_hw);
@@ -265,7 +269,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   float *sDel = reinterpret_cast<float *>(smem + SmemOffsets::del);
   uint32_t *misc = reinterpret_cast<uint32_t *>(smem + SmemOffsets::misc);
   // misc[0] tmem base, misc[1..2] scheduled items, misc[3] abort flag
-  float *tab = reinterpret_cast<float *>(smem + SmemOffsets::tab);
+  float *stab = reinterpret_cast<float *>(smem + SmemOffsets::tab);
+  const float *tab = p.tab_floats ? stab : p.rope_tab;
   Ctx ctx;
   ctx.bar0 = lcptx::smem_addr(smem + SmemOffsets::bars);
   ctx.abort_flag = reinterpret_cast<volatile int *>(&misc[3]);
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
   ctx.timeout_ns = p.timeout_ns;
   const long long N = (long long)p.Nc + p.Nn;
 
-  for (int i = tid; i < p.tab_floats; i += kThreads) tab[i] = p.rope_tab[i];
+  for (int i = tid; i < p.tab_floats; i += kThreads) stab[i] = p.rope_tab[i];
   if (tid == 0) {
     misc[3] = 0;
     for (int i = 0; i < 2; ++i) {
@@ -521,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             if (rt < qn) {
               const int tok = (qs ? p.Nc : 0) + qr + rt;
               l2r[i] = __ldg(lse_bh + tok) * kLog2e;
-              dlr[i] = __ldg(del_bh + tok);
+              dlr[i] = __ldg(del_bh + tok) * p.scale;
             }
           }
         }
@@ -563,6 +568,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
       for (int t = 0; t < nsteps; ++t, ++dq_step) {
+        // the step's two list entries (reduce-add coordinates), loaded while
+        // the step's dQ is computed
+        uint32_t ents[2] = {0u, 0u};
+        if (qrow == 0) {
+#pragma unroll
+          for (int blk = 0; blk < 2; ++blk)
+            if (2 * t + blk < it.len) ents[blk] = __ldg(it.ent + 2 * t + blk);
+        }
         ok = wait_warp(ctx, ctx.bar(B_DQ_FULL), dq_ph);
         if (!ok) break;
         dq_ph ^= 1;
@@ -595,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             for (int blk = 0; blk < 2; ++blk) {
               const int e = 2 * t + blk;
               if (e >= it.len) continue;
-              const uint32_t ent = __ldg(it.ent + e);
+              const uint32_t ent = ents[blk];
               if (!qentry_ok(p, ent)) {
                 atomicOr(p.status, LC_DEVSTAT_CHECK);
                 continue;
@@ -645,18 +658,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const bool key_valid = (kr >> 6) < it.cnt && it.krow(kr >> 6) + (kr & 63) < it.seg_len;
       const int nsteps = (it.len + 1) >> 1;
       bool ok = true;
+      // This warp's list entry for the step: fetched one step ahead, so the
+      // load's latency hides behind the previous step (0 = no query block).
+      uint32_t ent_next = key_valid && half < it.len ? __ldg(it.ent + half) : 0u;
       for (int t = 0; t < nsteps; ++t, ++q_it) {
         const int s = q_it % kQStages;
+        const uint32_t ent = ent_next;
+        const int e_next = 2 * (t + 1) + half;
+        ent_next = key_valid && e_next < it.len ? __ldg(it.ent + e_next) : 0u;
         // attended query tokens of this warp's query block, for this key row
+        // (an entry failing the plan check only yields a mask here; the
+        // producer flags it)
         int lim = 0;
-        const int e = 2 * t + half;
-        if (key_valid && e < it.len) {  // (an entry failing the plan check only
-          const uint32_t ent = __ldg(it.ent + e);  // yields a mask here; the producer flags it)
-          if ((ent >> (24 + (kr >> 6))) & 1u) {
-            int qs, qr, qn;
-            qblock(p, ent, qs, qr, qn);
-            lim = qn;
-          }
+        if ((ent >> (24 + (kr >> 6))) & 1u) {
+          int qs, qr, qn;
+          qblock(p, ent, qs, qr, qn);
+          lim = qn;
         }
         // the staged lse / D of this step (written by the RoPE warps), then S^T, dP^T
         ok = wait_warp(ctx, ctx.bar(B_QG_READY + s), (q_it / kQStages) & 1) &&
@@ -669,9 +686,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         // 16 queries at a time; the next chunk's TMEM loads are in flight while
         // this one is computed (double buffer)
         uint32_t sr[2][16], dr[2][16];
-        // the whole row's P^T and dS^T, packed, before the waits for their
-        // space (the previous step's dV, then its dK / dQ)
-        uint32_t pk[4][8], dk[4][8];
+        // P^T goes to TMEM chunk by chunk (after the wait for the previous
+        // step's dV, which lands during the first chunk); dS^T of the whole
+        // row is held, packed, until the previous step's dK / dQ are done
+        // with the tile
+        uint32_t dk[4][8];
         lcptx::tmem_ld16(tST + 64 * half, sr[0]);
         lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
         lcptx::tmem_wait_ld();
@@ -689,30 +708,34 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
           const uint32_t(&scur)[16] = sr[k & 1];
           const uint32_t(&dcur)[16] = dr[k & 1];
           const int jb = k * 16;  // first query of the chunk within its block
+          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
+              // P = 2^(log2e (scale S - lse)); dS = P * (scale dP - scale D)
               const int j = 16 * c + 2 * i + u;
               const bool on = jb + 2 * i + u < lim;
               const float pe = on ? ex2(__uint_as_float(scur[2 * i + u]) * sl2 - l2[j]) : 0.f;
               pv[u] = pe;
-              dv2[u] = pe * (__uint_as_float(dcur[2 * i + u]) - dl[j]) * p.scale;
+              dv2[u] = pe * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dl[j]);
             }
-            pk[k][i] = pack_bf16(pv[0], pv[1]);
+            pk[i] = pack_bf16(pv[0], pv[1]);
             dk[k][i] = pack_bf16(dv2[0], dv2[1]);
           }
+          if (k == 0 && q_it > 0) {  // the previous step's dV is done with the P^T columns
+            ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
+            lcptx::tc_fence_after();
+          }
+          // P^T row kr, this block's queries 16k .. 16k + 15: TMEM columns 32 * half + 8k ..
+          if (ok) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk);
           if (k < 3) lcptx::tmem_wait_ld();
         }
-        // P^T row kr, this block's 64 queries: TMEM columns 32 * half .. + 31
-        if (q_it > 0) {
-          ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
-          if (!ok) break;
-          lcptx::tc_fence_after();
+        if (!ok) {
+          lcptx::tmem_wait_st();
+          break;
         }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk[k]);
         if (q_it > 0) {  // the previous step's dK / dQ are done with the dS^T tiles
           ok = wait_warp(ctx, ctx.bar(B_STEP), (q_it - 1) & 1);
           if (!ok) {
@@ -810,8 +833,11 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
   const long long total = (long long)batch * heads * plan->KG;
   if (total == 0) return LC_OK;
   if (total >= (1LL << 31)) return LC_ERR_UNSUPPORTED;
-  const size_t smem = 1024 + SmemOffsets::tab + sizeof(float) * (size_t)rope->n_floats;
-  if (smem > 227 * 1024) return LC_ERR_UNSUPPORTED;
+  // the RoPE table goes to shared memory when it fits beside the tiles
+  static_assert(1024 + SmemOffsets::tab <= 227 * 1024, "shared memory");
+  const size_t tab_bytes = sizeof(float) * (size_t)rope->n_floats;
+  const bool tab_in_smem = 1024 + SmemOffsets::tab + tab_bytes <= 227 * 1024;
+  const size_t smem = 1024 + SmemOffsets::tab + (tab_in_smem ? tab_bytes : 0);
   lc_status s = LC_OK;
   prm.status = lc_device_status_ptr(&s);
   if (s != LC_OK) return s;
@@ -893,7 +919,7 @@ lc_status lc_launch_backward_sm100(const void *q, const void *k, const void *v, 
     prm.n_blocks = plan->Cb + plan->Nb;
     prm.ent_cap = (int)plan->nnz;
     prm.total_items = (int)total;
-    prm.tab_floats = (int)rope->n_floats;
+    prm.tab_floats = tab_in_smem ? (int)rope->n_floats : 0;
     prm.scale = scale;
     const int grid = (int)(total < n_sm ? total : n_sm);
     kern<<<grid, kThreads, smem, stream>>>(prm);

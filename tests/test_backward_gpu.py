@@ -33,6 +33,10 @@ CASES = {
                             dtype="bf16"),
     "tiny_tokens": Workload("tiny_tokens", T=5, H=1, W=7, n_cond=2, heads=2, local=0, stride=3,
                             dtype="bf16"),
+    # a grid whose RoPE table (16 T + 24 H + 24 W floats) does not fit in the
+    # tensor-core kernel's shared memory beside its tiles: read from global memory
+    "wide_grid": Workload("wide_grid", T=2, H=1, W=330, n_cond=0, heads=2, local=1, stride=2,
+                          dtype="bf16"),
 }
 
 

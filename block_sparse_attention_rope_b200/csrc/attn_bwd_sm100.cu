@@ -712,14 +712,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float pv[2], dv2[2];
+            // log2e * lse and scale * D of queries 2i, 2i + 1 of the chunk
+            // (16-byte shared loads, one per four queries)
+            const float4 l4 = reinterpret_cast<const float4 *>(l2 + 16 * c)[i >> 1];
+            const float4 d4 = reinterpret_cast<const float4 *>(dl + 16 * c)[i >> 1];
+            const float lq[2] = {(i & 1) ? l4.z : l4.x, (i & 1) ? l4.w : l4.y};
+            const float dq[2] = {(i & 1) ? d4.z : d4.x, (i & 1) ? d4.w : d4.y};
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
               // P = 2^(log2e (scale S - lse)); dS = P * (scale dP - scale D)
-              const int j = 16 * c + 2 * i + u;
               const bool on = jb + 2 * i + u < lim;
-              const float pe = on ? ex2(__uint_as_float(scur[2 * i + u]) * sl2 - l2[j]) : 0.f;
+              const float pe = on ? ex2(__uint_as_float(scur[2 * i + u]) * sl2 - lq[u]) : 0.f;
               pv[u] = pe;
-              dv2[u] = pe * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dl[j]);
+              dv2[u] = pe * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dq[u]);
             }
             pk[i] = pack_bf16(pv[0], pv[1]);
             dk[k][i] = pack_bf16(dv2[0], dv2[1]);

@@ -13,13 +13,14 @@
 //               step.
 //   per step, with keys as TMEM lanes (M = 128):
 //     S^T  = K' Q'^T        dP^T = V dO^T          (tcgen05, into TMEM)
-//     P^T  = exp(scale S^T - lse),  dS^T = P^T (dP^T - D) scale
+//     P^T  = exp(scale S^T - lse),  dS^T = P^T (scale dP^T - scale D)
 //                           (warps 0-7, one key row and query block per
-//                            thread, the whole row formed before the waits
-//                            for the previous step's MMAs; P^T written as
-//                            bf16 pairs into TMEM, dS^T as bf16 tiles into
-//                            shared memory, so the next step's S^T, dP^T can
-//                            be computed while they are formed)
+//                            thread; P^T written as bf16 pairs into TMEM 16
+//                            queries at a time, dS^T held for the row until
+//                            the previous step's dK / dQ are done, then
+//                            written as bf16 tiles into shared memory, so the
+//                            next step's S^T, dP^T can be computed while they
+//                            are formed)
 //     dV  += P^T dO         (A = P^T from TMEM, only dO read from shared memory)
 //     dK' += dS^T Q'        (A from shared memory)
 //     dQ'  = dS K'          (A = dS from shared memory, MN-major; queries as
@@ -27,7 +28,8 @@
 //                            12-15 and added to the fp32 buffer by TMA
 //                            reduce-adds
 //   item end: dK = R^T dK' (and the RMSNorm transpose), dK and dV stored.
-//   warp 8: TMA producer (K', V per item; Q', dO per step, 2 stages); warp 9: MMA issuer; warps 10-11: stage lse / D per step.
+//   warp 8: TMA producer (K', V per item; Q', dO per step, 3 stages); warp 9:
+//   MMA issuer; warps 10-11: stage log2e * lse and scale * D per step.
 //   Q' = R(norm(q)) and K' = R(norm(k)) are formed once, before the kernel,
 //   by the one-pass rotation the forward uses for K (same arithmetic).
 //   TMEM: S^T [0,128) dP^T [128,256) dV [256,320) dK [320,384) dQ [384,448)

@@ -515,12 +515,15 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       const float *del_bh = p.delta + ((long long)it.b * p.heads + it.h) * N;
       for (int t = 0; t < nsteps && ok; ++t, ++q_it) {
         const int s = q_it % kQStages;
-        // This thread's two query rows (rt of each query block): lse and D of
-        // their tokens (0 for rows that do not exist; they are masked).
+        // This thread's two query rows (rt of each query block): log2e * lse
+        // and scale * D of their tokens.  A row that does not exist (past a
+        // block's last token, an absent block, an entry failing the plan
+        // check) gets lse = +inf, so its P is exactly 0 in every key row.
         float l2r[2], dlr[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          l2r[i] = dlr[i] = 0.f;
+          l2r[i] = __int_as_float(0x7f800000);
+          dlr[i] = 0.f;
           const int e = 2 * t + i;
           if (e < it.len && qentry_ok(p, __ldg(it.ent + e))) {
             int qs, qr, qn;
@@ -662,21 +665,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
       bool ok = true;
       // This warp's list entry for the step: fetched one step ahead, so the
       // load's latency hides behind the previous step (0 = no query block).
-      uint32_t ent_next = key_valid && half < it.len ? __ldg(it.ent + half) : 0u;
+      uint32_t ent_next = half < it.len ? __ldg(it.ent + half) : 0u;
       for (int t = 0; t < nsteps; ++t, ++q_it) {
         const int s = q_it % kQStages;
         const uint32_t ent = ent_next;
         const int e_next = 2 * (t + 1) + half;
-        ent_next = key_valid && e_next < it.len ? __ldg(it.ent + e_next) : 0u;
-        // attended query tokens of this warp's query block, for this key row
-        // (an entry failing the plan check only yields a mask here; the
-        // producer flags it)
-        int lim = 0;
-        if ((ent >> (24 + (kr >> 6))) & 1u) {
-          int qs, qr, qn;
-          qblock(p, ent, qs, qr, qn);
-          lim = qn;
-        }
+        ent_next = e_next < it.len ? __ldg(it.ent + e_next) : 0u;
+        // Does this warp's key block attend the step's query block?  The same
+        // answer for all the warp's rows (one key block, one list entry), so
+        // the branch below is uniform.  Within an attending block every pair
+        // is attended: the query tokens a block lacks have lse = +inf; key
+        // rows past a segment's end meet zero K' / V rows (their P, clamped
+        // at 1, reaches no stored gradient).
+        const bool member = ((ent >> (24 + (kr >> 6))) & 1u) != 0;
         // the staged lse / D of this step (written by the RoPE warps), then S^T, dP^T
         ok = wait_warp(ctx, ctx.bar(B_QG_READY + s), (q_it / kQStages) & 1) &&
              wait_warp(ctx, ctx.bar(B_SDP), sdp_ph);
@@ -685,59 +686,75 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
         lcptx::tc_fence_after();
         const float *l2 = sLse + s * 128, *dl = sDel + s * 128;
         uint8_t *tile = sDS + half * kTileBytes;  // dS^T, this query block's MN-major chunk
-        // 16 queries at a time; the next chunk's TMEM loads are in flight while
-        // this one is computed (double buffer)
-        uint32_t sr[2][16], dr[2][16];
         // P^T goes to TMEM chunk by chunk (after the wait for the previous
         // step's dV, which lands during the first chunk); dS^T of the whole
         // row is held, packed, until the previous step's dK / dQ are done
         // with the tile
         uint32_t dk[4][8];
-        lcptx::tmem_ld16(tST + 64 * half, sr[0]);
-        lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
-        lcptx::tmem_wait_ld();
+        if (member) {
+          // 16 queries at a time; the next chunk's TMEM loads are in flight
+          // while this one is computed (double buffer)
+          uint32_t sr[2][16], dr[2][16];
+          lcptx::tmem_ld16(tST + 64 * half, sr[0]);
+          lcptx::tmem_ld16(tDPT + 64 * half, dr[0]);
+          lcptx::tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int c = 4 * half + k;
-          if (k < 3) {
-            lcptx::tmem_ld16(tST + 64 * half + 16 * (k + 1), sr[(k + 1) & 1]);
-            lcptx::tmem_ld16(tDPT + 64 * half + 16 * (k + 1), dr[(k + 1) & 1]);
-          } else {  // every TMEM load of the step has landed: S^T, dP^T may be overwritten
-            lcptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_ST_FREE));
-          }
-          const uint32_t(&scur)[16] = sr[k & 1];
-          const uint32_t(&dcur)[16] = dr[k & 1];
-          const int jb = k * 16;  // first query of the chunk within its block
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float pv[2], dv2[2];
-            // log2e * lse and scale * D of queries 2i, 2i + 1 of the chunk
-            // (16-byte shared loads, one per four queries)
-            const float4 l4 = reinterpret_cast<const float4 *>(l2 + 16 * c)[i >> 1];
-            const float4 d4 = reinterpret_cast<const float4 *>(dl + 16 * c)[i >> 1];
-            const float lq[2] = {(i & 1) ? l4.z : l4.x, (i & 1) ? l4.w : l4.y};
-            const float dq[2] = {(i & 1) ? d4.z : d4.x, (i & 1) ? d4.w : d4.y};
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              // P = 2^(log2e (scale S - lse)); dS = P * (scale dP - scale D)
-              const bool on = jb + 2 * i + u < lim;
-              const float pe = on ? ex2(__uint_as_float(scur[2 * i + u]) * sl2 - lq[u]) : 0.f;
-              pv[u] = pe;
-              dv2[u] = pe * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dq[u]);
+          for (int k = 0; k < 4; ++k) {
+            const int c = 4 * half + k;
+            if (k < 3) {
+              lcptx::tmem_ld16(tST + 64 * half + 16 * (k + 1), sr[(k + 1) & 1]);
+              lcptx::tmem_ld16(tDPT + 64 * half + 16 * (k + 1), dr[(k + 1) & 1]);
+            } else {  // every TMEM load of the step has landed: S^T, dP^T may be overwritten
+              lcptx::tc_fence_before();
+              __syncwarp();
+              if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_ST_FREE));
             }
-            pk[i] = pack_bf16(pv[0], pv[1]);
-            dk[k][i] = pack_bf16(dv2[0], dv2[1]);
+            const uint32_t(&scur)[16] = sr[k & 1];
+            const uint32_t(&dcur)[16] = dr[k & 1];
+            uint32_t pk[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float pv[2], dv2[2];
+              // log2e * lse and scale * D of queries 2i, 2i + 1 of the chunk
+              // (16-byte shared loads, one per four queries)
+              const float4 l4 = reinterpret_cast<const float4 *>(l2 + 16 * c)[i >> 1];
+              const float4 d4 = reinterpret_cast<const float4 *>(dl + 16 * c)[i >> 1];
+              const float lq[2] = {(i & 1) ? l4.z : l4.x, (i & 1) ? l4.w : l4.y};
+              const float dq[2] = {(i & 1) ? d4.z : d4.x, (i & 1) ? d4.w : d4.y};
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                // P = 2^(log2e (scale S - lse)) <= 1; dS = P * (scale dP - scale D)
+                pv[u] = ex2(fminf(fmaf(__uint_as_float(scur[2 * i + u]), sl2, -lq[u]), 0.f));
+                dv2[u] = pv[u] * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dq[u]);
+              }
+              pk[i] = pack_bf16(pv[0], pv[1]);
+              dk[k][i] = pack_bf16(dv2[0], dv2[1]);
+            }
+            if (k == 0 && q_it > 0) {  // the previous step's dV is done with the P^T columns
+              ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
+              lcptx::tc_fence_after();
+            }
+            // P^T row kr, this block's queries 16k .. 16k + 15: TMEM columns 32 * half + 8k ..
+            if (ok) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk);
+            if (k < 3) lcptx::tmem_wait_ld();
           }
-          if (k == 0 && q_it > 0) {  // the previous step's dV is done with the P^T columns
+        } else {
+          // no pair of this key block and query block is attended: P^T and
+          // dS^T are zero, and S^T / dP^T need not be read
+          lcptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) lcptx::mbar_arrive(ctx.bar(B_ST_FREE));
+          if (q_it > 0) {
             ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);
             lcptx::tc_fence_after();
           }
-          // P^T row kr, this block's queries 16k .. 16k + 15: TMEM columns 32 * half + 8k ..
-          if (ok) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, pk);
-          if (k < 3) lcptx::tmem_wait_ld();
+          const uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if (ok) lcptx::tmem_st8(tmem + lane_base + kColPT + 32 * half + 8 * k, zero);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dk[k][i] = 0u;
+          }
         }
         if (!ok) {
           lcptx::tmem_wait_st();

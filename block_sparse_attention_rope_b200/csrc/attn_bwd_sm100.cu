@@ -651,6 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tST = tmem + lane_base + kColST, tDPT = tmem + lane_base + kColDPT;
     const float sl2 = p.scale * kLog2e;
+    const float2 sl2x2 = make_float2(sl2, sl2), scx2 = make_float2(p.scale, p.scale);
     uint32_t item_it = 0, q_it = 0, sdp_ph = 0;
     for (;;) {
       const int slot = item_it & 1;
@@ -714,21 +715,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_sm100_kernel(const __grid
             uint32_t pk[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              float pv[2], dv2[2];
               // log2e * lse and scale * D of queries 2i, 2i + 1 of the chunk
               // (16-byte shared loads, one per four queries)
               const float4 l4 = reinterpret_cast<const float4 *>(l2 + 16 * c)[i >> 1];
               const float4 d4 = reinterpret_cast<const float4 *>(dl + 16 * c)[i >> 1];
-              const float lq[2] = {(i & 1) ? l4.z : l4.x, (i & 1) ? l4.w : l4.y};
-              const float dq[2] = {(i & 1) ? d4.z : d4.x, (i & 1) ? d4.w : d4.y};
-#pragma unroll
-              for (int u = 0; u < 2; ++u) {
-                // P = 2^(log2e (scale S - lse)) <= 1; dS = P * (scale dP - scale D)
-                pv[u] = ex2(fminf(fmaf(__uint_as_float(scur[2 * i + u]), sl2, -lq[u]), 0.f));
-                dv2[u] = pv[u] * fmaf(__uint_as_float(dcur[2 * i + u]), p.scale, -dq[u]);
-              }
-              pk[i] = pack_bf16(pv[0], pv[1]);
-              dk[k][i] = pack_bf16(dv2[0], dv2[1]);
+              const float2 nlq = (i & 1) ? make_float2(-l4.z, -l4.w) : make_float2(-l4.x, -l4.y);
+              const float2 ndq = (i & 1) ? make_float2(-d4.z, -d4.w) : make_float2(-d4.x, -d4.y);
+              // P = 2^(log2e (scale S - lse)) <= 1; dS = P * (scale dP - scale D),
+              // two queries per packed fp32 instruction
+              const float2 x = __ffma2_rn(
+                  make_float2(__uint_as_float(scur[2 * i]), __uint_as_float(scur[2 * i + 1])), sl2x2, nlq);
+              const float2 pv = make_float2(ex2(fminf(x.x, 0.f)), ex2(fminf(x.y, 0.f)));
+              const float2 g = __ffma2_rn(
+                  make_float2(__uint_as_float(dcur[2 * i]), __uint_as_float(dcur[2 * i + 1])), scx2, ndq);
+              const float2 dv2 = __fmul2_rn(pv, g);
+              pk[i] = pack_bf16(pv.x, pv.y);
+              dk[k][i] = pack_bf16(dv2.x, dv2.y);
             }
             if (k == 0 && q_it > 0) {  // the previous step's dV is done with the P^T columns
               ok = wait_warp(ctx, ctx.bar(B_PT_FREE), (q_it - 1) & 1);

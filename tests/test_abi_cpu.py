@@ -94,6 +94,51 @@ def test_forward_rejects_null_handles(lib):
     assert g(None, None, None, None, None, None, None, 1, 2, 64, 0, 0.0, None, None, None) == 1
 
 
+def test_other_entry_points_reject_bad_arguments_before_any_gpu_work(lib):
+    """The _ex forwards, the cache producer, the backward, the allocation-free
+    forward and the plan / table accessors return LC_ERR_INVALID_ARGUMENT for
+    NULL tensors, handles or outputs (and for bad options) on a machine
+    without a GPU: none of them reaches a CUDA call first."""
+    vp, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+
+    class Opts(ctypes.Structure):
+        _fields_ = [("flags", ctypes.c_uint), ("q_norm_weight", vp), ("k_norm_weight", vp),
+                    ("norm_eps", F)]
+
+    bad_flags = Opts(flags=64)
+    bad_eps = Opts(flags=0, norm_eps=-1.0)
+    f = lib.lc_bsa_forward_ex
+    f.argtypes = [vp] * 5 + [I] * 4 + [F] + [vp] * 4
+    g = lib.lc_bsa_forward_cached_ex
+    g.argtypes = [vp] * 7 + [I] * 4 + [F] + [vp] * 4
+    c = lib.lc_bsa_cond_cache
+    c.argtypes = [vp] * 6 + [I] * 4 + [F] + [vp] * 4
+    b = lib.lc_bsa_backward
+    b.argtypes = [vp] * 9 + [I] * 4 + [F] + [vp] * 4
+    for opts in (None, ctypes.byref(bad_flags), ctypes.byref(bad_eps)):
+        assert f(None, None, None, None, None, 1, 2, 64, 0, 0.0, opts, None, None, None) == 1
+        assert g(*[None] * 7, 1, 2, 64, 0, 0.0, opts, None, None, None) == 1
+        assert c(*[None] * 6, 1, 2, 64, 0, 0.0, opts, None, None, None) == 1
+        assert b(*[None] * 9, 1, 2, 64, 0, 0.0, opts, None, None, None) == 1
+    n = lib.lc_bsa_forward_noalloc
+    n.argtypes = [vp] * 5 + [I] * 4 + [F] + [vp] * 3
+    assert n(None, None, None, None, None, 1, 2, 64, 0, 0.0, None, None, None) == 1
+    for name, nargs in (("lc_bsa_plan_info", 2), ("lc_bsa_plan_copy_csc", 4),
+                        ("lc_bsa_plan_copy_csr", 4), ("lc_bsa_plan_token_range", 5),
+                        ("lc_rope3d_copy_tables", 3)):
+        fn = getattr(lib, name)
+        fn.argtypes = [vp] * nargs
+        assert fn(*[None] * nargs) == 1, name
+    s = lib.lc_debug_scratch_pool_used_high
+    s.argtypes = [vp, I]
+    assert s(None, 0) == 1
+    # destroying a NULL handle is a no-op
+    for name in ("lc_bsa_plan_destroy", "lc_rope3d_destroy"):
+        fn = getattr(lib, name)
+        fn.argtypes = [vp, vp]
+        assert fn(None, None) == 0, name
+
+
 def test_python_binding_imports_only_the_library():
     """The binding module must not reach the oracle (no CPU fallback)."""
     src = open(os.path.join(ROOT, "block_sparse_attention_rope_b200", "api.py")).read()
